@@ -1,0 +1,209 @@
+"""CPU oracle for the block-scaled FP8 linear and its M-grouped contiguous variant.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package.  The product path (the CUDA
+library and its Python binding) never imports, links or runs anything here, and
+this package never imports the product.
+
+The arithmetic lives in ``lnq_oracle.c`` (plain C, FP64 accumulation, IEEE
+single-precision division for the scales and quotients); this module only builds
+it with gcc and marshals numpy arrays.  Every function cites the page passage it
+follows in the C source.  Pins against the pages and the mathematics live in
+``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lnq_oracle.c")
+_LIB = os.path.join(_HERE, "liblnq_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+GROUP = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (OpenMP, no FMA contraction, no fast-math)."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    cmd = [
+        "gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+        "-fPIC", "-shared", "-Wall", "-o", tmp, _SRC, "-lm",
+    ]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode_array.argtypes = [P, I64, P]
+        lib.oracle_e4m3_value_array.argtypes = [P, I64, P]
+        lib.oracle_quantize_fp8_groups.restype = ctypes.c_int
+        lib.oracle_quantize_fp8_groups.argtypes = [P, I64, I64, I64, P, I64, P, I64]
+        lib.oracle_quantize_fp8_blocks.restype = ctypes.c_int
+        lib.oracle_quantize_fp8_blocks.argtypes = [P, I64, I64, P, P]
+        lib.oracle_gemm_nt.restype = ctypes.c_int
+        lib.oracle_gemm_nt.argtypes = [P, P, I64, P, P, I64, I64, I64, P]
+        lib.oracle_gemm_nt_points.restype = ctypes.c_int
+        lib.oracle_gemm_nt_points.argtypes = [P, P, I64, P, P, I64, I64, I64, P, P, I64, P]
+        lib.oracle_m_grouped_gemm_contiguous.restype = ctypes.c_int
+        lib.oracle_m_grouped_gemm_contiguous.argtypes = [P, P, P, P, P, ctypes.c_int32, I64, I64, I64, P]
+        lib.oracle_m_grouped_gemm_points.restype = ctypes.c_int
+        lib.oracle_m_grouped_gemm_points.argtypes = [
+            P, P, P, P, P, ctypes.c_int32, I64, I64, I64, P, P, I64, P]
+        _lib = lib
+        return lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype) -> np.ndarray:
+    a = np.asarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {np.dtype(dtype)}, got {a.dtype}")
+    return np.ascontiguousarray(a)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (rc={rc})")
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use."""
+    return int(_load().oracle_num_threads())
+
+
+def ceil4(m: int) -> int:
+    return -(-m // 4) * 4
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """Exact value (float64) of each E4M3 code; NaN for 0x7F / 0xFF."""
+    c = _c(np.asarray(codes, dtype=np.uint8), np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    _load().oracle_e4m3_value_array(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def e4m3_encode(t) -> np.ndarray:
+    """E4M3 code of each float32 value: RNE, ties to even, saturating at 448."""
+    a = _c(np.asarray(t, dtype=np.float32), np.float32)
+    out = np.empty(a.shape, dtype=np.uint8)
+    _load().oracle_e4m3_encode_array(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def quantize_fp8_groups(x_bf16_bits: np.ndarray, M4: int | None = None):
+    """1x128 activation quantization of a bf16 matrix given as uint16 bits [M, K].
+
+    Returns (q uint8 [M, K], sfa float32 [K/128, M4]) with M4 = ceil4(M) unless given.
+    """
+    x = _c(x_bf16_bits, np.uint16)
+    M, K = x.shape
+    M4 = ceil4(M) if M4 is None else int(M4)
+    q = np.empty((M, K), dtype=np.uint8)
+    sfa = np.empty((K // GROUP, M4), dtype=np.float32)
+    _check(_load().oracle_quantize_fp8_groups(_ptr(x), M, K, K, _ptr(q), K, _ptr(sfa), M4),
+           "quantize_fp8_groups")
+    return q, sfa
+
+
+def quantize_fp8_blocks(w_bf16_bits: np.ndarray):
+    """128x128 weight quantization of a bf16 matrix given as uint16 bits [N, K].
+
+    Returns (q uint8 [N, K], sfb float32 [ceil(N/128), K/128]).
+    """
+    w = _c(w_bf16_bits, np.uint16)
+    N, K = w.shape
+    q = np.empty((N, K), dtype=np.uint8)
+    sfb = np.empty((-(-N // GROUP), K // GROUP), dtype=np.float32)
+    _check(_load().oracle_quantize_fp8_blocks(_ptr(w), N, K, _ptr(q), _ptr(sfb)),
+           "quantize_fp8_blocks")
+    return q, sfb
+
+
+def gemm_nt(qa, sfa, qb, sfb, M: int | None = None) -> np.ndarray:
+    """FP64 D [M, N] of the dequantized operands (qa [M, K], qb [N, K])."""
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    sfa = _c(sfa, np.float32)
+    sfb = _c(sfb, np.float32)
+    M = qa.shape[0] if M is None else M
+    K = qa.shape[1]
+    N = qb.shape[0]
+    D = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_gemm_nt(_ptr(qa), _ptr(sfa), sfa.shape[1], _ptr(qb), _ptr(sfb),
+                                  M, N, K, _ptr(D)), "gemm_nt")
+    return D
+
+
+def gemm_nt_points(qa, sfa, qb, sfb, rows, cols) -> np.ndarray:
+    """FP64 D at the points (rows[i], cols[i])."""
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    sfa = _c(sfa, np.float32)
+    sfb = _c(sfb, np.float32)
+    rows = _c(np.asarray(rows, dtype=np.int64), np.int64)
+    cols = _c(np.asarray(cols, dtype=np.int64), np.int64)
+    out = np.empty(rows.shape, dtype=np.float64)
+    _check(_load().oracle_gemm_nt_points(_ptr(qa), _ptr(sfa), sfa.shape[1], _ptr(qb), _ptr(sfb),
+                                         qa.shape[0], qb.shape[0], qa.shape[1], _ptr(rows),
+                                         _ptr(cols), rows.size, _ptr(out)), "gemm_nt_points")
+    return out
+
+
+def m_grouped_gemm_contiguous(qa, sfa, qb, sfb, m_indices, num_groups: int) -> np.ndarray:
+    """FP64 D [M_total, N]; rows with a negative group id are NaN."""
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    sfa = _c(sfa, np.float32)
+    sfb = _c(sfb, np.float32)
+    mi = _c(np.asarray(m_indices, dtype=np.int32), np.int32)
+    M_total, K = qa.shape
+    N = qb.shape[0] // num_groups
+    D = np.full((M_total, N), np.nan, dtype=np.float64)
+    _check(_load().oracle_m_grouped_gemm_contiguous(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb),
+                                                    _ptr(mi), num_groups, M_total, N, K, _ptr(D)),
+           "m_grouped_gemm_contiguous")
+    return D
+
+
+def m_grouped_gemm_points(qa, sfa, qb, sfb, m_indices, num_groups: int, rows, cols) -> np.ndarray:
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    sfa = _c(sfa, np.float32)
+    sfb = _c(sfb, np.float32)
+    mi = _c(np.asarray(m_indices, dtype=np.int32), np.int32)
+    rows = _c(np.asarray(rows, dtype=np.int64), np.int64)
+    cols = _c(np.asarray(cols, dtype=np.int64), np.int64)
+    M_total, K = qa.shape
+    N = qb.shape[0] // num_groups
+    out = np.empty(rows.shape, dtype=np.float64)
+    _check(_load().oracle_m_grouped_gemm_points(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(mi),
+                                                num_groups, M_total, N, K, _ptr(rows), _ptr(cols),
+                                                rows.size, _ptr(out)), "m_grouped_gemm_points")
+    return out
