@@ -1,0 +1,580 @@
+#!/usr/bin/env python
+"""Benchmark of the block-scaled FP8 linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill|decode|moe|square|tiny]
+
+One step is one pass of the hot path over one batch of synthetic input: for each
+linear of the workload, the 1x128 activation quantize (lnq_quantize_fp8_groups)
+and the block-scaled FP8 GEMM (lnq_fp8_block_gemm_nt, or the M-grouped
+contiguous GEMM for `moe`).  Weights are model parameters: quantized to
+128x128 blocks once, before timing (lnq_quantize_fp8_blocks).
+
+Default workload (`prefill`): the dense-transformer prefill linears at M = 2048
+tokens, K = 4096 -- QKV N=6144, O N=4096, gate_up N=24576, down K=12288 -> N=4096.
+A ~ N(0,1), W ~ N(0,0.02), bf16, seeded.  The step touches ~500 MB, more than
+the 126 MB L2, so no extra L2 flush is used between steps.
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (its own
+tokens, replicated weights); no collective is on the data path.  The timed
+region is bracketed by a barrier and a device synchronize on every rank; the
+reported time is the max over ranks (an all-reduce of one number).
+
+Output: one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "block-scaled FP8 GEMM TFLOP/s (and GB/s for decode) + % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+KERNEL_SOURCES = ["moe_grouped_gemm_quantize_b200/csrc/lnq_gemm.cuh",
+                  "moe_grouped_gemm_quantize_b200/csrc/lnq_ptx.cuh",
+                  "moe_grouped_gemm_quantize_b200/csrc/lnq_quantize.cuh",
+                  "moe_grouped_gemm_quantize_b200/csrc/lnq_api.cu"]
+
+
+# --------------------------------------------------------------------------- setup
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str = "nccl"):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank number over all ranks (identity on one process)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    e = rec.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self._nv = None
+            self.error = f"nvml unavailable: {e}"
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception as e:
+                self.error = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.error}
+        med = statistics.median(self.samples) if self.samples else None
+        out = {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+               "samples": len(self.samples)}
+        if self.error:
+            out["note"] = self.error
+        return out
+
+
+# --------------------------------------------------------------------------- workloads
+
+class Linear:
+    """One dense linear: bf16 activations resident on the device, weights pre-quantized."""
+
+    def __init__(self, cfg, dev):
+        import moe_grouped_gemm_quantize_b200 as lnq
+        from moe_grouped_gemm_quantize_b200 import synthetic
+        self.cfg = cfg
+        a, w = synthetic.make_linear_inputs(cfg)
+        self.x = a.to(dev)
+        self.wq, self.ws = lnq.quantize_weights(w.to(dev))
+        del w
+        M, N, K = cfg.M, cfg.N, cfg.K
+        self.M4 = lnq.ceil4(M)
+        self.q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev)
+        self.sfa = torch.empty((K // 128, self.M4), dtype=torch.float32, device=dev)
+        self.d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.flops = 2.0 * M * N * K
+        self.gemm_bytes = (M * K + 4 * (K // 128) * self.M4 + N * K
+                           + 4 * (-(-N // 128)) * (K // 128) + 2 * M * N)
+        self.quant_bytes = 2 * M * K + M * K + 4 * (K // 128) * self.M4
+        self.h2d_bytes = 2 * M * K
+        self.d2h_bytes = 2 * M * N
+        self.host_x = self.x.cpu().pin_memory()
+        self.host_d = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+
+    def calls(self, stream_ptr):
+        """Pre-marshalled C-ABI calls (quantize, gemm)."""
+        import ctypes
+        import moe_grouped_gemm_quantize_b200 as lnq
+        L = lnq.lib()
+        P = ctypes.c_void_p
+        c = self.cfg
+        s = P(stream_ptr)
+        qargs = (P(self.x.data_ptr()), c.M, c.K, self.x.stride(0), P(self.q.data_ptr()), c.K,
+                 P(self.sfa.data_ptr()), self.M4, s)
+        gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), self.M4, P(self.wq.data_ptr()),
+                 P(self.ws.data_ptr()), P(self.d.data_ptr()), c.M, c.N, c.K, s)
+        return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_fp8_block_gemm_nt, gargs)
+
+
+class Grouped:
+    """The M-grouped contiguous MoE GEMM: 16384 routed rows over 32 experts."""
+
+    def __init__(self, cfg, dev):
+        import moe_grouped_gemm_quantize_b200 as lnq
+        from moe_grouped_gemm_quantize_b200 import synthetic
+        self.cfg = cfg
+        a, w, m_indices, sizes = synthetic.make_moe_inputs(cfg)
+        self.M = a.shape[0]
+        self.x = a.to(dev)
+        self.wq, self.ws = lnq.quantize_weights(w.to(dev))
+        del w
+        self.mi = torch.from_numpy(m_indices).to(dev)
+        K, N, G = cfg.K, cfg.N, cfg.groups
+        self.q = torch.empty((self.M, K), dtype=torch.float8_e4m3fn, device=dev)
+        self.sfa = torch.empty((K // 128, self.M), dtype=torch.float32, device=dev)
+        self.d = torch.empty((self.M, N), dtype=torch.bfloat16, device=dev)
+        self.flops = cfg.flops   # real rows only
+        self.gemm_bytes = (self.M * K + 4 * (K // 128) * self.M + G * N * K
+                           + 4 * G * (-(-N // 128)) * (K // 128) + 2 * self.M * N + 4 * self.M)
+        self.quant_bytes = 3 * self.M * K + 4 * (K // 128) * self.M
+        self.h2d_bytes = 2 * self.M * K
+        self.d2h_bytes = 2 * self.M * N
+        self.host_x = self.x.cpu().pin_memory()
+        self.host_d = torch.empty((self.M, N), dtype=torch.bfloat16).pin_memory()
+
+    def calls(self, stream_ptr):
+        import ctypes
+        import moe_grouped_gemm_quantize_b200 as lnq
+        L = lnq.lib()
+        P = ctypes.c_void_p
+        c = self.cfg
+        s = P(stream_ptr)
+        qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K,
+                 P(self.sfa.data_ptr()), self.M, s)
+        gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), P(self.wq.data_ptr()),
+                 P(self.ws.data_ptr()), P(self.mi.data_ptr()), c.groups, P(self.d.data_ptr()),
+                 self.M, c.N, c.K, s)
+        return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_m_grouped_fp8_gemm_contiguous, gargs)
+
+
+def workload_units(name: str):
+    from moe_grouped_gemm_quantize_b200 import synthetic
+    if name == "prefill":
+        return list(synthetic.PREFILL), "linear"
+    if name == "decode":
+        return list(synthetic.DECODE), "linear"
+    if name == "square":
+        return [synthetic.SQUARE], "linear"
+    if name == "tiny":
+        return [synthetic.TINY], "linear"
+    if name == "moe":
+        return [synthetic.MOE], "grouped"
+    raise ValueError(name)
+
+
+WORKLOAD_DESC = {
+    "prefill": "prefill linears M=2048: QKV 6144x4096, O 4096x4096, gate_up 24576x4096, down 4096x12288",
+    "decode": "decode linears M in {1,8,32,64}, N=12288, K=4096",
+    "moe": "M-grouped contiguous MoE: 16384 rows over 32 experts (multinomial seed 0), N=4096, K=7168",
+    "square": "square 8192^3 with 5% outlier 1x128 groups (x100)",
+    "tiny": "tiny 128x256x512",
+}
+
+
+def is_hbm_bound(name: str) -> bool:
+    return name == "decode"
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local):
+    import moe_grouped_gemm_quantize_b200 as lnq
+    from moe_grouped_gemm_quantize_b200 import build as lnq_build
+
+    dist = init_dist(world)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        lnq_build.build()
+    barrier(dist)
+    lnq.lib()
+
+    cfgs, kind = workload_units(args.workload)
+    units = [Grouped(c, dev) if kind == "grouped" else Linear(c, dev) for c in cfgs]
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    calls = [u.calls(sp) for u in units]
+    n_units = len(units)
+    flops_step = sum(u.flops for u in units)
+    bytes_step = sum(u.gemm_bytes for u in units)
+
+    def launch_step(ev=None):
+        for i, ((qf, qa), (gf, ga)) in enumerate(calls):
+            if ev is not None:
+                ev[2 * i].record(stream)
+            rc = qf(*qa)
+            if rc:
+                raise lnq.LnqError(rc, "quantize")
+            if ev is not None:
+                ev[2 * i + 1].record(stream)
+            rc = gf(*ga)
+            if rc:
+                raise lnq.LnqError(rc, "gemm")
+        if ev is not None:
+            ev[2 * n_units].record(stream)
+
+    for _ in range(args.warmup):
+        launch_step()
+    torch.cuda.synchronize()
+    if lnq.lnq_get_last_device_error() != 0:
+        raise RuntimeError("device reported an error during warm-up")
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_units + 1)] for _ in range(K)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        t0.record(stream)
+        for k in range(K):
+            launch_step(evs[k])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(dist)
+    ms_local = t0.elapsed_time(t1)
+    if lnq.lnq_get_last_device_error() != 0:
+        raise RuntimeError("device reported an error in the timed region")
+    ms = max_over_ranks(ms_local, dist, dev)
+    q_ms = sum(evs[k][2 * i].elapsed_time(evs[k][2 * i + 1]) for k in range(K) for i in range(n_units))
+    g_ms = sum(evs[k][2 * i + 1].elapsed_time(evs[k][2 * i + 2]) for k in range(K)
+               for i in range(n_units))
+    per_gemm = [statistics.mean(evs[k][2 * i + 1].elapsed_time(evs[k][2 * i + 2]) for k in range(K))
+                for i in range(n_units)]
+    per_quant = [statistics.mean(evs[k][2 * i].elapsed_time(evs[k][2 * i + 1]) for k in range(K))
+                 for i in range(n_units)]
+
+    # ---- end to end through the public API: host inputs in, host outputs back
+    e2e = None
+    if not args.no_e2e:
+        Ke = max(1, min(K, args.e2e_steps))
+        for u in units:                       # warm the copy paths
+            u.x.copy_(u.host_x, non_blocking=True)
+            u.host_d.copy_(u.d, non_blocking=True)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier(dist)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(Ke):
+            for u, ((qf, qa), (gf, ga)) in zip(units, calls):
+                u.x.copy_(u.host_x, non_blocking=True)
+                rc = qf(*qa) or gf(*ga)
+                if rc:
+                    raise lnq.LnqError(rc, "e2e")
+                u.host_d.copy_(u.d, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(dist)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        if is_hbm_bound(args.workload):
+            ev_val = bytes_step * Ke * world / (e_ms * 1e-3) / 1e9
+            ev_unit = "GB/s"
+        else:
+            ev_val = flops_step * Ke * world / (e_ms * 1e-3) / 1e12
+            ev_unit = "TFLOP/s"
+        e2e = {"value": round(ev_val, 3), "unit": ev_unit, "steps": Ke,
+               "h2d_bytes_per_step": int(sum(u.h2d_bytes for u in units)),
+               "d2h_bytes_per_step": int(sum(u.d2h_bytes for u in units)),
+               "note": "pinned host bf16 activations copied in and bf16 outputs copied back "
+                       "every step; weights resident (model parameters)"}
+
+    # ---- numbers
+    peaks, peak_src = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    if is_hbm_bound(args.workload):
+        value = bytes_step * K * world / (ms * 1e-3) / 1e9
+        unit = "GB/s"
+        ach = bytes_step * K / (g_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 4)}
+        peak_note = f"HBM copy bandwidth ({peak_src})"
+    else:
+        value = flops_step * K * world / (ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        ach = flops_step * K / (g_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4)}
+        peak_note = (f"dense FP8 = {FP8_OVER_BF16:g} x bf16 cuBLAS burst {peaks['bf16_tflops']} "
+                     f"TFLOP/s ({peak_src})")
+    traffic = recorded_traffic("k_fp8_block_gemm", args.workload)
+    roof["traffic"] = traffic
+    roof["kernel"] = "k_fp8_block_gemm"
+    roof["peak_source"] = peak_note
+    roof["algorithmic_per_launch"] = ({"bytes": [int(u.gemm_bytes) for u in units]}
+                                      if is_hbm_bound(args.workload)
+                                      else {"flops": [float(u.flops) for u in units]})
+    quant_gbs = sum(u.quant_bytes for u in units) * K / (q_ms * 1e-3) / 1e9
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": unit,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, bf16)",
+        "config": {"workload": args.workload, "desc": WORKLOAD_DESC[args.workload],
+                   "parallelism": f"replicas x{world} (independent tokens per rank)",
+                   "l2": "working set per step > 126 MB L2; no extra flush"},
+        "roofline": roof,
+        "kernels": {
+            "gemm_ms_per_launch": [round(x, 5) for x in per_gemm],
+            "quantize_ms_per_launch": [round(x, 5) for x in per_quant],
+            "quantize_gbs": round(quant_gbs, 1),
+            "quantize_frac_of_hbm": round(quant_gbs / peaks["hbm_gbs"], 4),
+            "gemm_share_of_step": round(g_ms / (g_ms + q_ms), 4),
+        },
+        "gpu_launches": K * 2 * n_units,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, target_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- the oracle (CPU)
+
+def oracle_sample(workload: str, rows: int):
+    """Inputs for the oracle on the first `rows` activation rows of each linear."""
+    import oracle
+    from moe_grouped_gemm_quantize_b200 import synthetic
+    cfgs, kind = workload_units(workload)
+    items = []
+    for c in cfgs:
+        if kind == "grouped":
+            a, w, m_indices, _ = synthetic.make_moe_inputs(c)
+            r = min(rows, 128)
+            a_bits = synthetic.bf16_bits(a[:r])
+            # the first rows belong to group 0: its weights are the product's B
+            wq, ws = oracle.quantize_fp8_blocks(synthetic.bf16_bits(w[:c.N]))
+            items.append((a_bits, wq, ws, 2.0 * r * c.N * c.K))
+        else:
+            a, w = synthetic.make_linear_inputs(c)
+            r = min(rows, c.M)
+            wq, ws = oracle.quantize_fp8_blocks(synthetic.bf16_bits(w))
+            items.append((synthetic.bf16_bits(a[:r]), wq, ws, 2.0 * r * c.N * c.K))
+    return items
+
+
+def oracle_step(items):
+    import oracle
+    for a_bits, wq, ws, _ in items:
+        qa, sa = oracle.quantize_fp8_groups(a_bits)
+        oracle.gemm_nt(qa, sa, wq, ws)
+
+
+def cpu_baseline(workload: str, target_s: float = 10.0):
+    """The oracle, as it stands, timed on this host on a bounded sample of the workload."""
+    import oracle
+    items = oracle_sample(workload, 1)
+    t = time.perf_counter()
+    oracle_step(items)
+    t1 = time.perf_counter() - t
+    rows = int(max(1, min(64, target_s / max(t1, 1e-3))))
+    items = oracle_sample(workload, rows)
+    t = time.perf_counter()
+    oracle_step(items)
+    dt = time.perf_counter() - t
+    flops = sum(it[3] for it in items)
+    if is_hbm_bound(workload):
+        byts = sum(it[0].size * 3 + it[1].size + 2 * it[0].shape[0] * it[1].shape[0] for it in items)
+        val, unit = byts / dt / 1e9, "GB/s"
+    else:
+        val, unit = flops / dt / 1e12, "TFLOP/s"
+    return {"value": val, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {rows} activation row(s) of each linear of the workload "
+                      f"(quantize + FP64 product, weights pre-quantized), {dt:.2f} s"}
+
+
+def run_reference(args, world, rank, local):
+    """The reference arm: the CPU oracle on a bounded sample, on rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    rows = 1
+    items = oracle_sample(args.workload, rows)
+    for _ in range(args.warmup):
+        oracle_step(items)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(items)
+    dt = time.perf_counter() - t
+    flops = sum(it[3] for it in items) * args.steps
+    if is_hbm_bound(args.workload):
+        byts = sum(it[0].size * 3 + it[1].size + 2 * it[0].shape[0] * it[1].shape[0]
+                   for it in items) * args.steps
+        val, unit = byts / dt / 1e9, "GB/s"
+    else:
+        val, unit = flops / dt / 1e12, "TFLOP/s"
+    sample = (f"first {rows} activation row of each linear per step "
+              f"(quantize + FP64 product, weights pre-quantized)")
+    out = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": val,
+        "unit": unit,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": args.workload, "desc": WORKLOAD_DESC[args.workload]},
+        "cpu_baseline": {"value": val, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill", "decode", "moe", "square", "tiny"],
+                    default="prefill")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank, local)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

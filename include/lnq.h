@@ -1,0 +1,172 @@
+/*
+ * lnq.h -- C ABI of liblnq.so: the fine-grained block-scaled FP8 linear
+ * D = A . B^T on NVIDIA B200 (sm_100a), and its M-grouped contiguous MoE
+ * variant.
+ *
+ * Numerics (the "DeepSeek gran-128" recipe):
+ *   - activations are quantized per row in groups of 128 consecutive inputs,
+ *     each group with its own FP32 scale s = amax / 448 and E4M3 codes
+ *     q = E4M3_RNE_saturating(x / s)
+ *       (Linnet "Backend plugins", DeepGEMM plugin source, docstring and
+ *        _BlockProduct.execute; deepgemm-rust README, "What's implemented",
+ *        fp8_gemm_nt row);
+ *   - weights are E4M3 in 128 x 128 blocks with one FP32 scale per block
+ *       (Linnet plugin docstring; deepgemm-rust README, "Quick start");
+ *   - the product of each 128-wide K block is accumulated in FP32 on the
+ *     tensor cores, multiplied by sa * sb and added into an FP32 accumulator;
+ *     the output is BF16 (deepgemm-rust README, "What's implemented":
+ *     "FP32 promotion, BF16 out").
+ *
+ * Conventions shared by every call:
+ *   - All pointers are device pointers (cudaMalloc / PyTorch CUDA memory) on
+ *     the current device, 16-byte aligned.  The library never takes
+ *     ownership, never allocates device memory and never synchronizes the
+ *     stream (except lnq_get_last_device_error).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is asynchronous on that stream.
+ *   - Argument errors are detected on the host and returned before any CUDA
+ *     call; on such an error nothing is launched and no output is written.
+ *     LNQ_ERR_CUDA reports a failed CUDA runtime/driver call (launch or
+ *     descriptor encoding).  A kernel whose bounded wait expired reports it
+ *     through lnq_get_last_device_error.
+ *   - K must be a multiple of 128 (deepgemm-rust README, "Quick start":
+ *     "k must be a multiple of 128").
+ *   - E4M3 tensors are OCP FP8 E4M3 ("e4m3fn") bytes, BF16 tensors raw
+ *     bfloat16, all row-major.
+ */
+#ifndef LNQ_H
+#define LNQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lnq_status {
+    LNQ_OK = 0,
+    LNQ_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad stride */
+    LNQ_ERR_UNSUPPORTED_SHAPE = 2, /* K % 128 != 0, N % 16 != 0, M4 < ceil4(M), ... */
+    LNQ_ERR_MISALIGNED = 3,        /* a pointer not 16-byte aligned */
+    LNQ_ERR_UNSUPPORTED_ARCH = 4,  /* current device is not compute capability 10.0 */
+    LNQ_ERR_CUDA = 5,              /* a CUDA call failed */
+    LNQ_ERR_TIMEOUT = 6            /* a kernel's bounded wait expired (device-reported) */
+} lnq_status;
+
+/*
+ * Activation quantization, 1 x 128 groups (amax, scale and E4M3 cast fused in
+ * one pass over the input).
+ *
+ *   x_bf16  [M][ld_x] bf16; the first K columns of each row are read.
+ *   q_e4m3  [M][ld_q] E4M3; the first K columns of each row are written.
+ *   sfa     [K/128][M4] fp32, MN-major ("column by column"): the scale of
+ *           row m, group g is sfa[g*M4 + m].  Entries m in [M, M4) are
+ *           written as 0.0f.  M4 >= ceil4(M) and M4 % 4 == 0, so each scale
+ *           column starts 16-byte aligned (Linnet plugin: "the rows padded
+ *           to a multiple of four and the scales column by column";
+ *           _BlockProduct.execute, `padded`).
+ *   Scale s = amax/448 as an IEEE fp32 division; q = E4M3 round-to-nearest-
+ *   even of the correctly rounded fp32 quotient x/s, saturating at +-448.  A
+ *   group with amax == 0 gets s = 0.0f and codes 0x00 (0x80 for -0.0).
+ *
+ *   Requires: M >= 0 (M == 0 writes nothing), K % 128 == 0, ld_x >= K,
+ *   ld_x % 8 == 0, ld_q >= K, ld_q % 16 == 0, pointers 16-byte aligned.
+ */
+lnq_status lnq_quantize_fp8_groups(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x,
+                                   void* q_e4m3, int64_t ld_q, float* sfa, int64_t M4,
+                                   void* stream);
+
+/*
+ * Weight quantization, 128 x 128 blocks (offline preparation of the weight
+ * operand; Linnet plugin docstring, "weight blocks of 128 by 128";
+ * deepgemm-rust README, "Quick start", sfb shape (n/128, k/128)).
+ *
+ *   w_bf16  [N][K] bf16 row-major.
+ *   q_e4m3  [N][K] E4M3.
+ *   sfb     [ceil(N/128)][K/128] fp32 row-major: the scale of the block
+ *           (nb, kb) is sfb[nb*(K/128) + kb].  A ragged last row block takes
+ *           its amax over the rows that exist.
+ *   Same scale and rounding rule as lnq_quantize_fp8_groups.
+ *   Requires: N >= 1, K % 128 == 0, pointers 16-byte aligned.
+ */
+lnq_status lnq_quantize_fp8_blocks(const void* w_bf16, int64_t N, int64_t K, void* q_e4m3,
+                                   float* sfb, void* stream);
+
+/*
+ * Block-scaled FP8 GEMM, "nt" (both operands K-major):
+ *   D[m][n] = bf16_RN( sum_g  sfa[g*M4+m] * sfb[(n/128)*(K/128)+g]
+ *                              * sum_{k in block g} a[m][k] * b[n][k] )
+ * with the inner sums on the tensor cores (FP32) and the promotion in FP32
+ * (deepgemm-rust README, "What's implemented", fp8_gemm_nt; Linnet plugin,
+ * _BlockProduct.execute, deep_gemm.fp8_gemm_nt((q, scales), (weight, f32
+ * scale), out, disable_ue8m0_cast=True)).
+ *
+ *   a_e4m3  [M][K] E4M3 (activations, row stride K).
+ *   sfa     [K/128][M4] fp32 MN-major, as written by lnq_quantize_fp8_groups.
+ *   b_e4m3  [N][K] E4M3 (weights, row stride K).
+ *   sfb     [ceil(N/128)][K/128] fp32, as written by lnq_quantize_fp8_blocks.
+ *   d_bf16  [M][N] bf16 row-major (row stride N), fully overwritten.
+ *   Requires: M >= 1, N >= 16, N % 16 == 0, K % 128 == 0, M4 >= ceil4(M),
+ *   M4 % 4 == 0, pointers 16-byte aligned.  M <= 64 runs the decode
+ *   configuration (weights in the MMA's M slot); larger M runs the
+ *   persistent 128 x BN tile kernel.
+ */
+lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4,
+                                 const void* b_e4m3, const float* sfb, void* d_bf16, int64_t M,
+                                 int64_t N, int64_t K, void* stream);
+
+/*
+ * M-grouped contiguous block-scaled FP8 GEMM (MoE experts): tokens of all
+ * groups concatenated along M, every group starting at a multiple of 128
+ * rows, a per-row group id (deepgemm-rust README, "Grouped (contiguous) MoE
+ * GEMM" and "What's implemented", m_grouped_fp8_gemm_nt_contiguous;
+ * Triton_Grouped_GEMM README, "Example DeepGEMM layout creation").
+ *
+ *   a_e4m3     [M_total][K] E4M3.
+ *   sfa        [K/128][M_total] fp32 MN-major.
+ *   b_e4m3     [num_groups*N][K] E4M3: rows g*N .. g*N+N-1 are group g's weights.
+ *   sfb        [num_groups*ceil(N/128)][K/128] fp32: row g*ceil(N/128)+nb.
+ *   m_indices  [M_total] int32: group of each row, or -1 for a pad row.  Each
+ *              128-row block takes the group of its first row; a block whose
+ *              first row is -1 is skipped (its D rows are not written).  Pad
+ *              rows inside a block are computed with the block's group and
+ *              their D rows are unspecified.
+ *   d_bf16     [M_total][N] bf16.
+ *   Requires: M_total >= 128, M_total % 128 == 0, num_groups >= 1,
+ *   N % 16 == 0, K % 128 == 0, ids < num_groups, pointers 16-byte aligned.
+ */
+lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sfa,
+                                             const void* b_e4m3, const float* sfb,
+                                             const int32_t* m_indices, int32_t num_groups,
+                                             void* d_bf16, int64_t M_total, int64_t N, int64_t K,
+                                             void* stream);
+
+/* Static text for a status code. */
+const char* lnq_status_string(lnq_status status);
+
+/*
+ * Synchronizes `stream`, then reads and clears the library's device status
+ * word on the current device.  Returns LNQ_ERR_TIMEOUT if a kernel launched
+ * since the last call gave up on a bounded wait (the kernel then skipped its
+ * remaining work and released its tensor memory; its outputs are
+ * unspecified), LNQ_ERR_CUDA if the synchronization failed, else LNQ_OK.
+ */
+lnq_status lnq_get_last_device_error(void* stream);
+
+/*
+ * Diagnostic: launches one tiny kernel that waits on a barrier nobody
+ * arrives on, with a limit of `timeout_ns` nanoseconds (1e3 .. 1e10), then
+ * records LNQ_ERR_TIMEOUT in the device status word exactly as the GEMM
+ * kernels do when one of their waits expires.  Used to test the timeout path
+ * without faulting or hanging the GPU.  Returns the launch status.
+ */
+lnq_status lnq_selftest_wait_timeout(int64_t timeout_ns, void* stream);
+
+/* Version of this ABI (major*10000 + minor*100 + patch). */
+int32_t lnq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LNQ_H */

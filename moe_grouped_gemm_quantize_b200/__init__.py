@@ -1,1 +1,233 @@
-"""Block-scaled FP8 linear for B200 (sm_100a): Python binding of liblnq.so (placeholder)."""
+"""Block-scaled FP8 linear for NVIDIA B200 (sm_100a): Python binding of liblnq.so.
+
+The functions named ``lnq_*`` mirror the C ABI in ``include/lnq.h`` one to one;
+they only marshal torch tensors to pointers, sizes and the current CUDA stream
+and raise :class:`LnqError` on a non-zero status.  Every step of the path runs
+in the CUDA kernels of ``liblnq.so``; there is no CPU fallback, and a missing
+library raises.
+
+Numerics: activations quantized per row in 1x128 groups and weights in
+128x128 blocks to E4M3 with FP32 scales amax/448; the product of each 128-wide
+K block accumulated in FP32 on the tensor cores and promoted by sa*sb in FP32;
+BF16 output (Linnet "Backend plugins", DeepGEMM plugin; deepgemm-rust README,
+"What's implemented").
+
+The helpers below the ABI wrappers (``quantize_activations``,
+``quantize_weights``, ``linear``, ``m_grouped_linear``) allocate their outputs
+with torch and call the same entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "LnqError", "library_path", "lib",
+    "lnq_quantize_fp8_groups", "lnq_quantize_fp8_blocks", "lnq_fp8_block_gemm_nt",
+    "lnq_m_grouped_fp8_gemm_contiguous", "lnq_get_last_device_error", "lnq_status_string",
+    "lnq_selftest_wait_timeout", "quantize_activations", "quantize_weights", "linear",
+    "m_grouped_linear", "ceil4",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liblnq.so")
+_lock = threading.Lock()
+_lib = None
+
+LNQ_OK = 0
+STATUS_NAMES = {
+    0: "LNQ_OK", 1: "LNQ_ERR_INVALID_ARG", 2: "LNQ_ERR_UNSUPPORTED_SHAPE", 3: "LNQ_ERR_MISALIGNED",
+    4: "LNQ_ERR_UNSUPPORTED_ARCH", 5: "LNQ_ERR_CUDA", 6: "LNQ_ERR_TIMEOUT",
+}
+
+
+class LnqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)} "
+                         f"({lnq_status_string(self.status)})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded liblnq.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m moe_grouped_gemm_quantize_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+        sigs = {
+            "lnq_quantize_fp8_groups": [P, I64, I64, I64, P, I64, P, I64, P],
+            "lnq_quantize_fp8_blocks": [P, I64, I64, P, P, P],
+            "lnq_fp8_block_gemm_nt": [P, P, I64, P, P, P, I64, I64, I64, P],
+            "lnq_m_grouped_fp8_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
+            "lnq_get_last_device_error": [P],
+            "lnq_selftest_wait_timeout": [I64, P],
+        }
+        for name, args in sigs.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        L.lnq_status_string.argtypes = [ctypes.c_int]
+        L.lnq_status_string.restype = ctypes.c_char_p
+        L.lnq_abi_version.restype = ctypes.c_int32
+        _lib = L
+        return L
+
+
+def lnq_status_string(status: int) -> str:
+    return lib().lnq_status_string(int(status)).decode()
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != LNQ_OK:
+        raise LnqError(rc, where)
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _is_fp8(t: torch.Tensor) -> bool:
+    return t.dtype in (torch.float8_e4m3fn, torch.uint8)
+
+
+def ceil4(m: int) -> int:
+    return -(-int(m) // 4) * 4
+
+
+# ----------------------------------------------------------------- the C ABI
+
+def lnq_quantize_fp8_groups(x: torch.Tensor, q: torch.Tensor, sfa: torch.Tensor, stream=None) -> None:
+    """x bf16 [M, K] (row stride ld_x), q e4m3 [M, K] (row stride ld_q), sfa fp32 [K/128, M4]."""
+    if x.dtype != torch.bfloat16 or not _is_fp8(q) or sfa.dtype != torch.float32:
+        raise TypeError("x must be bf16, q float8_e4m3fn/uint8, sfa float32")
+    M, K = x.shape
+    if x.stride(1) != 1 or q.stride(1) != 1 or not sfa.is_contiguous() or tuple(q.shape) != (M, K):
+        raise ValueError("x, q need unit column stride, sfa must be contiguous, q shaped like x")
+    if sfa.shape[0] != K // 128:
+        raise ValueError("sfa must be [K/128, M4]")
+    _check(lib().lnq_quantize_fp8_groups(_ptr(x), M, K, x.stride(0), _ptr(q), q.stride(0),
+                                         _ptr(sfa), sfa.shape[1], _stream(stream)),
+           "lnq_quantize_fp8_groups")
+
+
+def lnq_quantize_fp8_blocks(w: torch.Tensor, q: torch.Tensor, sfb: torch.Tensor, stream=None) -> None:
+    """w bf16 [N, K], q e4m3 [N, K], sfb fp32 [ceil(N/128), K/128], all contiguous."""
+    if w.dtype != torch.bfloat16 or not _is_fp8(q) or sfb.dtype != torch.float32:
+        raise TypeError("w must be bf16, q float8_e4m3fn/uint8, sfb float32")
+    N, K = w.shape
+    if not (w.is_contiguous() and q.is_contiguous() and sfb.is_contiguous()):
+        raise ValueError("w, q, sfb must be contiguous")
+    if tuple(q.shape) != (N, K) or tuple(sfb.shape) != (-(-N // 128), K // 128):
+        raise ValueError("q must be [N, K] and sfb [ceil(N/128), K/128]")
+    _check(lib().lnq_quantize_fp8_blocks(_ptr(w), N, K, _ptr(q), _ptr(sfb), _stream(stream)),
+           "lnq_quantize_fp8_blocks")
+
+
+def lnq_fp8_block_gemm_nt(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                          d: torch.Tensor, stream=None) -> None:
+    """a e4m3 [M, K], sfa fp32 [K/128, M4], b e4m3 [N, K], sfb fp32 [ceil(N/128), K/128], d bf16 [M, N]."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.float32 or \
+            sfb.dtype != torch.float32 or d.dtype != torch.bfloat16:
+        raise TypeError("a, b float8_e4m3fn/uint8; sfa, sfb float32; d bf16")
+    M, K = a.shape
+    N = b.shape[0]
+    for t in (a, sfa, b, sfb, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    if b.shape[1] != K or tuple(d.shape) != (M, N) or sfa.shape[0] != K // 128 or \
+            tuple(sfb.shape) != (-(-N // 128), K // 128):
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_fp8_block_gemm_nt(_ptr(a), _ptr(sfa), sfa.shape[1], _ptr(b), _ptr(sfb), _ptr(d),
+                                       M, N, K, _stream(stream)), "lnq_fp8_block_gemm_nt")
+
+
+def lnq_m_grouped_fp8_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,
+                                      sfb: torch.Tensor, m_indices: torch.Tensor, num_groups: int,
+                                      d: torch.Tensor, stream=None) -> None:
+    """a e4m3 [M_total, K], sfa [K/128, M_total], b e4m3 [G*N, K], sfb [G*ceil(N/128), K/128],
+    m_indices int32 [M_total], d bf16 [M_total, N]."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.float32 or \
+            sfb.dtype != torch.float32 or d.dtype != torch.bfloat16 or m_indices.dtype != torch.int32:
+        raise TypeError("a, b e4m3; sfa, sfb float32; m_indices int32; d bf16")
+    for t in (a, sfa, b, sfb, m_indices, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    M_total, K = a.shape
+    G = int(num_groups)
+    N = d.shape[1]
+    if b.shape[0] != G * N or b.shape[1] != K or tuple(sfa.shape) != (K // 128, M_total) or \
+            tuple(sfb.shape) != (G * -(-N // 128), K // 128) or m_indices.shape[0] != M_total or \
+            d.shape[0] != M_total:
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_m_grouped_fp8_gemm_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb),
+                                                   _ptr(m_indices), G, _ptr(d), M_total, N, K,
+                                                   _stream(stream)),
+           "lnq_m_grouped_fp8_gemm_contiguous")
+
+
+def lnq_get_last_device_error(stream=None) -> int:
+    """Synchronizes the stream; returns (and clears) the device-reported status."""
+    return int(lib().lnq_get_last_device_error(_stream(stream)))
+
+
+def lnq_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:
+    _check(lib().lnq_selftest_wait_timeout(int(timeout_ns), _stream(stream)),
+           "lnq_selftest_wait_timeout")
+
+
+# ----------------------------------------------------------------- helpers
+
+def quantize_activations(x: torch.Tensor, stream=None):
+    """(q e4m3 [M, K], sfa fp32 [K/128, ceil4(M)]) of a bf16 [M, K] CUDA tensor."""
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    sfa = torch.empty((K // 128, ceil4(M)), dtype=torch.float32, device=x.device)
+    lnq_quantize_fp8_groups(x, q, sfa, stream)
+    return q, sfa
+
+
+def quantize_weights(w: torch.Tensor, stream=None):
+    """(q e4m3 [N, K], sfb fp32 [ceil(N/128), K/128]) of a bf16 [N, K] CUDA tensor."""
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
+    sfb = torch.empty((-(-N // 128), K // 128), dtype=torch.float32, device=w.device)
+    lnq_quantize_fp8_blocks(w.contiguous(), q, sfb, stream)
+    return q, sfb
+
+
+def linear(x: torch.Tensor, w_q: torch.Tensor, w_s: torch.Tensor, stream=None) -> torch.Tensor:
+    """y = x . W^T in bf16 with x quantized on the fly (1x128) and W pre-quantized (128x128)."""
+    q, sfa = quantize_activations(x, stream)
+    d = torch.empty((x.shape[0], w_q.shape[0]), dtype=torch.bfloat16, device=x.device)
+    lnq_fp8_block_gemm_nt(q, sfa, w_q, w_s, d, stream)
+    return d
+
+
+def m_grouped_linear(x: torch.Tensor, w_q: torch.Tensor, w_s: torch.Tensor, m_indices: torch.Tensor,
+                     num_groups: int, stream=None) -> torch.Tensor:
+    """Grouped y for the contiguous MoE layout (x rows already padded per group to 128)."""
+    q, sfa = quantize_activations(x, stream)
+    N = w_q.shape[0] // num_groups
+    d = torch.empty((x.shape[0], N), dtype=torch.bfloat16, device=x.device)
+    lnq_m_grouped_fp8_gemm_contiguous(q, sfa, w_q, w_s, m_indices, num_groups, d, stream)
+    return d

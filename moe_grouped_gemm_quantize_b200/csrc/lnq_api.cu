@@ -1,0 +1,318 @@
+// lnq_api.cu -- host layer of liblnq.so: argument checks, device checks, TMA
+// descriptor encoding, tile-configuration choice and kernel launches behind
+// the C ABI declared in include/lnq.h.
+//
+// The library allocates no device memory and never synchronizes a stream on
+// the compute path.  Argument errors are returned before any CUDA call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "lnq.h"
+#include "lnq_gemm.cuh"
+#include "lnq_ptx.cuh"
+#include "lnq_quantize.cuh"
+
+namespace lnq {
+
+// Device status word: timeout and bad-group bits set by the kernels.
+__device__ unsigned int g_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceInfo {
+    bool ready = false;
+    bool supported = false;
+    int sm_count = 0;
+    unsigned int* status = nullptr;  // device address of g_status
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device's capabilities; resolves the driver's tensor-map encoder once.
+lnq_status device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LNQ_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return LNQ_ERR_UNSUPPORTED_ARCH;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& d = g_devices[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return LNQ_ERR_CUDA;
+        d.supported = (major == 10 && minor == 0);
+        d.sm_count = sms;
+        if (d.supported) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return LNQ_ERR_CUDA;
+            d.status = static_cast<unsigned int*>(p);
+        }
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return LNQ_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        d.ready = true;
+    }
+    if (!d.supported) return LNQ_ERR_UNSUPPORTED_ARCH;
+    *out = &d;
+    return LNQ_OK;
+}
+
+// 2-D E4M3 tensor [rows][cols] (cols contiguous, row stride = cols bytes),
+// box of 128 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+lnq_status encode_e4m3_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                           int box_rows) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+    cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+template <class C>
+lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
+                       const void* wgt, int64_t wgt_rows, int64_t K, GemmArgs args,
+                       cudaStream_t stream) {
+    CUtensorMap map_p, map_q;
+    lnq_status st;
+    if (C::SWAP) {
+        st = encode_e4m3_map(&map_p, wgt, wgt_rows, K, C::kP);
+        if (st == LNQ_OK) st = encode_e4m3_map(&map_q, act, act_rows, K, C::BNQ);
+    } else {
+        st = encode_e4m3_map(&map_p, act, act_rows, K, C::kP);
+        if (st == LNQ_OK) st = encode_e4m3_map(&map_q, wgt, wgt_rows, K, C::BNQ);
+    }
+    if (st != LNQ_OK) return st;
+    static bool attr_set[kMaxDevices] = {};
+    int devno = 0;
+    cudaGetDevice(&devno);
+    if (!attr_set[devno]) {
+        if (cudaFuncSetAttribute(k_fp8_block_gemm<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes) != cudaSuccess)
+            return LNQ_ERR_CUDA;
+        attr_set[devno] = true;
+    }
+    args.status = dev.status;
+    args.timeout_ns = kDefaultTimeoutNs;
+    const int grid = args.num_tiles < dev.sm_count ? args.num_tiles : dev.sm_count;
+    if (grid <= 0) return LNQ_OK;
+    k_fp8_block_gemm<C><<<grid, C::kThreads, C::kSmemBytes, stream>>>(map_p, map_q, args);
+    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+// Tile configurations (P = MMA M slot, Q = MMA N slot).
+using CfgDense256 = GemmCfg<256, 4, 2, false, false>;
+using CfgDense128 = GemmCfg<128, 6, 2, false, false>;
+using CfgGrouped256 = GemmCfg<256, 4, 2, false, true>;
+using CfgGrouped128 = GemmCfg<128, 6, 2, false, true>;
+using CfgSwap32 = GemmCfg<32, 8, 1, true, false>;
+using CfgSwap64 = GemmCfg<64, 8, 1, true, false>;
+
+constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
+
+}  // namespace
+}  // namespace lnq
+
+using namespace lnq;
+
+extern "C" {
+
+int32_t lnq_abi_version(void) { return 10000; }
+
+const char* lnq_status_string(lnq_status s) {
+    switch (s) {
+        case LNQ_OK: return "ok";
+        case LNQ_ERR_INVALID_ARG: return "invalid argument";
+        case LNQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case LNQ_ERR_MISALIGNED: return "misaligned pointer or stride";
+        case LNQ_ERR_UNSUPPORTED_ARCH: return "device is not sm_100 (B200)";
+        case LNQ_ERR_CUDA: return "CUDA call failed";
+        case LNQ_ERR_TIMEOUT: return "a kernel wait timed out";
+    }
+    return "unknown status";
+}
+
+lnq_status lnq_quantize_fp8_groups(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x,
+                                   void* q_e4m3, int64_t ld_q, float* sfa, int64_t M4,
+                                   void* stream) {
+    if (M < 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
+    if (K % 128 != 0) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (ld_x < K || ld_q < K) return LNQ_ERR_INVALID_ARG;
+    if (M4 < ((M + 3) / 4) * 4 || M4 % 4 != 0 || M4 > kMaxRows) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (K / 256 + 1 > 65535) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (M4 == 0) return LNQ_OK;
+    if (!sfa || (M > 0 && (!x_bf16 || !q_e4m3))) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(q_e4m3) || !aligned16(sfa) || ld_x % 8 != 0 ||
+        ld_q % 16 != 0)
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    dim3 grid(static_cast<unsigned>((M4 + kQuantRowsPerCta - 1) / kQuantRowsPerCta),
+              static_cast<unsigned>((K + kQuantColsPerCta - 1) / kQuantColsPerCta));
+    k_quantize_groups<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(x_bf16), M, K, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sfa,
+        M4);
+    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+lnq_status lnq_quantize_fp8_blocks(const void* w_bf16, int64_t N, int64_t K, void* q_e4m3,
+                                   float* sfb, void* stream) {
+    if (N <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N > kMaxRows || K / 128 > 65535) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!w_bf16 || !q_e4m3 || !sfb) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(w_bf16) || !aligned16(q_e4m3) || !aligned16(sfb)) return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>(K / 128));
+    k_quantize_blocks<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(w_bf16), N, K, static_cast<uint8_t*>(q_e4m3), sfb);
+    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4,
+                                 const void* b_e4m3, const float* sfb, void* d_bf16, int64_t M,
+                                 int64_t N, int64_t K, void* stream) {
+    if (M <= 0 || N <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N % 16 != 0 || N < 16 || M > kMaxRows || N > kMaxRows ||
+        K > (int64_t{1} << 31))
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (M4 < ((M + 3) / 4) * 4 || M4 % 4 != 0) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!a_e4m3 || !sfa || !b_e4m3 || !sfb || !d_bf16) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned16(sfb) ||
+        !aligned16(d_bf16))
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+
+    GemmArgs args{};
+    args.sfa = sfa;
+    args.sfb = sfb;
+    args.d = static_cast<uint16_t*>(d_bf16);
+    args.M4 = M4;
+    args.M = static_cast<int>(M);
+    args.N = static_cast<int>(N);
+    args.num_kb = static_cast<int>(K / 128);
+    args.nb = static_cast<int>((N + 127) / 128);
+    args.num_groups = 1;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= 64) {
+        // decode: weights in the MMA's 128-row slot, tokens padded to 32 or 64
+        args.tiles_p = static_cast<int>((N + 127) / 128);
+        if (M <= 32) {
+            args.tiles_q = static_cast<int>((M + 31) / 32);
+            args.num_tiles = args.tiles_p * args.tiles_q;
+            return launch_gemm<CfgSwap32>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
+        }
+        args.tiles_q = static_cast<int>((M + 63) / 64);
+        args.num_tiles = args.tiles_p * args.tiles_q;
+        return launch_gemm<CfgSwap64>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
+    }
+    args.tiles_p = static_cast<int>((M + 127) / 128);
+    if (N >= 256) {
+        args.tiles_q = static_cast<int>((N + 255) / 256);
+        args.num_tiles = args.tiles_p * args.tiles_q;
+        return launch_gemm<CfgDense256>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
+    }
+    args.tiles_q = static_cast<int>((N + 127) / 128);
+    args.num_tiles = args.tiles_p * args.tiles_q;
+    return launch_gemm<CfgDense128>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
+}
+
+lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sfa,
+                                             const void* b_e4m3, const float* sfb,
+                                             const int32_t* m_indices, int32_t num_groups,
+                                             void* d_bf16, int64_t M_total, int64_t N, int64_t K,
+                                             void* stream) {
+    if (M_total <= 0 || N <= 0 || K <= 0 || num_groups <= 0) return LNQ_ERR_INVALID_ARG;
+    if (M_total % 128 != 0 || K % 128 != 0 || N % 16 != 0 || N < 16 || M_total > kMaxRows ||
+        K > (int64_t{1} << 31) || static_cast<int64_t>(num_groups) * N > kMaxRows)
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!a_e4m3 || !sfa || !b_e4m3 || !sfb || !m_indices || !d_bf16) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned16(sfb) ||
+        !aligned16(d_bf16) || (reinterpret_cast<uintptr_t>(m_indices) & 3u) != 0)
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+
+    GemmArgs args{};
+    args.sfa = sfa;
+    args.sfb = sfb;
+    args.d = static_cast<uint16_t*>(d_bf16);
+    args.m_indices = m_indices;
+    args.M4 = M_total;
+    args.M = static_cast<int>(M_total);
+    args.N = static_cast<int>(N);
+    args.num_kb = static_cast<int>(K / 128);
+    args.nb = static_cast<int>((N + 127) / 128);
+    args.num_groups = num_groups;
+    args.tiles_p = static_cast<int>(M_total / 128);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t wrows = static_cast<int64_t>(num_groups) * N;
+    if (N >= 256) {
+        args.tiles_q = static_cast<int>((N + 255) / 256);
+        args.num_tiles = args.tiles_p * args.tiles_q;
+        return launch_gemm<CfgGrouped256>(*dev, a_e4m3, M_total, b_e4m3, wrows, K, args, s);
+    }
+    args.tiles_q = static_cast<int>((N + 127) / 128);
+    args.num_tiles = args.tiles_p * args.tiles_q;
+    return launch_gemm<CfgGrouped128>(*dev, a_e4m3, M_total, b_e4m3, wrows, K, args, s);
+}
+
+lnq_status lnq_get_last_device_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return LNQ_ERR_CUDA;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return LNQ_ERR_CUDA;
+    }
+    if (v & kStatusTimeout) return LNQ_ERR_TIMEOUT;
+    if (v & kStatusBadGroup) return LNQ_ERR_INVALID_ARG;
+    return LNQ_OK;
+}
+
+lnq_status lnq_selftest_wait_timeout(int64_t timeout_ns, void* stream) {
+    if (timeout_ns < 1000 || timeout_ns > 10000000000LL) return LNQ_ERR_INVALID_ARG;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    k_wait_timeout_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        dev->status, static_cast<unsigned long long>(timeout_ns));
+    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+}  // extern "C"

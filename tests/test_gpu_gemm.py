@@ -1,0 +1,134 @@
+"""GPU parity of the block-scaled FP8 GEMM (dense and decode) against the oracle.
+
+The oracle quantizes the same seeded bf16 inputs itself and computes D in FP64;
+the CUDA path quantizes with its own kernels (bit-exact with the oracle, see
+test_gpu_quantize) and multiplies.  Small and ragged shapes are compared element
+by element; the full workloads, in the launch configuration the benchmark times,
+on sampled points (random points plus one whole row and one whole column).
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_grouped_gemm_quantize_b200 as lnq
+import oracle
+from moe_grouped_gemm_quantize_b200 import synthetic
+from parity import assert_gemm_close, codes, oracle_quantize_a, oracle_quantize_w, sample_points, to_f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def gpu_linear(a: torch.Tensor, w: torch.Tensor):
+    wq, ws = lnq.quantize_weights(w.to(DEV))
+    aq, sa = lnq.quantize_activations(a.to(DEV))
+    d = torch.full((a.shape[0], w.shape[0]), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lnq.lnq_fp8_block_gemm_nt(aq, sa, wq, ws, d)
+    assert lnq.lnq_get_last_device_error() == 0
+    return d, (aq, sa, wq, ws)
+
+
+def oracle_linear(a, w):
+    qa, sa = oracle_quantize_a(a)
+    qb, sb = oracle_quantize_w(w)
+    return oracle.gemm_nt(qa, sa, qb, sb), (qa, sa, qb, sb)
+
+
+def check_full(a, w, what):
+    d, _ = gpu_linear(a, w)
+    ref, _ = oracle_linear(a, w)
+    return assert_gemm_close(to_f64(d), ref, what)
+
+
+def test_tiny_workload_elementwise():
+    a, w = synthetic.make_linear_inputs(synthetic.TINY)
+    check_full(a, w, "tiny 128x256x512")
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (65, 256, 128), (100, 128, 256), (128, 16, 128), (130, 272, 384), (200, 640, 512),
+    (257, 384, 640), (384, 1024, 1024), (129, 48, 256), (300, 4096, 128),
+])
+def test_dense_shapes_elementwise(M, N, K):
+    a = synthetic.gaussian_bf16((M, K), 1.0, seed=M + 7 * N + K)
+    w = synthetic.gaussian_bf16((N, K), 0.02, seed=M + N + 3 * K)
+    check_full(a, w, f"{M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 17, 31, 32, 33, 48, 63, 64])
+@pytest.mark.parametrize("N,K", [(256, 512), (384, 1024)])
+def test_decode_shapes_elementwise(M, N, K):
+    a = synthetic.gaussian_bf16((M, K), 1.0, seed=M * 5 + N)
+    w = synthetic.gaussian_bf16((N, K), 0.02, seed=N + K)
+    check_full(a, w, f"decode {M}x{N}x{K}")
+
+
+def test_outlier_groups_elementwise():
+    a = synthetic.gaussian_bf16_with_outliers((256, 1024), 1.0, 1, 2)
+    w = synthetic.gaussian_bf16_with_outliers((512, 1024), 1.0, 3, 4)
+    check_full(a, w, "outliers 256x512x1024")
+
+
+def test_oracle_quantized_operands_give_the_same_product():
+    # feed the oracle's own codes and scales to the GEMM: the result must equal the
+    # product of the GPU-quantized operands bit for bit (the quantize is bit-exact)
+    a, w = synthetic.make_linear_inputs(synthetic.TINY)
+    d, (aq, sa, wq, ws) = gpu_linear(a, w)
+    qa, sao = oracle_quantize_a(a)
+    qb, sbo = oracle_quantize_w(w)
+    d2 = torch.empty_like(d)
+    lnq.lnq_fp8_block_gemm_nt(torch.from_numpy(qa).to(DEV), torch.from_numpy(sao).to(DEV),
+                              torch.from_numpy(qb).to(DEV), torch.from_numpy(sbo).to(DEV), d2)
+    torch.cuda.synchronize()
+    assert torch.equal(d.view(torch.int16), d2.view(torch.int16))
+
+
+def test_deterministic():
+    a = synthetic.gaussian_bf16((512, 2048), 1.0, 5)
+    w = synthetic.gaussian_bf16((1024, 2048), 0.02, 6)
+    d1, _ = gpu_linear(a, w)
+    d2, _ = gpu_linear(a, w)
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+
+
+def check_sampled(a, w, what, count=20000, seed=0):
+    d, _ = gpu_linear(a, w)
+    qa, sa = oracle_quantize_a(a)
+    qb, sb = oracle_quantize_w(w)
+    M, N = d.shape
+    rows, cols = sample_points(M, N, count, seed, full_row=M - 1, full_col=N // 2 + 1)
+    ref = oracle.gemm_nt_points(qa, sa, qb, sb, rows, cols)
+    got = to_f64(d)[rows, cols]
+    return assert_gemm_close(got, ref, what)
+
+
+@pytest.mark.parametrize("idx", range(4))
+def test_prefill_workloads_sampled(idx):
+    cfg = synthetic.PREFILL[idx]
+    a, w = synthetic.make_linear_inputs(cfg)
+    check_sampled(a, w, cfg.name)
+
+
+def test_decode_workloads():
+    for cfg in synthetic.DECODE:
+        a, w = synthetic.make_linear_inputs(cfg)
+        if cfg.M <= 8:
+            check_full(a, w, cfg.name)
+        else:
+            check_sampled(a, w, cfg.name)
+
+
+def test_square_outlier_workload_sampled():
+    cfg = synthetic.SQUARE
+    a, w = synthetic.make_linear_inputs(cfg)
+    check_sampled(a, w, cfg.name, count=30000)
+
+
+def test_timeout_path_reports_and_recovers():
+    # a wait that nobody satisfies gives up after 20 ms and reports LNQ_ERR_TIMEOUT;
+    # the context stays usable and the status is cleared once read
+    lnq.lnq_selftest_wait_timeout(20_000_000)
+    assert lnq.lnq_get_last_device_error() == 6
+    assert lnq.lnq_get_last_device_error() == 0
+    a, w = synthetic.make_linear_inputs(synthetic.TINY)
+    check_full(a, w, "tiny after timeout")
