@@ -227,7 +227,7 @@ class Grouped:
         a, w, m_indices, sizes = synthetic.make_moe_inputs(cfg)
         self.M = a.shape[0]
         self.x = a.to(dev)
-        self.wq, self.ws = lnq.quantize_weights(w.to(dev))
+        self.wq, self.ws = lnq.quantize_weights_grouped(w.to(dev), cfg.groups)
         del w
         self.mi = torch.from_numpy(m_indices).to(dev)
         K, N, G = cfg.K, cfg.N, cfg.groups

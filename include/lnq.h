@@ -19,9 +19,10 @@
  *
  * Conventions shared by every call:
  *   - All pointers are device pointers (cudaMalloc / PyTorch CUDA memory) on
- *     the current device, 16-byte aligned.  The library never takes
- *     ownership, never allocates device memory and never synchronizes the
- *     stream (except lnq_get_last_device_error).
+ *     the current device, 16-byte aligned, except the weight-scale tensor
+ *     sfb and the group ids m_indices, which need 4-byte alignment.  The
+ *     library never takes ownership, never allocates device memory and
+ *     never synchronizes the stream (except lnq_get_last_device_error).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Every call is asynchronous on that stream.
  *   - Argument errors are detected on the host and returned before any CUDA
@@ -87,7 +88,11 @@ lnq_status lnq_quantize_fp8_groups(const void* x_bf16, int64_t M, int64_t K, int
  *           (nb, kb) is sfb[nb*(K/128) + kb].  A ragged last row block takes
  *           its amax over the rows that exist.
  *   Same scale and rounding rule as lnq_quantize_fp8_groups.
- *   Requires: N >= 1, K % 128 == 0, pointers 16-byte aligned.
+ *   Grouped weights [G*N][K] whose N is not a multiple of 128 are quantized
+ *   one group at a time (w + g*N*K, q + g*N*K, sfb + g*ceil(N/128)*(K/128)),
+ *   so that no 128 x 128 block spans two groups.
+ *   Requires: N >= 1, K % 128 == 0, w and q 16-byte aligned, sfb 4-byte
+ *   aligned.
  */
 lnq_status lnq_quantize_fp8_blocks(const void* w_bf16, int64_t N, int64_t K, void* q_e4m3,
                                    float* sfb, void* stream);
@@ -107,9 +112,9 @@ lnq_status lnq_quantize_fp8_blocks(const void* w_bf16, int64_t N, int64_t K, voi
  *   sfb     [ceil(N/128)][K/128] fp32, as written by lnq_quantize_fp8_blocks.
  *   d_bf16  [M][N] bf16 row-major (row stride N), fully overwritten.
  *   Requires: M >= 1, N >= 16, N % 16 == 0, K % 128 == 0, M4 >= ceil4(M),
- *   M4 % 4 == 0, pointers 16-byte aligned.  M <= 64 runs the decode
- *   configuration (weights in the MMA's M slot); larger M runs the
- *   persistent 128 x BN tile kernel.
+ *   M4 % 4 == 0, sfb 4-byte aligned, the other pointers 16-byte aligned.
+ *   M <= 64 runs the decode configuration (weights in the MMA's M slot);
+ *   larger M runs the persistent 128 x BN tile kernel.
  */
 lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4,
                                  const void* b_e4m3, const float* sfb, void* d_bf16, int64_t M,
@@ -125,7 +130,8 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
  *   a_e4m3     [M_total][K] E4M3.
  *   sfa        [K/128][M_total] fp32 MN-major.
  *   b_e4m3     [num_groups*N][K] E4M3: rows g*N .. g*N+N-1 are group g's weights.
- *   sfb        [num_groups*ceil(N/128)][K/128] fp32: row g*ceil(N/128)+nb.
+ *   sfb        [num_groups*ceil(N/128)][K/128] fp32: row g*ceil(N/128)+nb
+ *              (each group's weights quantized on their own).
  *   m_indices  [M_total] int32: group of each row, or -1 for a pad row.  Each
  *              128-row block takes the group of its first row; a block whose
  *              first row is -1 is skipped (its D rows are not written).  Pad
@@ -133,7 +139,10 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
  *              their D rows are unspecified.
  *   d_bf16     [M_total][N] bf16.
  *   Requires: M_total >= 128, M_total % 128 == 0, num_groups >= 1,
- *   N % 16 == 0, K % 128 == 0, ids < num_groups, pointers 16-byte aligned.
+ *   N % 16 == 0, K % 128 == 0, ids < num_groups (a block whose id is out of
+ *   range is skipped and reported by lnq_get_last_device_error as
+ *   LNQ_ERR_INVALID_ARG), sfb and m_indices 4-byte aligned, the other
+ *   pointers 16-byte aligned.
  */
 lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sfa,
                                              const void* b_e4m3, const float* sfb,

@@ -28,7 +28,8 @@ __all__ = [
     "LnqError", "library_path", "lib",
     "lnq_quantize_fp8_groups", "lnq_quantize_fp8_blocks", "lnq_fp8_block_gemm_nt",
     "lnq_m_grouped_fp8_gemm_contiguous", "lnq_get_last_device_error", "lnq_status_string",
-    "lnq_selftest_wait_timeout", "quantize_activations", "quantize_weights", "linear",
+    "lnq_selftest_wait_timeout", "quantize_activations", "quantize_weights",
+    "quantize_weights_grouped", "linear",
     "m_grouped_linear", "ceil4",
 ]
 
@@ -212,6 +213,23 @@ def quantize_weights(w: torch.Tensor, stream=None):
     q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
     sfb = torch.empty((-(-N // 128), K // 128), dtype=torch.float32, device=w.device)
     lnq_quantize_fp8_blocks(w.contiguous(), q, sfb, stream)
+    return q, sfb
+
+
+def quantize_weights_grouped(w: torch.Tensor, num_groups: int, stream=None):
+    """Per-group 128x128 quantization of grouped weights [G*N, K]:
+    (q e4m3 [G*N, K], sfb fp32 [G*ceil(N/128), K/128]).  Each group is quantized on
+    its own, so no block spans two groups when N is not a multiple of 128."""
+    GN, K = w.shape
+    G = int(num_groups)
+    N = GN // G
+    NB = -(-N // 128)
+    w = w.contiguous()
+    q = torch.empty((GN, K), dtype=torch.float8_e4m3fn, device=w.device)
+    sfb = torch.empty((G * NB, K // 128), dtype=torch.float32, device=w.device)
+    for g in range(G):
+        lnq_quantize_fp8_blocks(w[g * N:(g + 1) * N], q[g * N:(g + 1) * N],
+                                sfb[g * NB:(g + 1) * NB], stream)
     return q, sfb
 
 

@@ -43,6 +43,7 @@ DeviceInfo g_devices[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // Current device's capabilities; resolves the driver's tensor-map encoder once.
 lnq_status device_info(DeviceInfo** out) {
@@ -187,7 +188,7 @@ lnq_status lnq_quantize_fp8_blocks(const void* w_bf16, int64_t N, int64_t K, voi
     if (N <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
     if (K % 128 != 0 || N > kMaxRows || K / 128 > 65535) return LNQ_ERR_UNSUPPORTED_SHAPE;
     if (!w_bf16 || !q_e4m3 || !sfb) return LNQ_ERR_INVALID_ARG;
-    if (!aligned16(w_bf16) || !aligned16(q_e4m3) || !aligned16(sfb)) return LNQ_ERR_MISALIGNED;
+    if (!aligned16(w_bf16) || !aligned16(q_e4m3) || !aligned4(sfb)) return LNQ_ERR_MISALIGNED;
     DeviceInfo* dev = nullptr;
     lnq_status st = device_info(&dev);
     if (st != LNQ_OK) return st;
@@ -206,7 +207,7 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
         return LNQ_ERR_UNSUPPORTED_SHAPE;
     if (M4 < ((M + 3) / 4) * 4 || M4 % 4 != 0) return LNQ_ERR_UNSUPPORTED_SHAPE;
     if (!a_e4m3 || !sfa || !b_e4m3 || !sfb || !d_bf16) return LNQ_ERR_INVALID_ARG;
-    if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned16(sfb) ||
+    if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned4(sfb) ||
         !aligned16(d_bf16))
         return LNQ_ERR_MISALIGNED;
     DeviceInfo* dev = nullptr;
@@ -257,8 +258,8 @@ lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sf
         K > (int64_t{1} << 31) || static_cast<int64_t>(num_groups) * N > kMaxRows)
         return LNQ_ERR_UNSUPPORTED_SHAPE;
     if (!a_e4m3 || !sfa || !b_e4m3 || !sfb || !m_indices || !d_bf16) return LNQ_ERR_INVALID_ARG;
-    if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned16(sfb) ||
-        !aligned16(d_bf16) || (reinterpret_cast<uintptr_t>(m_indices) & 3u) != 0)
+    if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned4(sfb) ||
+        !aligned16(d_bf16) || !aligned4(m_indices))
         return LNQ_ERR_MISALIGNED;
     DeviceInfo* dev = nullptr;
     lnq_status st = device_info(&dev);

@@ -78,7 +78,8 @@ def test_block_quantize_argument_errors(L):
     assert f(A16, 0, 128, A16b, A16c, None) == INVALID
     assert f(A16, 128, 130, A16b, A16c, None) == SHAPE
     assert f(A16, 128, 128, None, A16c, None) == INVALID
-    assert f(A16, 128, 128, A16b, A16c + 4, None) == MISALIGNED
+    assert f(A16, 128, 128, A16b, A16c + 2, None) == MISALIGNED
+    assert f(A16, 128, 128, A16b + 8, A16c, None) == MISALIGNED
 
 
 def test_gemm_argument_errors(L):
@@ -97,7 +98,8 @@ def test_gemm_argument_errors(L):
     assert call(M4=10) == SHAPE
     assert call(a=None) == INVALID
     assert call(d=A16e + 8) == MISALIGNED
-    assert call(sfb=A16d + 4) == MISALIGNED
+    assert call(sfb=A16d + 2) == MISALIGNED
+    assert call(sfa=A16b + 4) == MISALIGNED
 
 
 def test_grouped_argument_errors(L):

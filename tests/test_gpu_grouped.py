@@ -30,7 +30,7 @@ def make_inputs(sizes, N, K, seed):
 
 def run_gpu(a, w, m_indices, G, fill=float("nan")):
     aq, sa = lnq.quantize_activations(a.to(DEV))
-    wq, ws = lnq.quantize_weights(w.to(DEV))
+    wq, ws = lnq.quantize_weights_grouped(w.to(DEV), G)
     N = w.shape[0] // G
     d = torch.full((a.shape[0], N), fill, dtype=torch.bfloat16, device=DEV)
     lnq.lnq_m_grouped_fp8_gemm_contiguous(aq, sa, wq, ws, torch.from_numpy(m_indices).to(DEV), G, d)
@@ -38,9 +38,16 @@ def run_gpu(a, w, m_indices, G, fill=float("nan")):
     return to_f64(d)
 
 
+def oracle_quantize_w_grouped(w, G):
+    """Each group's [N, K] weights quantized on their own (blocks never span groups)."""
+    N = w.shape[0] // G
+    parts = [oracle_quantize_w(w[g * N:(g + 1) * N]) for g in range(G)]
+    return np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts])
+
+
 def run_oracle(a, w, m_indices, G):
     qa, sa = oracle_quantize_a(a)
-    qb, sb = oracle_quantize_w(w)
+    qb, sb = oracle_quantize_w_grouped(w, G)
     return oracle.m_grouped_gemm_contiguous(qa, sa, qb, sb, m_indices, G)
 
 
@@ -89,7 +96,7 @@ def test_moe_workload_sampled():
     G = cfg.groups
     d = run_gpu(a, w, m_indices, G)
     qa, sa = oracle_quantize_a(a)
-    qb, sb = oracle_quantize_w(w)
+    qb, sb = oracle_quantize_w_grouped(w, G)
     real_rows = np.nonzero(m_indices >= 0)[0]
     rows, cols = sample_points(real_rows.size, cfg.N, 30000, seed=1, full_row=real_rows.size - 1,
                                full_col=cfg.N - 1)
