@@ -135,6 +135,53 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
     return c;
 }
 
+// One K block of the per-block FP32 promotion: acc += partial * scale, where
+// the partial is this thread's TMEM lane (kCW columns starting at taddr).
+// TMEM loads are issued one 32-column chunk ahead of the packed (f32x2) FMAs
+// that consume the previous chunk.
+//   dense:  scale = sa[row] * sb[column block of this warpgroup]
+//   decode: scale = sa[token j] * sb[weight block of the tile], per column j
+template <class C>
+__device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint32_t taddr,
+                                                const float* slot, int row, int wg) {
+    constexpr int NC = C::kCW / 32;
+    float2 s2;
+    float sb = 0.f;
+    if constexpr (!C::SWAP) {
+        const float s = slot[row] * slot[256 + (wg * C::kCW) / 128];
+        s2 = make_float2(s, s);
+    } else {
+        sb = slot[256];
+        s2 = make_float2(sb, sb);
+    }
+    uint32_t ra[32], rb[32];
+    tmem_ld32_async(taddr, ra);
+    tmem_wait_ld(ra);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        if (c + 1 < NC) {
+            if (c & 1) tmem_ld32_async(taddr + (c + 1) * 32, ra);
+            else tmem_ld32_async(taddr + (c + 1) * 32, rb);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t lo = (c & 1) ? rb[2 * i] : ra[2 * i];
+            const uint32_t hi = (c & 1) ? rb[2 * i + 1] : ra[2 * i + 1];
+            const float2 v = make_float2(__uint_as_float(lo), __uint_as_float(hi));
+            float2 sc = s2;
+            if constexpr (C::SWAP) {
+                const float2 sa = *reinterpret_cast<const float2*>(slot + c * 32 + 2 * i);
+                sc = __fmul2_rn(sa, s2);
+            }
+            acc[c * 16 + i] = __ffma2_rn(v, sc, acc[c * 16 + i]);
+        }
+        if (c + 1 < NC) {
+            if (c & 1) tmem_wait_ld(ra);
+            else tmem_wait_ld(rb);
+        }
+    }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, 1)
     k_fp8_block_gemm(const __grid_constant__ CUtensorMap map_p,
@@ -167,11 +214,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), C::kEpiThreads);
+            mbar_init(tempty_bar(b), C::kEpiThreads / 32);
         }
         for (int s = 0; s < C::kScaleStages; ++s) {
             mbar_init(sfull_bar(s), 32);
-            mbar_init(sempty_bar(s), C::kEpiThreads);
+            mbar_init(sempty_bar(s), C::kEpiThreads / 32);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0u;
@@ -345,9 +392,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
             const TileCoord tc = tile_coord<C>(args, t);
             if (tc.group < 0) continue;
-            float acc[C::kCW];
+            float2 acc[C::kCW / 2];
 #pragma unroll
-            for (int i = 0; i < C::kCW; ++i) acc[i] = 0.f;
+            for (int i = 0; i < C::kCW / 2; ++i) acc[i] = make_float2(0.f, 0.f);
             for (int kb = 0; kb < args.num_kb; ++kb) {
                 if (!mbar_wait(sfull_bar(sstage), sphase, wctx) ||
                     !mbar_wait(tfull_bar(abuf), aphase, wctx)) {
@@ -357,29 +404,13 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 tc_fence_after();
                 const float* slot = scale_slots + sstage * C::kScaleSlotFloats;
                 const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(abuf * C::BNQ + wg * C::kCW);
-                if constexpr (!C::SWAP) {
-                    const float s = slot[row] * slot[256 + (wg * C::kCW) / 128];
-#pragma unroll
-                    for (int c = 0; c < C::kCW / 32; ++c) {
-                        float v[32];
-                        tmem_ld32(taddr + c * 32, v);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(v[i], s, acc[c * 32 + i]);
-                    }
-                } else {
-                    const float sb = slot[256];
-#pragma unroll
-                    for (int c = 0; c < C::kCW / 32; ++c) {
-                        float v[32];
-                        tmem_ld32(taddr + c * 32, v);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            acc[c * 32 + i] = fmaf(v[i], slot[c * 32 + i] * sb, acc[c * 32 + i]);
-                    }
-                }
+                promote_k_block<C>(acc, taddr, slot, row, wg);
                 tc_fence_before();
-                mbar_arrive(tempty_bar(abuf));
-                mbar_arrive(sempty_bar(sstage));
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(tempty_bar(abuf));
+                    mbar_arrive(sempty_bar(sstage));
+                }
                 if (++sstage == C::kScaleStages) {
                     sstage = 0;
                     sphase ^= 1u;
@@ -398,10 +429,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         const int n = tc.q0 + wg * C::kCW + c * 8;
                         if (n < args.N) {
                             uint4 w;
-                            w.x = pack_bf16x2(acc[c * 8 + 0], acc[c * 8 + 1]);
-                            w.y = pack_bf16x2(acc[c * 8 + 2], acc[c * 8 + 3]);
-                            w.z = pack_bf16x2(acc[c * 8 + 4], acc[c * 8 + 5]);
-                            w.w = pack_bf16x2(acc[c * 8 + 6], acc[c * 8 + 7]);
+                            w.x = pack_bf16x2(acc[c * 4 + 0].x, acc[c * 4 + 0].y);
+                            w.y = pack_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
+                            w.z = pack_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
+                            w.w = pack_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
                             *reinterpret_cast<uint4*>(drow + n) = w;
                         }
                     }
@@ -412,9 +443,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < C::kCW; ++j) {
                         const int m = tc.q0 + j;
+                        const float v = (j & 1) ? acc[j >> 1].y : acc[j >> 1].x;
                         if (m < args.M)
                             args.d[static_cast<long long>(m) * args.N + n] =
-                                static_cast<uint16_t>(pack_bf16x2(acc[j], 0.f) & 0xFFFFu);
+                                static_cast<uint16_t>(pack_bf16x2(v, 0.f) & 0xFFFFu);
                     }
                 }
             }

@@ -33,15 +33,56 @@ __device__ __forceinline__ float quotient(float x, float s, bool zero_group) {
     return zero_group ? x : __fdiv_rn(x, s);
 }
 
-// Four bf16 words (8 values) to eight codes packed in two words.
-__device__ __forceinline__ uint2 quantize8(const uint4& raw, float s, bool zero_group) {
+// True when the E4M3 rounding of t could differ from the E4M3 rounding of a
+// value at most 3 fp32 ulps away: t within 4 ulps of a rounding midpoint of the
+// normal E4M3 range (the 20 fp32 mantissa bits below the 3 E4M3 mantissa bits
+// within 4 of 0x80000), or 0 < |t| < 2^-6 (E4M3 subnormal range, where the
+// midpoints sit elsewhere).  Binade edges hold no midpoint, so one test covers
+// every exponent.
+__device__ __forceinline__ bool near_e4m3_midpoint(float t) {
+    const uint32_t b = __float_as_uint(t);
+    const bool near_mid = ((b & 0xFFFFFu) - 0x7FFFCu) < 9u;
+    const bool small = ((b & 0x7FFFFFFFu) - 1u) < 0x3C7FFFFFu;
+    return near_mid || small;
+}
+
+// Eight quotients x/s whose E4M3 codes equal those of the correctly rounded
+// quotients.  The fast path multiplies by r = RN(1/s): |x*r - x/s| is at most
+// 2^-23 |x/s| + 2^-48 |x/s|, so x*r and RN(x/s) are at most 3 ulps apart and
+// round to the same E4M3 code unless x*r lies within 4 ulps of an E4M3
+// midpoint (a rounding test in the manner of Ziv's correctly rounded
+// elementary functions).  Then, and for tiny scales where r is inexact or
+// infinite, the eight values take the IEEE division instead.
+__device__ __forceinline__ void quotients8(const uint4& raw, float s, float r, bool zero_group,
+                                           bool exact_group, float (&t)[8]) {
+    t[0] = bf16_lo(raw.x);
+    t[1] = bf16_hi(raw.x);
+    t[2] = bf16_lo(raw.y);
+    t[3] = bf16_hi(raw.y);
+    t[4] = bf16_lo(raw.z);
+    t[5] = bf16_hi(raw.z);
+    t[6] = bf16_lo(raw.w);
+    t[7] = bf16_hi(raw.w);
+    if (zero_group) return;  // all +-0: the codes keep the signs
+    float f[8];
+    bool risky = exact_group;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        f[j] = t[j] * r;
+        risky |= near_e4m3_midpoint(f[j]);
+    }
+    if (risky) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] = __fdiv_rn(t[j], s);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t[j] = f[j];
+}
+
+__device__ __forceinline__ uint2 pack8(const float (&t)[8]) {
     uint2 out;
-    out.x = e4m3x2(quotient(bf16_lo(raw.x), s, zero_group), quotient(bf16_hi(raw.x), s, zero_group)) |
-            (e4m3x2(quotient(bf16_lo(raw.y), s, zero_group), quotient(bf16_hi(raw.y), s, zero_group))
-             << 16);
-    out.y = e4m3x2(quotient(bf16_lo(raw.z), s, zero_group), quotient(bf16_hi(raw.z), s, zero_group)) |
-            (e4m3x2(quotient(bf16_lo(raw.w), s, zero_group), quotient(bf16_hi(raw.w), s, zero_group))
-             << 16);
+    out.x = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
+    out.y = e4m3x2(t[4], t[5]) | (e4m3x2(t[6], t[7]) << 16);
     return out;
 }
 
@@ -101,8 +142,9 @@ __global__ void __launch_bounds__(256)
         const float s = __fdiv_rn(amax, 448.0f);
         const int64_t r = row0 + warp + 8 * i;
         if (r < M && group_ok) {
-            const uint2 codes = quantize8(raw[i], s, amax == 0.0f);
-            *reinterpret_cast<uint2*>(q + r * ld_q + col) = codes;
+            float t[8];
+            quotients8(raw[i], s, __frcp_rn(s), amax == 0.0f, !(s >= 0x1p-125f), t);
+            *reinterpret_cast<uint2*>(q + r * ld_q + col) = pack8(t);
         }
         if ((lane & 15) == 0) s_scale[half][warp + 8 * i] = s;
     }

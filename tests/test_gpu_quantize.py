@@ -151,3 +151,42 @@ def test_moe_weights_full_size():
     cfg = synthetic.MOE
     w = synthetic.gaussian_bf16((cfg.groups * cfg.N, cfg.K), cfg.w_std, cfg.w_seed)
     assert_same_w(w)
+
+
+def near_midpoint_rows(max_rows=4096):
+    """Rows whose quotients x/s land near E4M3 rounding midpoints under scales that are
+    not powers of two: found by brute force over bf16 amax in [1, 2) x every bf16 x up
+    to amax.  Kept: x where RN(x * RN(1/s)) and RN(x / s) take different E4M3 codes, and
+    x where RN(x / s) is within 8 ulps of a midpoint."""
+    amax_bits = np.arange(0x3F80, 0x4000, dtype=np.uint16)           # bf16 values in [1, 2)
+    x_bits = np.arange(0, 0x4000, dtype=np.uint16)                   # bf16 values in [0, 2)
+    xs = (x_bits.astype(np.uint32) << 16).view(np.float32)
+    chosen = []
+    for ab in amax_bits:
+        amax = np.float32((np.uint32(ab) << 16).view(np.float32))
+        s = np.float32(amax / np.float32(448.0))
+        r = np.float32(np.float32(1.0) / s)
+        x = xs[xs <= amax]
+        t = (x / s).astype(np.float32)
+        f = (x * r).astype(np.float32)
+        ct = torch.from_numpy(t).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        cf = torch.from_numpy(f).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        low = t.view(np.uint32) & 0xFFFFF
+        near = np.abs(low.astype(np.int64) - 0x80000) <= 8
+        pick = x[(ct != cf) | near]
+        for i in range(0, pick.size, 127):
+            chosen.append((amax, pick[i:i + 127]))
+    rows = chosen[:max_rows]
+    out = np.zeros((len(rows), 128), np.float64)
+    for k, (amax, vals) in enumerate(rows):
+        out[k, 0] = amax
+        out[k, 1:1 + vals.size] = vals
+        out[k, 1 + vals.size:] = -vals[0] if vals.size else 0.0
+    return out
+
+
+def test_quotients_near_e4m3_midpoints():
+    x = near_midpoint_rows()
+    assert x.shape[0] > 100
+    for scale in (1.0, -3.0, 2.0 ** 40, 2.0 ** -60):
+        assert_same_a(torch.tensor(x * scale).to(torch.bfloat16))
