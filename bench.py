@@ -299,6 +299,7 @@ def run_ours(args, world, rank, local):
         lnq_build.build()
     barrier(dist)
     lnq.lib()
+    lnq.lnq_set_dense_cta_pairs(args.cta_pairs)
 
     cfgs, kind = workload_units(args.workload)
     units = [Grouped(c, dev) if kind == "grouped" else Linear(c, dev) for c in cfgs]
@@ -433,6 +434,7 @@ def run_ours(args, world, rank, local):
         "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out",
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, bf16)",
         "config": {"workload": args.workload, "desc": WORKLOAD_DESC[args.workload],
+                   "dense_cta_pairs": bool(args.cta_pairs),
                    "parallelism": f"replicas x{world} (independent tokens per rank)",
                    "l2": "working set per step > 126 MB L2; no extra flush"},
         "roofline": roof,
@@ -566,6 +568,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cta-pairs", action="store_true",
+                    help="run dense GEMMs (M > 128, N >= 256) on CTA pairs")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -171,6 +171,15 @@ lnq_status lnq_get_last_device_error(void* stream);
  */
 lnq_status lnq_selftest_wait_timeout(int64_t timeout_ns, void* stream);
 
+/*
+ * Tuning knob (process-wide, default 0): when non-zero, dense GEMMs with
+ * M > 128 and N >= 256 run on pairs of CTAs (a cluster of two sharing one
+ * tcgen05 MMA of 256 x 256, each CTA loading half of the weight tile) instead
+ * of one CTA per 128 x 256 tile.  Results are the same up to FP32 summation
+ * order.  Returns the previous setting.
+ */
+int32_t lnq_set_dense_cta_pairs(int32_t enable);
+
 /* Version of this ABI (major*10000 + minor*100 + patch). */
 int32_t lnq_abi_version(void);
 

@@ -28,7 +28,7 @@ __all__ = [
     "LnqError", "library_path", "lib",
     "lnq_quantize_fp8_groups", "lnq_quantize_fp8_blocks", "lnq_fp8_block_gemm_nt",
     "lnq_m_grouped_fp8_gemm_contiguous", "lnq_get_last_device_error", "lnq_status_string",
-    "lnq_selftest_wait_timeout", "quantize_activations", "quantize_weights",
+    "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "quantize_activations", "quantize_weights",
     "quantize_weights_grouped", "linear",
     "m_grouped_linear", "ceil4",
 ]
@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.lnq_status_string.argtypes = [ctypes.c_int]
         L.lnq_status_string.restype = ctypes.c_char_p
         L.lnq_abi_version.restype = ctypes.c_int32
+        L.lnq_set_dense_cta_pairs.argtypes = [ctypes.c_int32]
+        L.lnq_set_dense_cta_pairs.restype = ctypes.c_int32
         _lib = L
         return L
 
@@ -189,6 +191,11 @@ def lnq_m_grouped_fp8_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: tor
 def lnq_get_last_device_error(stream=None) -> int:
     """Synchronizes the stream; returns (and clears) the device-reported status."""
     return int(lib().lnq_get_last_device_error(_stream(stream)))
+
+
+def lnq_set_dense_cta_pairs(enable: bool) -> bool:
+    """Route dense GEMMs (M > 128, N >= 256) to CTA pairs; returns the previous setting."""
+    return bool(lib().lnq_set_dense_cta_pairs(1 if enable else 0))
 
 
 def lnq_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:

@@ -9,6 +9,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "lnq.h"
@@ -107,7 +108,8 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
         if (st == LNQ_OK) st = encode_e4m3_map(&map_q, act, act_rows, K, C::BNQ);
     } else {
         st = encode_e4m3_map(&map_p, act, act_rows, K, C::kP);
-        if (st == LNQ_OK) st = encode_e4m3_map(&map_q, wgt, wgt_rows, K, C::BNQ);
+        if (st == LNQ_OK)
+            st = encode_e4m3_map(&map_q, wgt, wgt_rows, K, C::PAIR ? C::kSliceQRows : C::kQRowsPerCta);
     }
     if (st != LNQ_OK) return st;
     static bool attr_set[kMaxDevices] = {};
@@ -121,6 +123,34 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
     }
     args.status = dev.status;
     args.timeout_ns = kDefaultTimeoutNs;
+    if constexpr (C::PAIR) {
+        // clusters of two CTAs; as many pairs as can be resident at once
+        static int max_clusters[kMaxDevices] = {};
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.blockDim = dim3(C::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (max_clusters[devno] == 0) {
+            int n = 0;
+            cfg.gridDim = dim3(2 * (dev.sm_count / 2), 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&n, k_fp8_block_gemm<C>, &cfg) != cudaSuccess || n <= 0)
+                return LNQ_ERR_CUDA;
+            max_clusters[devno] = n;
+        }
+        const int pairs = args.num_tiles < max_clusters[devno] ? args.num_tiles : max_clusters[devno];
+        if (pairs <= 0) return LNQ_OK;
+        cfg.gridDim = dim3(2 * pairs, 1, 1);
+        if (cudaLaunchKernelEx(&cfg, k_fp8_block_gemm<C>, map_p, map_q, args) != cudaSuccess)
+            return LNQ_ERR_CUDA;
+        return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+    }
     const int grid = args.num_tiles < dev.sm_count ? args.num_tiles : dev.sm_count;
     if (grid <= 0) return LNQ_OK;
     k_fp8_block_gemm<C><<<grid, C::kThreads, C::kSmemBytes, stream>>>(map_p, map_q, args);
@@ -129,6 +159,10 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
 
 // Tile configurations (P = MMA M slot, Q = MMA N slot).
 using CfgDense256 = GemmCfg<256, 4, 2, false, false>;
+using CfgPair256 = GemmCfg<256, 6, 2, false, false, true>;
+
+// Dense GEMMs with M > 128 and N >= 256 run on CTA pairs only when enabled.
+std::atomic<int> g_dense_pairs{0};
 using CfgDense128 = GemmCfg<128, 6, 2, false, false>;
 using CfgGrouped256 = GemmCfg<256, 4, 2, false, true>;
 using CfgGrouped128 = GemmCfg<128, 6, 2, false, true>;
@@ -145,6 +179,11 @@ using namespace lnq;
 extern "C" {
 
 int32_t lnq_abi_version(void) { return 10000; }
+
+int32_t lnq_set_dense_cta_pairs(int32_t enable) {
+    const int previous = g_dense_pairs.exchange(enable ? 1 : 0);
+    return previous;
+}
 
 const char* lnq_status_string(lnq_status s) {
     switch (s) {
@@ -166,7 +205,6 @@ lnq_status lnq_quantize_fp8_groups(const void* x_bf16, int64_t M, int64_t K, int
     if (K % 128 != 0) return LNQ_ERR_UNSUPPORTED_SHAPE;
     if (ld_x < K || ld_q < K) return LNQ_ERR_INVALID_ARG;
     if (M4 < ((M + 3) / 4) * 4 || M4 % 4 != 0 || M4 > kMaxRows) return LNQ_ERR_UNSUPPORTED_SHAPE;
-    if (K / 256 + 1 > 65535) return LNQ_ERR_UNSUPPORTED_SHAPE;
     if (M4 == 0) return LNQ_OK;
     if (!sfa || (M > 0 && (!x_bf16 || !q_e4m3))) return LNQ_ERR_INVALID_ARG;
     if (!aligned16(x_bf16) || !aligned16(q_e4m3) || !aligned16(sfa) || ld_x % 8 != 0 ||
@@ -175,11 +213,52 @@ lnq_status lnq_quantize_fp8_groups(const void* x_bf16, int64_t M, int64_t K, int
     DeviceInfo* dev = nullptr;
     lnq_status st = device_info(&dev);
     if (st != LNQ_OK) return st;
-    dim3 grid(static_cast<unsigned>((M4 + kQuantRowsPerCta - 1) / kQuantRowsPerCta),
-              static_cast<unsigned>((K + kQuantColsPerCta - 1) / kQuantColsPerCta));
-    k_quantize_groups<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint16_t*>(x_bf16), M, K, ld_x, static_cast<uint8_t*>(q_e4m3), ld_q, sfa,
-        M4);
+    if (M == 0) {
+        // no rows: only the pad scales, which are zero
+        return cudaMemsetAsync(sfa, 0, static_cast<size_t>(K / 128) * M4 * sizeof(float),
+                               static_cast<cudaStream_t>(stream)) == cudaSuccess
+                   ? LNQ_OK
+                   : LNQ_ERR_CUDA;
+    }
+    // bf16 [M][ld_x] as a 2-D tensor of K columns, box of 256 columns x 32 rows
+    CUtensorMap xmap;
+    {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_x) * 2};
+        cuuint32_t box[2] = {static_cast<cuuint32_t>(kQuantCols), static_cast<cuuint32_t>(kQuantRows)};
+        cuuint32_t estr[2] = {1u, 1u};
+        if (g_encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x_bf16), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return LNQ_ERR_CUDA;
+    }
+    QuantArgs qa{};
+    qa.q = static_cast<uint8_t*>(q_e4m3);
+    qa.sfa = sfa;
+    qa.status = dev->status;
+    qa.timeout_ns = kDefaultTimeoutNs;
+    qa.M = M;
+    qa.K = K;
+    qa.ld_q = ld_q;
+    qa.M4 = M4;
+    qa.col_tiles = static_cast<int>((K + kQuantCols - 1) / kQuantCols);
+    const long long tiles = ((M4 + kQuantRows - 1) / kQuantRows) * static_cast<long long>(qa.col_tiles);
+    if (tiles > 0x7FFFFFFFLL) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    qa.num_tiles = static_cast<int>(tiles);
+    static bool attr_set[kMaxDevices] = {};
+    int devno = 0;
+    cudaGetDevice(&devno);
+    if (!attr_set[devno]) {
+        if (cudaFuncSetAttribute(k_quantize_groups, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kQuantSmemBytes) != cudaSuccess)
+            return LNQ_ERR_CUDA;
+        attr_set[devno] = true;
+    }
+    const long long max_ctas = 3LL * dev->sm_count;
+    const int grid = static_cast<int>(tiles < max_ctas ? tiles : max_ctas);
+    k_quantize_groups<<<grid, kQuantThreads, kQuantSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+        xmap, qa);
     return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
 }
 
@@ -236,6 +315,13 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
         args.tiles_q = static_cast<int>((M + 63) / 64);
         args.num_tiles = args.tiles_p * args.tiles_q;
         return launch_gemm<CfgSwap64>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
+    }
+    if (N >= 256 && M > 128 && g_dense_pairs.load(std::memory_order_relaxed)) {
+        // pairs of CTAs on 256 x 256 tiles
+        args.tiles_p = static_cast<int>((M + 255) / 256);
+        args.tiles_q = static_cast<int>((N + 255) / 256);
+        args.num_tiles = args.tiles_p * args.tiles_q;
+        return launch_gemm<CfgPair256>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
     }
     args.tiles_p = static_cast<int>((M + 127) / 128);
     if (N >= 256) {

@@ -4,11 +4,15 @@
 // (deepgemm-rust README, "What's implemented": per-(1x128) activation scales
 // x per-(128x128) weight scales, FP32 promotion, BF16 out).
 //
-// One persistent, warp-specialized kernel serves three shapes:
-//   * dense (M > 64): the MMA's M slot ("P operand") holds 128 activation rows,
-//     its N slot ("Q operand") BNQ weight rows;
-//   * M-grouped contiguous (MoE): as dense, each 128-row block of activations
-//     takes the weights of the group named by its first row's id
+// One persistent, warp-specialized kernel serves four shapes:
+//   * dense, CTA pairs (M > 64, PAIR): two CTAs of a cluster run one
+//     tcgen05.mma.cta_group::2 of 256 x 256; each CTA loads its own 128
+//     activation rows and 128 of the 256 weight rows per K block, so each
+//     CTA streams 32 KB instead of 48 KB per 128 x 256 of output;
+//   * dense, single CTA: 128 activation rows in the MMA's M slot ("P
+//     operand"), BNQ weight rows in its N slot ("Q operand");
+//   * M-grouped contiguous (MoE): as single-CTA dense, each 128-row block of
+//     activations takes the weights of the group named by its first row's id
 //     (deepgemm-rust README, "Grouped (contiguous) MoE GEMM");
 //   * decode (M <= 64, "swap AB"): the weights fill the 128-row M slot and the
 //     few tokens the N slot, so the tensor core is not idle on padding rows.
@@ -16,9 +20,10 @@
 // Roles (warps of one CTA):
 //   warp 0      TMA producer: P and Q tiles of one 128-wide K block per stage
 //               into a ring of shared-memory stages (128-byte swizzle).
-//   warp 1      allocates tensor memory; one lane issues tcgen05.mma
-//               kind::f8f6f4 (E4M3 x E4M3 -> FP32), 4 MMAs of K=32 per K block,
-//               into one of two TMEM accumulators that alternate per K block.
+//   warp 1      allocates tensor memory; one lane (of the pair's first CTA)
+//               issues tcgen05.mma kind::f8f6f4 (E4M3 x E4M3 -> FP32), 4 MMAs
+//               of K=32 per K block, into one of two TMEM accumulators that
+//               alternate per K block.
 //   warp 2      scale producer: loads the K block's activation and weight
 //               scales into a small shared-memory ring.
 //   warps 4..   epilogue: per K block, reads the FP32 partial product from TMEM
@@ -49,30 +54,35 @@ struct GemmArgs {
     int num_kb;       // K / 128
     int nb;           // ceil(N / 128): weight scale rows per group
     int num_groups;   // grouped only
-    int tiles_p;      // tiles along the MMA M slot
+    int tiles_p;      // tiles along the MMA M slot (of 256 rows for PAIR)
     int tiles_q;      // tiles along the MMA N slot
     int num_tiles;
 };
 
 constexpr unsigned int kStatusBadGroup = 2u;
 
-template <int BNQ_, int STAGES_, int EPI_WG_, bool SWAP_, bool GROUPED_>
+template <int BNQ_, int STAGES_, int EPI_WG_, bool SWAP_, bool GROUPED_, bool PAIR_ = false,
+          int SLICES_ = 1>
 struct GemmCfg {
-    static constexpr int BNQ = BNQ_;
+    static constexpr int BNQ = BNQ_;   // MMA N (the whole pair's N for PAIR)
     static constexpr int STAGES = STAGES_;
     static constexpr int EPI_WG = EPI_WG_;
     static constexpr bool SWAP = SWAP_;
     static constexpr bool GROUPED = GROUPED_;
+    static constexpr bool PAIR = PAIR_;
     static_assert(!(SWAP && GROUPED), "decode configuration is dense only");
-    static_assert(BNQ % 16 == 0 && BNQ >= 16 && BNQ <= 256, "MMA N for M=128");
+    static_assert(!(PAIR && (SWAP || GROUPED)), "CTA pairs serve the dense configuration");
+    static_assert(BNQ % 16 == 0 && BNQ >= 16 && BNQ <= 256, "MMA N for M=128/256");
     static_assert(!SWAP || EPI_WG == 1, "decode epilogue: one thread per weight row");
     static_assert(!SWAP || BNQ % 32 == 0, "decode tiles read TMEM in 32-column chunks");
     static_assert(SWAP || BNQ % 128 == 0, "dense tiles cover whole 128-column scale blocks");
 
-    static constexpr int kP = 128;                // MMA M
+    static constexpr int kP = 128;                // P rows per CTA (MMA M per CTA)
+    static constexpr int kTileM = PAIR ? 256 : 128;  // P rows per tile
     static constexpr int kBK = 128;               // K elements (bytes) per stage
     static constexpr int kPBytes = kP * kBK;
-    static constexpr int kQBytes = BNQ * kBK;
+    static constexpr int kQRowsPerCta = PAIR ? BNQ / 2 : BNQ;
+    static constexpr int kQBytes = kQRowsPerCta * kBK;
     static constexpr int kScaleStages = 8;
     static constexpr int kCW = BNQ / EPI_WG;      // accumulator columns per epilogue thread
     static constexpr int kEpiThreads = 128 * EPI_WG;
@@ -80,8 +90,19 @@ struct GemmCfg {
     static constexpr int kTmemCols = (2 * BNQ < 32) ? 32 : 2 * BNQ;
     static constexpr int kSbPerTile = SWAP ? 1 : BNQ / 128;
     static constexpr int kSaPerTile = SWAP ? BNQ : kP;
-    static constexpr uint32_t kIdesc = f8f6f4_e4m3_idesc(kP, BNQ);
     static constexpr bool kRegSplit = (!SWAP && kCW == 128);
+    // With kSlices > 1 each epilogue warpgroup owns one column slice of the
+    // accumulator: the MMA of a K block is issued slice by slice (N = BNQ /
+    // kSlices), each slice with its own full/empty barriers, so the tensor core
+    // may run up to 2*kSlices-1 slices ahead of the promotion.  With kSlices = 1
+    // one MMA of N = BNQ covers the K block and all epilogue warps release it.
+    static constexpr int kSlices = SLICES_;
+    static_assert(kSlices == 1 || kSlices == EPI_WG, "slices follow the epilogue warpgroups");
+    static constexpr int kSliceN = BNQ / kSlices;                   // MMA N per slice
+    static constexpr int kSliceQRows = PAIR ? kSliceN / 2 : kSliceN;  // B rows per slice per CTA
+    static constexpr int kEpiWarpsPerSlice = (PAIR ? 2 : 1) * 4 * (EPI_WG / kSlices);
+    static constexpr uint32_t kIdesc = f8f6f4_e4m3_idesc(PAIR ? 256 : 128, kSliceN);
+    static_assert(kSliceN % 16 == 0 && kSliceQRows % 8 == 0, "slice shapes");
 
     // shared-memory layout (offsets from a 1024-byte aligned base)
     static constexpr int kOffP = 0;
@@ -89,7 +110,7 @@ struct GemmCfg {
     static constexpr int kOffScale = kOffQ + STAGES * kQBytes;
     static constexpr int kScaleSlotFloats = 256 + 4;
     static constexpr int kOffBar = kOffScale + kScaleStages * kScaleSlotFloats * 4;
-    static constexpr int kNumBars = 2 * STAGES + 4 + 2 * kScaleStages + 1;
+    static constexpr int kNumBars = 2 * STAGES + 4 * kSlices + 2 * kScaleStages + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -97,13 +118,14 @@ struct GemmCfg {
 };
 
 struct TileCoord {
-    int p0;     // first row of the P operand (activation row, or weight row for SWAP)
-    int q0;     // first row of the Q operand (weight row within the group, or token)
+    int p0;     // first row of this CTA's P operand (activation row, or weight row for SWAP)
+    int q0;     // first output column of the tile (weight row within the group, or token)
     int group;  // grouped: group id of the tile, -1 skip; else 0
 };
 
+// Tile t of this CTA (or of this CTA pair; `rank` is the CTA's rank in the pair).
 template <class C>
-__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32_t rank) {
     TileCoord c;
     if constexpr (C::SWAP) {
         c.p0 = (t % a.tiles_p) * C::kP;
@@ -120,15 +142,15 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
             c.group = -1;
         }
     } else {
-        // bands of 16 row blocks: a wave of tiles shares 16 activation blocks
+        // bands of row tiles: a wave of tiles shares a band of activation rows
         // and a few weight column tiles
-        constexpr int kBand = 16;
+        constexpr int kBand = C::PAIR ? 8 : 16;
         const int band_tiles = kBand * a.tiles_q;
         const int band = t / band_tiles;
         const int first = band * kBand;
         const int rows = min(a.tiles_p - first, kBand);
         const int r = t - band * band_tiles;
-        c.p0 = (first + r % rows) * C::kP;
+        c.p0 = (first + r % rows) * C::kTileM + static_cast<int>(rank) * C::kP;
         c.q0 = (r / rows) * C::BNQ;
         c.group = 0;
     }
@@ -136,49 +158,66 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
 }
 
 // One K block of the per-block FP32 promotion: acc += partial * scale, where
-// the partial is this thread's TMEM lane (kCW columns starting at taddr).
-// TMEM loads are issued one 32-column chunk ahead of the packed (f32x2) FMAs
-// that consume the previous chunk.
+// the partial is this thread's TMEM lane (kCW columns starting at taddr).  The
+// columns are read in chunks of 64 (32 when the slice is narrower); `release`
+// runs as soon as the last chunk has arrived in registers, before its FMAs, so
+// the tensor core may overwrite the slice early.
 //   dense:  scale = sa[row] * sb[column block of this warpgroup]
 //   decode: scale = sa[token j] * sb[weight block of the tile], per column j
-template <class C>
+template <class C, int W>
+__device__ __forceinline__ void promote_chunk(float2 (&acc)[C::kCW / 2], const uint32_t (&r)[W],
+                                              int col0, const float* slot, float2 s2) {
+#pragma unroll
+    for (int i = 0; i < W / 2; ++i) {
+        const float2 v = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+        float2 sc = s2;
+        if constexpr (C::SWAP) {
+            const float2 sa = *reinterpret_cast<const float2*>(slot + col0 + 2 * i);
+            sc = __fmul2_rn(sa, s2);
+        }
+        acc[col0 / 2 + i] = __ffma2_rn(v, sc, acc[col0 / 2 + i]);
+    }
+}
+
+template <class C, class Release>
 __device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint32_t taddr,
-                                                const float* slot, int row, int wg) {
-    constexpr int NC = C::kCW / 32;
+                                                const float* slot, int row, int wg,
+                                                Release&& release) {
     float2 s2;
-    float sb = 0.f;
     if constexpr (!C::SWAP) {
         const float s = slot[row] * slot[256 + (wg * C::kCW) / 128];
         s2 = make_float2(s, s);
     } else {
-        sb = slot[256];
+        const float sb = slot[256];
         s2 = make_float2(sb, sb);
     }
+    // 32-column chunks, each load issued one chunk ahead of the FMAs
+    constexpr int NC = C::kCW / 32;
     uint32_t ra[32], rb[32];
     tmem_ld32_async(taddr, ra);
     tmem_wait_ld(ra);
+    if (NC == 1) release();
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
         if (c + 1 < NC) {
             if (c & 1) tmem_ld32_async(taddr + (c + 1) * 32, ra);
             else tmem_ld32_async(taddr + (c + 1) * 32, rb);
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t lo = (c & 1) ? rb[2 * i] : ra[2 * i];
-            const uint32_t hi = (c & 1) ? rb[2 * i + 1] : ra[2 * i + 1];
-            const float2 v = make_float2(__uint_as_float(lo), __uint_as_float(hi));
-            float2 sc = s2;
-            if constexpr (C::SWAP) {
-                const float2 sa = *reinterpret_cast<const float2*>(slot + c * 32 + 2 * i);
-                sc = __fmul2_rn(sa, s2);
-            }
-            acc[c * 16 + i] = __ffma2_rn(v, sc, acc[c * 16 + i]);
-        }
+        if (c & 1) promote_chunk<C, 32>(acc, rb, c * 32, slot, s2);
+        else promote_chunk<C, 32>(acc, ra, c * 32, slot, s2);
         if (c + 1 < NC) {
             if (c & 1) tmem_wait_ld(ra);
             else tmem_wait_ld(rb);
+            if (c + 2 == NC) release();
         }
+    }
+}
+
+// Spin for `ns` nanoseconds (bounded); lets copies already issued by a CTA
+// that gave up land before it leaves.
+__device__ __forceinline__ void settle_ns(uint64_t ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < ns) {
     }
 }
 
@@ -196,25 +235,32 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     const uint32_t bars = s_base + C::kOffBar;
     auto full_bar = [&](int s) { return bars + 8u * s; };
     auto empty_bar = [&](int s) { return bars + 8u * (C::STAGES + s); };
+    // accumulator slot = buffer * kSlices + slice
     auto tfull_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + b); };
-    auto tempty_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + 2 + b); };
-    auto sfull_bar = [&](int s) { return bars + 8u * (2 * C::STAGES + 4 + s); };
-    auto sempty_bar = [&](int s) { return bars + 8u * (2 * C::STAGES + 4 + C::kScaleStages + s); };
-    const uint32_t drain_bar = bars + 8u * (2 * C::STAGES + 4 + 2 * C::kScaleStages);
+    auto tempty_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + 2 * C::kSlices + b); };
+    auto sfull_bar = [&](int s) { return bars + 8u * (2 * C::STAGES + 4 * C::kSlices + s); };
+    auto sempty_bar = [&](int s) {
+        return bars + 8u * (2 * C::STAGES + 4 * C::kSlices + C::kScaleStages + s);
+    };
+    const uint32_t drain_bar = bars + 8u * (2 * C::STAGES + 4 * C::kSlices + 2 * C::kScaleStages);
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile uint32_t* abort_flag = misc + 1;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // CTA pairs: rank in the pair; tiles are numbered per pair
+    const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
+    const int unit = C::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int units = C::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < 2 * C::kSlices; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), C::kEpiThreads / 32);
+            mbar_init(tempty_bar(b), C::kEpiWarpsPerSlice);
         }
         for (int s = 0; s < C::kScaleStages; ++s) {
             mbar_init(sfull_bar(s), 32);
@@ -225,11 +271,17 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(misc), C::kTmemCols);
-        tmem_relinquish();
+        if constexpr (C::PAIR) {
+            tmem_alloc_pair(smem_u32(misc), C::kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(misc), C::kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (C::PAIR) cluster_sync();  // the peer's barriers exist before any remote signal
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
 
@@ -250,8 +302,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             uint32_t phase = 0;
             uint32_t filled = 0, fill_parity = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
-                const TileCoord tc = tile_coord<C>(args, t);
+            for (int t = unit; t < args.num_tiles && ok; t += units) {
+                const TileCoord tc = tile_coord<C>(args, t, rank);
                 if (tc.group < 0) continue;
                 int p_row, q_row;
                 if constexpr (C::SWAP) {
@@ -259,16 +311,29 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     q_row = tc.q0;
                 } else {
                     p_row = tc.p0;
-                    q_row = tc.group * args.N + tc.q0;
+                    q_row = tc.group * args.N + tc.q0 + static_cast<int>(rank) * C::kSliceQRows;
                 }
                 for (int kb = 0; kb < args.num_kb; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, wctx)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(full_bar(stage), C::kPBytes + C::kQBytes);
-                    tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK, p_row);
-                    tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK, q_row);
+                    if constexpr (C::PAIR) {
+                        // both CTAs' bytes complete on the first CTA's full barrier
+                        if (rank == 0)
+                            mbar_arrive_expect_tx(full_bar(stage), 2 * (C::kPBytes + C::kQBytes));
+                        const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
+                        tma_load_2d_pair(sP + stage * C::kPBytes, &map_p, leader_full, kb * C::kBK, p_row);
+                        // slice h of the tile's N: this CTA holds its kSliceQRows rows of it
+#pragma unroll
+                        for (int h = 0; h < C::kSlices; ++h)
+                            tma_load_2d_pair(sQ + stage * C::kQBytes + h * C::kSliceQRows * C::kBK, &map_q,
+                                             leader_full, kb * C::kBK, q_row + h * C::kSliceN);
+                    } else {
+                        mbar_arrive_expect_tx(full_bar(stage), C::kPBytes + C::kQBytes);
+                        tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK, p_row);
+                        tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK, q_row);
+                    }
                     filled |= 1u << stage;
                     fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
                     if (++stage == C::STAGES) {
@@ -279,38 +344,69 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             }
             if (!ok) {
                 // let the copies already issued land before the CTA can exit
-                WaitCtx drain = wctx;
-                uint32_t never = 0u;
-                drain.abort = &never;
-                for (int s = 0; s < C::STAGES; ++s)
-                    if (filled & (1u << s)) (void)mbar_wait(full_bar(s), (fill_parity >> s) & 1u, drain);
+                if (C::PAIR && rank != 0) {
+                    settle_ns(200000);
+                } else {
+                    WaitCtx drain = wctx;
+                    uint32_t never = 0u;
+                    drain.abort = &never;
+                    for (int s = 0; s < C::STAGES; ++s)
+                        if (filled & (1u << s))
+                            (void)mbar_wait(full_bar(s), (fill_parity >> s) & 1u, drain);
+                    if (C::PAIR) settle_ns(200000);
+                }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             int stage = 0, abuf = 0;
             uint32_t phase = 0, aphase = 0;
             bool ok = true, issued = false;
-            for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
-                const TileCoord tc = tile_coord<C>(args, t);
+            for (int t = unit; t < args.num_tiles && ok; t += units) {
+                const TileCoord tc = tile_coord<C>(args, t, 0);
                 if (tc.group < 0) continue;
-                for (int kb = 0; kb < args.num_kb; ++kb) {
-                    if (!mbar_wait(tempty_bar(abuf), aphase ^ 1u, wctx) ||
-                        !mbar_wait(full_bar(stage), phase, wctx)) {
+                for (int kb = 0; kb < args.num_kb && ok; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, wctx)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::BNQ);
                     const uint64_t adesc = sw128_kmajor_desc(sP + stage * C::kPBytes);
-                    const uint64_t bdesc = sw128_kmajor_desc(sQ + stage * C::kQBytes);
 #pragma unroll
-                    for (int k = 0; k < C::kBK / 32; ++k)
-                        mma_f8f6f4(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc, k > 0 ? 1u : 0u);
-                    mma_commit(empty_bar(stage));
-                    mma_commit(tfull_bar(abuf));
-                    issued = true;
+                    for (int h = 0; h < C::kSlices; ++h) {
+                        const int slot = abuf * C::kSlices + h;
+                        if (!mbar_wait(tempty_bar(slot), aphase ^ 1u, wctx)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::BNQ + h * C::kSliceN);
+                        const uint64_t bdesc =
+                            sw128_kmajor_desc(sQ + stage * C::kQBytes + h * C::kSliceQRows * C::kBK);
+                        if constexpr (C::PAIR) {
+#pragma unroll
+                            for (int k = 0; k < C::kBK / 32; ++k)
+                                mma_f8f6f4_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
+                                                k > 0 ? 1u : 0u);
+                            mma_commit_pair(mapa_shared(tfull_bar(slot), 0));
+                            mma_commit_pair(mapa_shared(tfull_bar(slot), 1));
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < C::kBK / 32; ++k)
+                                mma_f8f6f4(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
+                                           k > 0 ? 1u : 0u);
+                            mma_commit(tfull_bar(slot));
+                        }
+                        issued = true;
+                    }
+                    if (!ok) break;
+                    // the stage is free once every slice's MMAs have read it
+                    if constexpr (C::PAIR) {
+                        mma_commit_pair(mapa_shared(empty_bar(stage), 0));
+                        mma_commit_pair(mapa_shared(empty_bar(stage), 1));
+                    } else {
+                        mma_commit(empty_bar(stage));
+                    }
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -321,7 +417,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             }
             if (issued) {
                 // every MMA this thread issued completes before TMEM is released
-                mma_commit(drain_bar);
+                if constexpr (C::PAIR) mma_commit_pair(mapa_shared(drain_bar, 0));
+                else mma_commit(drain_bar);
                 WaitCtx drain = wctx;
                 uint32_t never = 0u;
                 drain.abort = &never;
@@ -335,8 +432,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         bool ok = true;
         constexpr int kBatch = 4;
         constexpr int kSaLanes = C::kSaPerTile / 4;  // lanes that load a float4 of sa
-        for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
-            const TileCoord tc = tile_coord<C>(args, t);
+        for (int t = unit; t < args.num_tiles && ok; t += units) {
+            const TileCoord tc = tile_coord<C>(args, t, rank);
             if (tc.group < 0) continue;
             // activation rows of the tile (tokens for SWAP) and weight scale rows
             const long long a_row0 = C::SWAP ? tc.q0 : tc.p0;
@@ -389,27 +486,41 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         int sstage = 0, abuf = 0;
         uint32_t sphase = 0, aphase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
-            const TileCoord tc = tile_coord<C>(args, t);
+        for (int t = unit; t < args.num_tiles && ok; t += units) {
+            const TileCoord tc = tile_coord<C>(args, t, rank);
             if (tc.group < 0) continue;
             float2 acc[C::kCW / 2];
 #pragma unroll
             for (int i = 0; i < C::kCW / 2; ++i) acc[i] = make_float2(0.f, 0.f);
             for (int kb = 0; kb < args.num_kb; ++kb) {
+                const int slot_id = abuf * C::kSlices + (C::kSlices == 1 ? 0 : wg);
                 if (!mbar_wait(sfull_bar(sstage), sphase, wctx) ||
-                    !mbar_wait(tfull_bar(abuf), aphase, wctx)) {
+                    !mbar_wait(tfull_bar(slot_id), aphase, wctx)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const float* slot = scale_slots + sstage * C::kScaleSlotFloats;
                 const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(abuf * C::BNQ + wg * C::kCW);
-                promote_k_block<C>(acc, taddr, slot, row, wg);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(tempty_bar(abuf));
-                    mbar_arrive(sempty_bar(sstage));
+                // the accumulator slice and the scale slot are only read, and each arrival
+                // follows the completion of those reads: no release fence is needed (one
+                // would also wait for this warp's outstanding output stores).  The slice is
+                // released as soon as its last chunk is in registers; the scale slot after
+                // the FMAs, which read per-token scales from it in the decode configuration.
+                const uint32_t sempty = sempty_bar(sstage);
+                promote_k_block<C>(acc, taddr, slot, row, wg, [&]() {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if constexpr (C::PAIR) mbar_arrive_cluster_relaxed(mapa_shared(tempty_bar(slot_id), 0));
+                        else mbar_arrive_relaxed(tempty_bar(slot_id));
+                        // dense: the scales were read before the first TMEM load
+                        if constexpr (!C::SWAP) mbar_arrive_relaxed(sempty);
+                    }
+                });
+                if constexpr (C::SWAP) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_relaxed(sempty);
                 }
                 if (++sstage == C::kScaleStages) {
                     sstage = 0;
@@ -453,10 +564,20 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         }
     }
 
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+    if constexpr (C::PAIR) {
+        // no CTA leaves while its peer may still signal its barriers or read TMEM
+        tc_fence_before();
+        cluster_sync();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc_pair(tmem_base, C::kTmemCols);
+        }
+    } else {
+        __syncthreads();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc(tmem_base, C::kTmemCols);
+        }
     }
 }
 

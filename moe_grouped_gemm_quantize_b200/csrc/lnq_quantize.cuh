@@ -3,10 +3,8 @@
 //  * k_quantize_groups: activations, one FP32 scale per 1 x 128 group of a row
 //    (Linnet "Backend plugins", DeepGEMM plugin: "each 128 inputs of a row to
 //    FP8 with a scale of their own"), scales written MN-major over rows padded
-//    to a multiple of four.  amax, scale and E4M3 cast are fused in one pass:
-//    128-bit bf16 loads, a half-warp shuffle reduction for amax, packed
-//    e4m3x2 conversion, and the scale column staged through shared memory so
-//    it is stored as contiguous 128-byte runs.
+//    to a multiple of four.  amax, scale and E4M3 cast are fused in one pass
+//    over tiles streamed into shared memory by TMA.
 //  * k_quantize_blocks: weights, one FP32 scale per 128 x 128 block (Linnet
 //    plugin docstring; deepgemm-rust README, "Quick start", sfb shape).
 //
@@ -16,6 +14,9 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
+
+#include "lnq_ptx.cuh"
 
 namespace lnq {
 
@@ -34,25 +35,42 @@ __device__ __forceinline__ float quotient(float x, float s, bool zero_group) {
 }
 
 // True when the E4M3 rounding of t could differ from the E4M3 rounding of a
-// value at most 3 fp32 ulps away: t within 4 ulps of a rounding midpoint of the
-// normal E4M3 range (the 20 fp32 mantissa bits below the 3 E4M3 mantissa bits
-// within 4 of 0x80000), or 0 < |t| < 2^-6 (E4M3 subnormal range, where the
+// value at most 16 fp32 ulps away: t within 32 ulps of a rounding midpoint of
+// the normal E4M3 range (the 20 fp32 mantissa bits below the 3 E4M3 mantissa
+// bits within 32 of 0x80000), or |t| < 2^-6 (E4M3 subnormal range, where the
 // midpoints sit elsewhere).  Binade edges hold no midpoint, so one test covers
 // every exponent.
 __device__ __forceinline__ bool near_e4m3_midpoint(float t) {
     const uint32_t b = __float_as_uint(t);
-    const bool near_mid = ((b & 0xFFFFFu) - 0x7FFFCu) < 9u;
-    const bool small = ((b & 0x7FFFFFFFu) - 1u) < 0x3C7FFFFFu;
-    return near_mid || small;
+    return ((b & 0xFFFFFu) - 0x7FFE0u) < 65u || fabsf(t) < 0x1p-6f;
+}
+
+// The correctly rounded amax / 448 from one multiplication and two FMAs: q0 =
+// RN(amax * c) with c = RN(1/448), then one correction step with the exact
+// remainder amax - 448 q0 (Markstein's division correction for a divisor known
+// in advance).  Checked exhaustively against the IEEE quotient over every
+// non-negative finite bf16 amax.
+__device__ __forceinline__ float scale_of_amax(float amax) {
+    constexpr float c = 1.0f / 448.0f;
+    const float q0 = __fmul_rn(amax, c);
+    const float rem = __fmaf_rn(-q0, 448.0f, amax);
+    return __fmaf_rn(rem, c, q0);
+}
+
+// Approximate reciprocal (hardware rcp.approx, within a few ulps).
+__device__ __forceinline__ float rcp_approx(float s) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    return r;
 }
 
 // Eight quotients x/s whose E4M3 codes equal those of the correctly rounded
-// quotients.  The fast path multiplies by r = RN(1/s): |x*r - x/s| is at most
-// 2^-23 |x/s| + 2^-48 |x/s|, so x*r and RN(x/s) are at most 3 ulps apart and
-// round to the same E4M3 code unless x*r lies within 4 ulps of an E4M3
-// midpoint (a rounding test in the manner of Ziv's correctly rounded
-// elementary functions).  Then, and for tiny scales where r is inexact or
-// infinite, the eight values take the IEEE division instead.
+// quotients.  The fast path multiplies by r ~ 1/s: with r within 2^-21 of 1/s,
+// x*r and RN(x/s) are at most 16 ulps apart and take the same E4M3 code unless
+// x*r lies within 32 ulps of an E4M3 midpoint (a rounding test in the manner of
+// Ziv's correctly rounded elementary functions).  Then, and for tiny scales
+// where r would be subnormal or infinite, the eight values take the IEEE
+// division instead.
 __device__ __forceinline__ void quotients8(const uint4& raw, float s, float r, bool zero_group,
                                            bool exact_group, float (&t)[8]) {
     t[0] = bf16_lo(raw.x);
@@ -106,55 +124,139 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
     return v;
 }
 
-constexpr int kQuantRowsPerCta = 32;   // rows of one activation tile
-constexpr int kQuantColsPerCta = 256;  // two 128-groups
-constexpr int kQuantRowsPerWarp = kQuantRowsPerCta / 8;
+constexpr int kQuantRows = 32;      // rows of one activation tile
+constexpr int kQuantCols = 256;     // columns of one tile: two 128-groups
+constexpr int kQuantStages = 4;     // tiles in flight per CTA
+constexpr int kQuantTileBytes = kQuantRows * kQuantCols * 2;
+constexpr int kQuantConsumerWarps = 8;
+constexpr int kQuantThreads = 32 * (kQuantConsumerWarps + 1);
+constexpr int kQuantSmemBytes = kQuantStages * kQuantTileBytes + 2 * kQuantStages * 8 + 16 + 128;
 
-// grid = (ceil(M4 / 32), ceil(K / 256)), block = 256 threads.
-// Warp w takes rows w, w+8, w+16, w+24 of the tile; lane l takes columns
-// 8l .. 8l+7 of the 256, so lanes 0-15 form the first group, 16-31 the second.
-__global__ void __launch_bounds__(256)
-    k_quantize_groups(const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ld_x,
-                      uint8_t* __restrict__ q, int64_t ld_q, float* __restrict__ sfa, int64_t M4) {
-    __shared__ float s_scale[2][kQuantRowsPerCta];
+struct QuantArgs {
+    uint8_t* q;
+    float* sfa;
+    unsigned int* status;
+    unsigned long long timeout_ns;
+    long long M, K, ld_q, M4;
+    int num_tiles;   // ceil(M4 / 32) * ceil(K / 256)
+    int col_tiles;   // ceil(K / 256)
+};
+
+// Persistent 1x128 activation quantize.  A producer warp streams 32 x 256 bf16
+// tiles into a 4-stage shared-memory ring with TMA (rows past M arrive as
+// zeros); eight consumer warps each own four consecutive rows of a tile: lane
+// l holds columns 8l .. 8l+7, so lanes 0-15 form the first 128-group and
+// 16-31 the second.  The amax is a half-warp shuffle reduction; lanes 0 and 16
+// store their four rows' scales as one 16-byte run (M4 is a multiple of 4).
+// Consumer warps never wait for one another.
+__global__ void __launch_bounds__(kQuantThreads)
+    k_quantize_groups(const __grid_constant__ CUtensorMap xmap, const QuantArgs args) {
+    extern __shared__ uint8_t qsmem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(qsmem_raw) + 127) & ~static_cast<uintptr_t>(127));
+    uint8_t* bar_area = smem + kQuantStages * kQuantTileBytes;
+    const uint32_t bars = smem_u32(bar_area);
+    auto full_bar = [&](int st) { return bars + 8u * st; };
+    auto empty_bar = [&](int st) { return bars + 8u * (kQuantStages + st); };
+    volatile uint32_t* abort_flag =
+        reinterpret_cast<volatile uint32_t*>(bar_area + 2 * kQuantStages * 8);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int half = lane >> 4;
-    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kQuantRowsPerCta;
-    const int64_t col0 = static_cast<int64_t>(blockIdx.y) * kQuantColsPerCta;
-    const int64_t groups = K >> 7;
-    const bool group_ok = (col0 >> 7) + half < groups;
-    const int64_t col = col0 + lane * 8;
 
-    uint4 raw[kQuantRowsPerWarp];
-#pragma unroll
-    for (int i = 0; i < kQuantRowsPerWarp; ++i) {
-        const int64_t r = row0 + warp + 8 * i;
-        raw[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (r < M && group_ok) raw[i] = ld_nc_v4(x + r * ld_x + col);
-    }
-#pragma unroll
-    for (int i = 0; i < kQuantRowsPerWarp; ++i) {
-        float amax = absmax8(raw[i]);
-#pragma unroll
-        for (int off = 8; off >= 1; off >>= 1)
-            amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-        const float s = __fdiv_rn(amax, 448.0f);
-        const int64_t r = row0 + warp + 8 * i;
-        if (r < M && group_ok) {
-            float t[8];
-            quotients8(raw[i], s, __frcp_rn(s), amax == 0.0f, !(s >= 0x1p-125f), t);
-            *reinterpret_cast<uint2*>(q + r * ld_q + col) = pack8(t);
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kQuantStages; ++st) {
+            mbar_init(full_bar(st), 1);
+            mbar_init(empty_bar(st), kQuantConsumerWarps);
         }
-        if ((lane & 15) == 0) s_scale[half][warp + 8 * i] = s;
+        *abort_flag = 0u;
+        fence_barrier_init();
     }
     __syncthreads();
-    if (threadIdx.x < 2 * kQuantRowsPerCta) {
-        const int h = threadIdx.x / kQuantRowsPerCta;
-        const int i = threadIdx.x % kQuantRowsPerCta;
-        const int64_t g = (col0 >> 7) + h;
-        const int64_t r = row0 + i;
-        if (g < groups && r < M4) sfa[g * M4 + r] = s_scale[h][i];
+    WaitCtx wctx;
+    wctx.abort = abort_flag;
+    wctx.status = args.status;
+    wctx.timeout_ns = args.timeout_ns;
+
+    if (warp == kQuantConsumerWarps) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            tma_prefetch_desc(&xmap);
+            int stage = 0;
+            uint32_t phase = 0, filled = 0, fill_parity = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
+                if (!mbar_wait(empty_bar(stage), phase ^ 1u, wctx)) {
+                    ok = false;
+                    break;
+                }
+                const int row0 = (t / args.col_tiles) * kQuantRows;
+                const int col0 = (t % args.col_tiles) * kQuantCols;
+                mbar_arrive_expect_tx(full_bar(stage), kQuantTileBytes);
+                tma_load_2d(smem_u32(smem + stage * kQuantTileBytes), &xmap, full_bar(stage), col0,
+                            row0);
+                filled |= 1u << stage;
+                fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == kQuantStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) {
+                WaitCtx drain = wctx;
+                uint32_t never = 0u;
+                drain.abort = &never;
+                for (int st = 0; st < kQuantStages; ++st)
+                    if (filled & (1u << st)) (void)mbar_wait(full_bar(st), (fill_parity >> st) & 1u, drain);
+            }
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    // warp w owns rows 4w .. 4w+3 of each tile and writes their scales itself
+    constexpr int kRowsPerWarp = kQuantRows / kQuantConsumerWarps;
+    static_assert(kRowsPerWarp == 4, "one float4 of scales per warp and group");
+    const int half = lane >> 4;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
+        const long long row0 = static_cast<long long>(t / args.col_tiles) * kQuantRows + warp * kRowsPerWarp;
+        const long long col0 = static_cast<long long>(t % args.col_tiles) * kQuantCols;
+        const long long group = (col0 >> 7) + half;
+        const bool group_ok = group < (args.K >> 7);
+        if (!mbar_wait(full_bar(stage), phase, wctx)) break;
+        const uint8_t* tile = smem + stage * kQuantTileBytes + warp * kRowsPerWarp * (kQuantCols * 2);
+        uint4 raw[kRowsPerWarp];
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i)
+            raw[i] = *reinterpret_cast<const uint4*>(tile + i * (kQuantCols * 2) + lane * 16);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(stage));
+        float sv[kRowsPerWarp];
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            float amax = absmax8(raw[i]);
+#pragma unroll
+            for (int off = 8; off >= 1; off >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+            sv[i] = scale_of_amax(amax);
+        }
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            const long long r = row0 + i;
+            if (r < args.M && group_ok) {
+                float tq[8];
+                quotients8(raw[i], sv[i], rcp_approx(sv[i]), sv[i] == 0.0f, !(sv[i] >= 0x1p-125f), tq);
+                *reinterpret_cast<uint2*>(args.q + r * args.ld_q + col0 + lane * 8) = pack8(tq);
+            }
+        }
+        if ((lane & 15) == 0 && group_ok && row0 < args.M4)
+            *reinterpret_cast<float4*>(args.sfa + group * args.M4 + row0) =
+                make_float4(sv[0], sv[1], sv[2], sv[3]);
+        if (++stage == kQuantStages) {
+            stage = 0;
+            phase ^= 1u;
+        }
     }
 }
 

@@ -45,11 +45,19 @@ def test_tiny_workload_elementwise():
     check_full(a, w, "tiny 128x256x512")
 
 
+@pytest.fixture(params=[False, True], ids=["one_cta", "cta_pairs"])
+def dense_pairs(request):
+    """Runs a test with dense GEMMs on single CTAs and again on CTA pairs."""
+    previous = lnq.lnq_set_dense_cta_pairs(request.param)
+    yield request.param
+    lnq.lnq_set_dense_cta_pairs(previous)
+
+
 @pytest.mark.parametrize("M,N,K", [
     (65, 256, 128), (100, 128, 256), (128, 16, 128), (130, 272, 384), (200, 640, 512),
-    (257, 384, 640), (384, 1024, 1024), (129, 48, 256), (300, 4096, 128),
+    (257, 384, 640), (384, 1024, 1024), (129, 48, 256), (300, 4096, 128), (640, 768, 512),
 ])
-def test_dense_shapes_elementwise(M, N, K):
+def test_dense_shapes_elementwise(M, N, K, dense_pairs):
     a = synthetic.gaussian_bf16((M, K), 1.0, seed=M + 7 * N + K)
     w = synthetic.gaussian_bf16((N, K), 0.02, seed=M + N + 3 * K)
     check_full(a, w, f"{M}x{N}x{K}")
@@ -103,7 +111,7 @@ def check_sampled(a, w, what, count=20000, seed=0):
 
 
 @pytest.mark.parametrize("idx", range(4))
-def test_prefill_workloads_sampled(idx):
+def test_prefill_workloads_sampled(idx, dense_pairs):
     cfg = synthetic.PREFILL[idx]
     a, w = synthetic.make_linear_inputs(cfg)
     check_sampled(a, w, cfg.name)
@@ -118,7 +126,7 @@ def test_decode_workloads():
             check_sampled(a, w, cfg.name)
 
 
-def test_square_outlier_workload_sampled():
+def test_square_outlier_workload_sampled(dense_pairs):
     cfg = synthetic.SQUARE
     a, w = synthetic.make_linear_inputs(cfg)
     check_sampled(a, w, cfg.name, count=30000)

@@ -153,11 +153,12 @@ def test_moe_weights_full_size():
     assert_same_w(w)
 
 
-def near_midpoint_rows(max_rows=4096):
+def near_midpoint_rows(max_rows=8192):
     """Rows whose quotients x/s land near E4M3 rounding midpoints under scales that are
-    not powers of two: found by brute force over bf16 amax in [1, 2) x every bf16 x up
-    to amax.  Kept: x where RN(x * RN(1/s)) and RN(x / s) take different E4M3 codes, and
-    x where RN(x / s) is within 8 ulps of a midpoint."""
+    not powers of two: found by brute force over every bf16 amax in [1, 2) (every
+    possible scale mantissa) x every bf16 x up to amax.  Kept: x where RN(x * RN(1/s))
+    and RN(x / s) take different E4M3 codes, and x where RN(x / s) is within 256 ulps
+    of a midpoint."""
     amax_bits = np.arange(0x3F80, 0x4000, dtype=np.uint16)           # bf16 values in [1, 2)
     x_bits = np.arange(0, 0x4000, dtype=np.uint16)                   # bf16 values in [0, 2)
     xs = (x_bits.astype(np.uint32) << 16).view(np.float32)
@@ -172,7 +173,7 @@ def near_midpoint_rows(max_rows=4096):
         ct = torch.from_numpy(t).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
         cf = torch.from_numpy(f).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
         low = t.view(np.uint32) & 0xFFFFF
-        near = np.abs(low.astype(np.int64) - 0x80000) <= 8
+        near = np.abs(low.astype(np.int64) - 0x80000) <= 256
         pick = x[(ct != cf) | near]
         for i in range(0, pick.size, 127):
             chosen.append((amax, pick[i:i + 127]))
@@ -190,3 +191,18 @@ def test_quotients_near_e4m3_midpoints():
     assert x.shape[0] > 100
     for scale in (1.0, -3.0, 2.0 ** 40, 2.0 ** -60):
         assert_same_a(torch.tensor(x * scale).to(torch.bfloat16))
+
+
+def test_zero_rows_write_zero_pad_scales():
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device=DEV)
+    q = torch.empty((0, 256), dtype=torch.uint8, device=DEV)
+    sfa = torch.full((2, 8), float("nan"), dtype=torch.float32, device=DEV)
+    lnq.lnq_quantize_fp8_groups(x, q, sfa)
+    torch.cuda.synchronize()
+    assert torch.all(sfa == 0)
+
+
+@pytest.mark.parametrize("M,K", [(1, 4096), (33, 384), (100, 640), (4097, 256)])
+def test_activation_more_ragged_shapes(M, K):
+    # K not a multiple of 256 (a half-empty column tile) and row counts off the 32-row tile
+    assert_same_a(synthetic.gaussian_bf16((M, K), 1.0, seed=M + K))
