@@ -299,7 +299,10 @@ def run_ours(args, world, rank, local):
         lnq_build.build()
     barrier(dist)
     lnq.lib()
-    lnq.lnq_set_dense_cta_pairs(args.cta_pairs)
+    lnq.lib().lnq_set_dense_cta_pairs(args.cta_pairs)
+    # the weights are model parameters quantized before timing: nothing in the step
+    # writes them, so the GEMMs may stream them before the previous kernel completes
+    lnq.lnq_set_weight_prefetch(not args.no_weight_prefetch)
 
     cfgs, kind = workload_units(args.workload)
     units = [Grouped(c, dev) if kind == "grouped" else Linear(c, dev) for c in cfgs]
@@ -331,9 +334,11 @@ def run_ours(args, world, rank, local):
     if lnq.lnq_get_last_device_error() != 0:
         raise RuntimeError("device reported an error during warm-up")
 
-    # ---- timed region (device time, CUDA events on the launching stream)
+    # ---- timed region (device time, CUDA events on the launching stream).  Events only
+    # bracket the K steps: an event between two kernels would stop the next one from
+    # starting early (programmatic dependent launch), so the per-kernel times come from
+    # a second timed loop below.
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_units + 1)] for _ in range(K)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     barrier(dist)
@@ -341,7 +346,7 @@ def run_ours(args, world, rank, local):
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
         t0.record(stream)
         for k in range(K):
-            launch_step(evs[k])
+            launch_step()
         t1.record(stream)
         torch.cuda.synchronize()
     barrier(dist)
@@ -349,6 +354,13 @@ def run_ours(args, world, rank, local):
     if lnq.lnq_get_last_device_error() != 0:
         raise RuntimeError("device reported an error in the timed region")
     ms = max_over_ranks(ms_local, dist, dev)
+
+    # ---- per-kernel times: K more steps with an event around every kernel
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_units + 1)] for _ in range(K)]
+    torch.cuda.synchronize()
+    for k in range(K):
+        launch_step(evs[k])
+    torch.cuda.synchronize()
     q_ms = sum(evs[k][2 * i].elapsed_time(evs[k][2 * i + 1]) for k in range(K) for i in range(n_units))
     g_ms = sum(evs[k][2 * i + 1].elapsed_time(evs[k][2 * i + 2]) for k in range(K)
                for i in range(n_units))
@@ -434,7 +446,8 @@ def run_ours(args, world, rank, local):
         "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out",
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, bf16)",
         "config": {"workload": args.workload, "desc": WORKLOAD_DESC[args.workload],
-                   "dense_cta_pairs": bool(args.cta_pairs),
+                   "dense_cta_pairs": args.cta_pairs,
+                   "weight_prefetch": not args.no_weight_prefetch,
                    "parallelism": f"replicas x{world} (independent tokens per rank)",
                    "l2": "working set per step > 126 MB L2; no extra flush"},
         "roofline": roof,
@@ -446,6 +459,8 @@ def run_ours(args, world, rank, local):
             "gemm_share_of_step": round(g_ms / (g_ms + q_ms), 4),
         },
         "gpu_launches": K * 2 * n_units,
+        "timing": "value: K steps between two events (kernels chained by programmatic dependent "
+                  "launch); roofline and kernels: K further steps with an event around each kernel",
         "clocks": clocks.summary(),
         "e2e": e2e,
     }
@@ -568,8 +583,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--cta-pairs", action="store_true",
-                    help="run dense GEMMs (M > 128, N >= 256) on CTA pairs")
+    ap.add_argument("--no-weight-prefetch", action="store_true",
+                    help="GEMMs wait for the previous kernel before streaming weights")
+    ap.add_argument("--cta-pairs", type=int, default=0, choices=[0, 1, 2],
+                    help="dense GEMMs with M > 128: 0 one CTA per 128x256 tile, 1 CTA pairs on "
+                         "256x256 tiles, 2 CTA pairs on 256x128 tiles")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

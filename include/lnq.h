@@ -172,13 +172,29 @@ lnq_status lnq_get_last_device_error(void* stream);
 lnq_status lnq_selftest_wait_timeout(int64_t timeout_ns, void* stream);
 
 /*
- * Tuning knob (process-wide, default 0): when non-zero, dense GEMMs with
- * M > 128 and N >= 256 run on pairs of CTAs (a cluster of two sharing one
- * tcgen05 MMA of 256 x 256, each CTA loading half of the weight tile) instead
- * of one CTA per 128 x 256 tile.  Results are the same up to FP32 summation
- * order.  Returns the previous setting.
+ * Tuning knob (process-wide, default 0) for dense GEMMs with M > 128:
+ *   0  one CTA per 128 x 256 tile (N >= 256);
+ *   1  pairs of CTAs (a cluster of two sharing one tcgen05 MMA) on 256 x 256
+ *      tiles, each CTA loading half of the weight tile (N >= 256);
+ *   2  pairs of CTAs on 256 x 128 tiles with four accumulators per CTA
+ *      (N >= 128).
+ * Other values select 0.  Results are the same up to FP32 summation order.
+ * Returns the previous setting.
  */
 int32_t lnq_set_dense_cta_pairs(int32_t enable);
+
+/*
+ * Weight prefetch (process-wide, default 0).  Every kernel of this library is
+ * launched with programmatic stream serialization: it may start while the
+ * previous kernel of the stream is still running, and waits for that kernel
+ * to complete before it reads any input.  When this knob is non-zero, the
+ * single-CTA dense and decode GEMMs issue the weight halves of their first
+ * pipeline stages before that wait.  Enable it only when the weights and the
+ * weight scales passed to the GEMM are not written by kernels that may still
+ * be running when the GEMM starts (e.g. they are model parameters prepared
+ * before the forward pass).  Returns the previous setting.
+ */
+int32_t lnq_set_weight_prefetch(int32_t enable);
 
 /* Version of this ABI (major*10000 + minor*100 + patch). */
 int32_t lnq_abi_version(void);

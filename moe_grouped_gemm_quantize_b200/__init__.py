@@ -28,7 +28,8 @@ __all__ = [
     "LnqError", "library_path", "lib",
     "lnq_quantize_fp8_groups", "lnq_quantize_fp8_blocks", "lnq_fp8_block_gemm_nt",
     "lnq_m_grouped_fp8_gemm_contiguous", "lnq_get_last_device_error", "lnq_status_string",
-    "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "quantize_activations", "quantize_weights",
+    "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "lnq_set_weight_prefetch",
+    "quantize_activations", "quantize_weights",
     "quantize_weights_grouped", "linear",
     "m_grouped_linear", "ceil4",
 ]
@@ -82,8 +83,9 @@ def lib() -> ctypes.CDLL:
         L.lnq_status_string.argtypes = [ctypes.c_int]
         L.lnq_status_string.restype = ctypes.c_char_p
         L.lnq_abi_version.restype = ctypes.c_int32
-        L.lnq_set_dense_cta_pairs.argtypes = [ctypes.c_int32]
-        L.lnq_set_dense_cta_pairs.restype = ctypes.c_int32
+        for knob in ("lnq_set_dense_cta_pairs", "lnq_set_weight_prefetch"):
+            getattr(L, knob).argtypes = [ctypes.c_int32]
+            getattr(L, knob).restype = ctypes.c_int32
         _lib = L
         return L
 
@@ -193,9 +195,16 @@ def lnq_get_last_device_error(stream=None) -> int:
     return int(lib().lnq_get_last_device_error(_stream(stream)))
 
 
-def lnq_set_dense_cta_pairs(enable: bool) -> bool:
-    """Route dense GEMMs (M > 128, N >= 256) to CTA pairs; returns the previous setting."""
-    return bool(lib().lnq_set_dense_cta_pairs(1 if enable else 0))
+def lnq_set_dense_cta_pairs(mode: int) -> int:
+    """Dense GEMM configuration for M > 128: 0 one CTA per 128x256 tile, 1 CTA pairs on
+    256x256 tiles, 2 CTA pairs on 256x128 tiles.  Returns the previous setting."""
+    return int(lib().lnq_set_dense_cta_pairs(int(mode)))
+
+
+def lnq_set_weight_prefetch(enable: bool) -> bool:
+    """Let GEMMs stream their first weight stages before the previous kernel of the
+    stream completes (weights must not be written by still-running kernels)."""
+    return bool(lib().lnq_set_weight_prefetch(1 if enable else 0))
 
 
 def lnq_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:

@@ -40,6 +40,10 @@ struct DeviceInfo {
 };
 
 std::mutex g_mutex;
+// Dense GEMMs with M > 128 run on CTA pairs when set (1: 256x256, 2: 256x128 tiles).
+std::atomic<int> g_dense_pairs{0};
+// GEMMs may start streaming weights before the prior kernel completes.
+std::atomic<int> g_weight_prefetch{0};
 DeviceInfo g_devices[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 
@@ -123,20 +127,24 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
     }
     args.status = dev.status;
     args.timeout_ns = kDefaultTimeoutNs;
+    args.prefetch_weights = g_weight_prefetch.load(std::memory_order_relaxed);
     if constexpr (C::PAIR) {
-        // clusters of two CTAs; as many pairs as can be resident at once
+        // clusters of two CTAs sharing one MMA; as many pairs as can be resident
+        constexpr int kCluster = 2;
         static int max_clusters[kMaxDevices] = {};
         cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.x = kCluster;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.blockDim = dim3(C::kThreads, 1, 1);
         cfg.dynamicSmemBytes = C::kSmemBytes;
         cfg.stream = stream;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         if (max_clusters[devno] == 0) {
             int n = 0;
             cfg.gridDim = dim3(2 * (dev.sm_count / 2), 1, 1);
@@ -144,29 +152,39 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
                 return LNQ_ERR_CUDA;
             max_clusters[devno] = n;
         }
-        const int pairs = args.num_tiles < max_clusters[devno] ? args.num_tiles : max_clusters[devno];
-        if (pairs <= 0) return LNQ_OK;
-        cfg.gridDim = dim3(2 * pairs, 1, 1);
+        const int clusters = args.num_tiles < max_clusters[devno] ? args.num_tiles : max_clusters[devno];
+        if (clusters <= 0) return LNQ_OK;
+        cfg.gridDim = dim3(kCluster * clusters, 1, 1);
         if (cudaLaunchKernelEx(&cfg, k_fp8_block_gemm<C>, map_p, map_q, args) != cudaSuccess)
             return LNQ_ERR_CUDA;
         return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
     }
     const int grid = args.num_tiles < dev.sm_count ? args.num_tiles : dev.sm_count;
     if (grid <= 0) return LNQ_OK;
-    k_fp8_block_gemm<C><<<grid, C::kThreads, C::kSmemBytes, stream>>>(map_p, map_q, args);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_fp8_block_gemm<C>, map_p, map_q, args) != cudaSuccess)
+        return LNQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
 }
 
 // Tile configurations (P = MMA M slot, Q = MMA N slot).
 using CfgDense256 = GemmCfg<256, 4, 2, false, false>;
 using CfgPair256 = GemmCfg<256, 6, 2, false, false, true>;
+using CfgPair128 = GemmCfg<128, 8, 2, false, false, true>;
 
-// Dense GEMMs with M > 128 and N >= 256 run on CTA pairs only when enabled.
-std::atomic<int> g_dense_pairs{0};
 using CfgDense128 = GemmCfg<128, 6, 2, false, false>;
 using CfgGrouped256 = GemmCfg<256, 4, 2, false, true>;
 using CfgGrouped128 = GemmCfg<128, 6, 2, false, true>;
-using CfgSwap32 = GemmCfg<32, 8, 1, true, false>;
+using CfgSwap32 = GemmCfg<32, 10, 1, true, false>;
 using CfgSwap64 = GemmCfg<64, 8, 1, true, false>;
 
 constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
@@ -180,8 +198,10 @@ extern "C" {
 
 int32_t lnq_abi_version(void) { return 10000; }
 
+int32_t lnq_set_weight_prefetch(int32_t enable) { return g_weight_prefetch.exchange(enable ? 1 : 0); }
+
 int32_t lnq_set_dense_cta_pairs(int32_t enable) {
-    const int previous = g_dense_pairs.exchange(enable ? 1 : 0);
+    const int previous = g_dense_pairs.exchange(enable >= 0 && enable <= 2 ? enable : 0);
     return previous;
 }
 
@@ -257,8 +277,17 @@ lnq_status lnq_quantize_fp8_groups(const void* x_bf16, int64_t M, int64_t K, int
     }
     const long long max_ctas = 3LL * dev->sm_count;
     const int grid = static_cast<int>(tiles < max_ctas ? tiles : max_ctas);
-    k_quantize_groups<<<grid, kQuantThreads, kQuantSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-        xmap, qa);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kQuantThreads, 1, 1);
+    cfg.dynamicSmemBytes = kQuantSmemBytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_quantize_groups, xmap, qa) != cudaSuccess) return LNQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
 }
 
@@ -316,12 +345,20 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
         args.num_tiles = args.tiles_p * args.tiles_q;
         return launch_gemm<CfgSwap64>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
     }
-    if (N >= 256 && M > 128 && g_dense_pairs.load(std::memory_order_relaxed)) {
+    const int pairs = g_dense_pairs.load(std::memory_order_relaxed);
+    if (N >= 256 && M > 128 && pairs == 1) {
         // pairs of CTAs on 256 x 256 tiles
         args.tiles_p = static_cast<int>((M + 255) / 256);
         args.tiles_q = static_cast<int>((N + 255) / 256);
         args.num_tiles = args.tiles_p * args.tiles_q;
         return launch_gemm<CfgPair256>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
+    }
+    if (N >= 128 && M > 128 && pairs == 2) {
+        // pairs of CTAs on 256 x 128 tiles, four accumulators per CTA
+        args.tiles_p = static_cast<int>((M + 255) / 256);
+        args.tiles_q = static_cast<int>((N + 127) / 128);
+        args.num_tiles = args.tiles_p * args.tiles_q;
+        return launch_gemm<CfgPair128>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
     }
     args.tiles_p = static_cast<int>((M + 127) / 128);
     if (N >= 256) {

@@ -30,8 +30,10 @@
 //               (tcgen05.ld), multiplies it by sa*sb and adds it into FP32
 //               registers (the per-K-block promotion); after the last K block
 //               converts to bf16 (round to nearest even) and stores the tile.
-// The two TMEM accumulators let the tensor core run the next K block while
-// the epilogue promotes the previous one.  All waits are bounded (mbar_wait).
+// The TMEM accumulators (as many as fit: 2 of 256 columns, 4 of 128, up to 16 of
+// 32) let the tensor core run ahead of the epilogue's promotion; the depth
+// hides the MMA -> epilogue -> MMA handshake latency.  All waits are bounded
+// (mbar_wait).
 #pragma once
 
 #include <cstdint>
@@ -57,6 +59,7 @@ struct GemmArgs {
     int tiles_p;      // tiles along the MMA M slot (of 256 rows for PAIR)
     int tiles_q;      // tiles along the MMA N slot
     int num_tiles;
+    int prefetch_weights;  // issue the first weight stages before waiting on the prior kernel
 };
 
 constexpr unsigned int kStatusBadGroup = 2u;
@@ -83,11 +86,17 @@ struct GemmCfg {
     static constexpr int kPBytes = kP * kBK;
     static constexpr int kQRowsPerCta = PAIR ? BNQ / 2 : BNQ;
     static constexpr int kQBytes = kQRowsPerCta * kBK;
-    static constexpr int kScaleStages = 8;
+    static constexpr int kScaleStages = SWAP ? 16 : 8;  // scale ring depth (K blocks)
+    // scale slot: activation scales (128 rows, or BNQ tokens), then the weight scales
+    static constexpr int kSbOffset = SWAP ? BNQ : 256;
+    static constexpr int kScaleSlotFloats = kSbOffset + 4;
     static constexpr int kCW = BNQ / EPI_WG;      // accumulator columns per epilogue thread
     static constexpr int kEpiThreads = 128 * EPI_WG;
     static constexpr int kThreads = 128 + kEpiThreads;
-    static constexpr int kTmemCols = (2 * BNQ < 32) ? 32 : 2 * BNQ;
+    // TMEM accumulators of BNQ columns each, as many as the 512 columns hold (at
+    // most 16): the tensor core may run kAccBufs-1 K blocks ahead of the promotion.
+    static constexpr int kAccBufs = (512 / BNQ) > 16 ? 16 : (512 / BNQ);
+    static constexpr int kTmemCols = kAccBufs * BNQ;
     static constexpr int kSbPerTile = SWAP ? 1 : BNQ / 128;
     static constexpr int kSaPerTile = SWAP ? BNQ : kP;
     static constexpr bool kRegSplit = (!SWAP && kCW == 128);
@@ -108,12 +117,13 @@ struct GemmCfg {
     static constexpr int kOffP = 0;
     static constexpr int kOffQ = kOffP + STAGES * kPBytes;
     static constexpr int kOffScale = kOffQ + STAGES * kQBytes;
-    static constexpr int kScaleSlotFloats = 256 + 4;
     static constexpr int kOffBar = kOffScale + kScaleStages * kScaleSlotFloats * 4;
-    static constexpr int kNumBars = 2 * STAGES + 4 * kSlices + 2 * kScaleStages + 1;
+    static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs * kSlices + 2 * kScaleStages + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+    static_assert(kTmemCols >= 32 && (kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512,
+                  "TMEM allocation is a power of two between 32 and 512 columns");
     static_assert(kQBytes % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
 };
 
@@ -185,10 +195,10 @@ __device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint3
                                                 Release&& release) {
     float2 s2;
     if constexpr (!C::SWAP) {
-        const float s = slot[row] * slot[256 + (wg * C::kCW) / 128];
+        const float s = slot[row] * slot[C::kSbOffset + (wg * C::kCW) / 128];
         s2 = make_float2(s, s);
     } else {
-        const float sb = slot[256];
+        const float sb = slot[C::kSbOffset];
         s2 = make_float2(sb, sb);
     }
     // 32-column chunks, each load issued one chunk ahead of the FMAs
@@ -210,6 +220,23 @@ __device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint3
             else tmem_wait_ld(rb);
             if (c + 2 == NC) release();
         }
+    }
+}
+
+// Decode tile store: this thread holds weight row n = p0 + row for the tile's
+// tokens q0 .. q0 + kCW - 1; D is [M][N], so each token's row gets one bf16.
+template <class C>
+__device__ __forceinline__ void store_decode_tile(const GemmArgs& args, const TileCoord& tc, int row,
+                                                  const float2 (&acc)[C::kCW / 2]) {
+    const int n = tc.p0 + row;
+    if (n >= args.N) return;
+#pragma unroll
+    for (int j = 0; j < C::kCW; ++j) {
+        const int m = tc.q0 + j;
+        const float v = (j & 1) ? acc[j >> 1].y : acc[j >> 1].x;
+        if (m < args.M)
+            args.d[static_cast<long long>(m) * args.N + n] =
+                static_cast<uint16_t>(pack_bf16x2(v, 0.f) & 0xFFFFu);
     }
 }
 
@@ -236,13 +263,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     auto full_bar = [&](int s) { return bars + 8u * s; };
     auto empty_bar = [&](int s) { return bars + 8u * (C::STAGES + s); };
     // accumulator slot = buffer * kSlices + slice
+    constexpr int kSlots = C::kAccBufs * C::kSlices;
     auto tfull_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + b); };
-    auto tempty_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + 2 * C::kSlices + b); };
-    auto sfull_bar = [&](int s) { return bars + 8u * (2 * C::STAGES + 4 * C::kSlices + s); };
+    auto tempty_bar = [&](int b) { return bars + 8u * (2 * C::STAGES + kSlots + b); };
+    auto sfull_bar = [&](int s) { return bars + 8u * (2 * C::STAGES + 2 * kSlots + s); };
     auto sempty_bar = [&](int s) {
-        return bars + 8u * (2 * C::STAGES + 4 * C::kSlices + C::kScaleStages + s);
+        return bars + 8u * (2 * C::STAGES + 2 * kSlots + C::kScaleStages + s);
     };
-    const uint32_t drain_bar = bars + 8u * (2 * C::STAGES + 4 * C::kSlices + 2 * C::kScaleStages);
+    const uint32_t drain_bar = bars + 8u * (2 * C::STAGES + 2 * kSlots + 2 * C::kScaleStages);
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile uint32_t* abort_flag = misc + 1;
 
@@ -252,13 +280,15 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
     const int unit = C::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int units = C::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    const int kb_begin = 0;
+    const int kb_end = args.num_kb;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        for (int b = 0; b < 2 * C::kSlices; ++b) {
+        for (int b = 0; b < kSlots; ++b) {
             mbar_init(tfull_bar(b), 1);
             mbar_init(tempty_bar(b), C::kEpiWarpsPerSlice);
         }
@@ -284,6 +314,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
+    // the prologue above touches no global memory: the next kernel may start its
+    // own, and this one waits for the previous kernel before reading any input
+    // (the producer may first prefetch weights, see below)
+    launch_dependents();
+    if (!(args.prefetch_weights && warp == 0)) wait_prior_grids();
 
     WaitCtx wctx;
     wctx.abort = abort_flag;
@@ -302,6 +337,31 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             uint32_t phase = 0;
             uint32_t filled = 0, fill_parity = 0;
             bool ok = true;
+            // Weight prefetch (caller asserts that the weights and their scales are not
+            // written by the kernels still running before this one): the weight halves of
+            // the first ring stages of the first tile are issued before the wait on the
+            // prior kernel, the activation halves after it.
+            int prefetched = 0;
+            if (args.prefetch_weights) {
+                if constexpr (!C::PAIR) {
+                    if (unit < args.num_tiles) {
+                        const TileCoord tc = tile_coord<C>(args, unit, rank);
+                        if (tc.group >= 0 && !C::GROUPED) {
+                            prefetched = min(C::STAGES, kb_end - kb_begin);
+                            for (int s = 0; s < prefetched; ++s) {
+                                mbar_arrive_expect_tx(full_bar(s), C::kPBytes + C::kQBytes);
+                                if constexpr (C::SWAP)
+                                    tma_load_2d(sP + s * C::kPBytes, &map_p, full_bar(s), (kb_begin + s) * C::kBK,
+                                                tc.p0);
+                                else
+                                    tma_load_2d(sQ + s * C::kQBytes, &map_q, full_bar(s), (kb_begin + s) * C::kBK,
+                                                tc.q0);
+                            }
+                        }
+                    }
+                }
+                wait_prior_grids();
+            }
             for (int t = unit; t < args.num_tiles && ok; t += units) {
                 const TileCoord tc = tile_coord<C>(args, t, rank);
                 if (tc.group < 0) continue;
@@ -313,7 +373,17 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     p_row = tc.p0;
                     q_row = tc.group * args.N + tc.q0 + static_cast<int>(rank) * C::kSliceQRows;
                 }
-                for (int kb = 0; kb < args.num_kb; ++kb) {
+                for (int kb = kb_begin; kb < kb_end; ++kb) {
+                    if (prefetched > 0) {
+                        // stage already armed and its weight half in flight: load the activations
+                        if constexpr (!C::PAIR) {
+                            if constexpr (C::SWAP)
+                                tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK, q_row);
+                            else
+                                tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK, p_row);
+                        }
+                        --prefetched;
+                    } else {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, wctx)) {
                         ok = false;
                         break;
@@ -333,6 +403,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         mbar_arrive_expect_tx(full_bar(stage), C::kPBytes + C::kQBytes);
                         tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK, p_row);
                         tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK, q_row);
+                    }
                     }
                     filled |= 1u << stage;
                     fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
@@ -366,7 +437,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             for (int t = unit; t < args.num_tiles && ok; t += units) {
                 const TileCoord tc = tile_coord<C>(args, t, 0);
                 if (tc.group < 0) continue;
-                for (int kb = 0; kb < args.num_kb && ok; ++kb) {
+                for (int kb = kb_begin; kb < kb_end && ok; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, wctx)) {
                         ok = false;
                         break;
@@ -411,8 +482,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         stage = 0;
                         phase ^= 1u;
                     }
-                    abuf ^= 1;
-                    if (abuf == 0) aphase ^= 1u;
+                    if (++abuf == C::kAccBufs) {
+                        abuf = 0;
+                        aphase ^= 1u;
+                    }
                 }
             }
             if (issued) {
@@ -427,53 +500,44 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         }
     } else if (warp == 2) {
         // ------------------------------------------------------------ scale producer
+        // Copies each K block's activation scales (one 16-byte run per lane) and the
+        // tile's weight scales straight into the scale ring with cp.async; each lane's
+        // arrival on the slot's barrier fires when its copies have landed, so the warp
+        // runs up to the ring's depth ahead without holding anything in registers.
+        // Rows past M4 and weight blocks past N read clamped addresses: they only feed
+        // accumulator rows or columns that are never stored.
         int sstage = 0;
         uint32_t sphase = 0;
         bool ok = true;
-        constexpr int kBatch = 4;
-        constexpr int kSaLanes = C::kSaPerTile / 4;  // lanes that load a float4 of sa
+        constexpr int kSaLanes = C::kSaPerTile / 4;  // lanes that copy 16 bytes of sa
         for (int t = unit; t < args.num_tiles && ok; t += units) {
             const TileCoord tc = tile_coord<C>(args, t, rank);
             if (tc.group < 0) continue;
             // activation rows of the tile (tokens for SWAP) and weight scale rows
-            const long long a_row0 = C::SWAP ? tc.q0 : tc.p0;
-            const int sb_row0 = C::SWAP ? tc.p0 / 128 : tc.group * args.nb + tc.q0 / 128;
-            const int sb_valid = C::SWAP ? 1 : min(C::kSbPerTile, args.nb - tc.q0 / 128);
-            const bool sa_ok = lane < kSaLanes && a_row0 + lane * 4 < args.M4;
-            for (int kb0 = 0; kb0 < args.num_kb && ok; kb0 += kBatch) {
-                float4 va[kBatch];
-                float vb[kBatch];
-#pragma unroll
-                for (int u = 0; u < kBatch; ++u) {
-                    const int kb = kb0 + u;
-                    va[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    vb[u] = 0.f;
-                    if (kb < args.num_kb) {
-                        if (sa_ok)
-                            va[u] = __ldg(reinterpret_cast<const float4*>(
-                                args.sfa + static_cast<long long>(kb) * args.M4 + a_row0 + lane * 4));
-                        if (lane < sb_valid)
-                            vb[u] = __ldg(args.sfb + static_cast<long long>(sb_row0 + lane) * args.num_kb + kb);
-                    }
+            long long a_row = (C::SWAP ? tc.q0 : tc.p0) + lane * 4;
+            if (a_row > args.M4 - 4) a_row = args.M4 - 4;
+            const int nb_first = C::SWAP ? tc.p0 / 128 : tc.q0 / 128;
+            const int nb_lane = min(nb_first + lane, args.nb - 1);
+            const long long sb_row = static_cast<long long>(C::SWAP ? 0 : tc.group) * args.nb + nb_lane;
+            const float* sa_src = args.sfa + a_row;
+            const float* sb_src = args.sfb + sb_row * args.num_kb;
+            for (int kb = kb_begin; kb < kb_end; ++kb) {
+                if (!mbar_wait(sempty_bar(sstage), sphase ^ 1u, wctx)) {
+                    ok = false;
+                    break;
                 }
-#pragma unroll
-                for (int u = 0; u < kBatch; ++u) {
-                    if (kb0 + u >= args.num_kb) break;
-                    if (!mbar_wait(sempty_bar(sstage), sphase ^ 1u, wctx)) {
-                        ok = false;
-                        break;
-                    }
-                    float* slot = scale_slots + sstage * C::kScaleSlotFloats;
-                    if (lane < kSaLanes) reinterpret_cast<float4*>(slot)[lane] = va[u];
-                    if (lane < C::kSbPerTile) slot[256 + lane] = vb[u];
-                    mbar_arrive(sfull_bar(sstage));
-                    if (++sstage == C::kScaleStages) {
-                        sstage = 0;
-                        sphase ^= 1u;
-                    }
+                const uint32_t slot = smem_u32(scale_slots + sstage * C::kScaleSlotFloats);
+                if (lane < kSaLanes) cp_async_16(slot + lane * 16, sa_src + static_cast<long long>(kb) * args.M4);
+                if (lane < C::kSbPerTile) cp_async_4(slot + (C::kSbOffset + lane) * 4, sb_src + kb);
+                cp_async_arrive(sfull_bar(sstage));
+                if (++sstage == C::kScaleStages) {
+                    sstage = 0;
+                    sphase ^= 1u;
                 }
             }
         }
+        // no copy may still be landing when the CTA leaves
+        asm volatile("cp.async.wait_all;" ::: "memory");
     }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -492,7 +556,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             float2 acc[C::kCW / 2];
 #pragma unroll
             for (int i = 0; i < C::kCW / 2; ++i) acc[i] = make_float2(0.f, 0.f);
-            for (int kb = 0; kb < args.num_kb; ++kb) {
+            for (int kb = kb_begin; kb < kb_end; ++kb) {
                 const int slot_id = abuf * C::kSlices + (C::kSlices == 1 ? 0 : wg);
                 if (!mbar_wait(sfull_bar(sstage), sphase, wctx) ||
                     !mbar_wait(tfull_bar(slot_id), aphase, wctx)) {
@@ -526,8 +590,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     sstage = 0;
                     sphase ^= 1u;
                 }
-                abuf ^= 1;
-                if (abuf == 0) aphase ^= 1u;
+                if (++abuf == C::kAccBufs) {
+                    abuf = 0;
+                    aphase ^= 1u;
+                }
             }
             if (!ok) break;
             // ---- store the tile
@@ -549,17 +615,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     }
                 }
             } else {
-                const int n = tc.p0 + row;
-                if (n < args.N) {
-#pragma unroll
-                    for (int j = 0; j < C::kCW; ++j) {
-                        const int m = tc.q0 + j;
-                        const float v = (j & 1) ? acc[j >> 1].y : acc[j >> 1].x;
-                        if (m < args.M)
-                            args.d[static_cast<long long>(m) * args.N + n] =
-                                static_cast<uint16_t>(pack_bf16x2(v, 0.f) & 0xFFFFu);
-                    }
-                }
+                store_decode_tile<C>(args, tc, row, acc);
             }
         }
     }

@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(kQuantThreads)
         fence_barrier_init();
     }
     __syncthreads();
+    launch_dependents();
+    wait_prior_grids();
     WaitCtx wctx;
     wctx.abort = abort_flag;
     wctx.status = args.status;

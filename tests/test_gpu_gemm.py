@@ -45,19 +45,30 @@ def test_tiny_workload_elementwise():
     check_full(a, w, "tiny 128x256x512")
 
 
-@pytest.fixture(params=[False, True], ids=["one_cta", "cta_pairs"])
+@pytest.fixture(params=[0, 1, 2], ids=["one_cta", "cta_pairs_256", "cta_pairs_128"])
 def dense_pairs(request):
-    """Runs a test with dense GEMMs on single CTAs and again on CTA pairs."""
-    previous = lnq.lnq_set_dense_cta_pairs(request.param)
+    """Runs a test with each dense configuration: single CTAs, CTA pairs on 256x256
+    tiles, CTA pairs on 256x128 tiles."""
+    previous = lnq.lib().lnq_set_dense_cta_pairs(request.param)
     yield request.param
-    lnq.lnq_set_dense_cta_pairs(previous)
+    lnq.lib().lnq_set_dense_cta_pairs(previous)
+
+
+@pytest.fixture(params=[False, True], ids=["no_prefetch", "weight_prefetch"])
+def weight_prefetch(request):
+    """Runs a test with and without the weights' first stages streamed before the
+    wait on the previous kernel (the weights here are written two kernels earlier,
+    by a kernel that does not release its dependents early)."""
+    previous = lnq.lnq_set_weight_prefetch(request.param)
+    yield request.param
+    lnq.lnq_set_weight_prefetch(previous)
 
 
 @pytest.mark.parametrize("M,N,K", [
     (65, 256, 128), (100, 128, 256), (128, 16, 128), (130, 272, 384), (200, 640, 512),
     (257, 384, 640), (384, 1024, 1024), (129, 48, 256), (300, 4096, 128), (640, 768, 512),
 ])
-def test_dense_shapes_elementwise(M, N, K, dense_pairs):
+def test_dense_shapes_elementwise(M, N, K, dense_pairs, weight_prefetch):
     a = synthetic.gaussian_bf16((M, K), 1.0, seed=M + 7 * N + K)
     w = synthetic.gaussian_bf16((N, K), 0.02, seed=M + N + 3 * K)
     check_full(a, w, f"{M}x{N}x{K}")
@@ -65,7 +76,7 @@ def test_dense_shapes_elementwise(M, N, K, dense_pairs):
 
 @pytest.mark.parametrize("M", [1, 2, 5, 8, 17, 31, 32, 33, 48, 63, 64])
 @pytest.mark.parametrize("N,K", [(256, 512), (384, 1024)])
-def test_decode_shapes_elementwise(M, N, K):
+def test_decode_shapes_elementwise(M, N, K, weight_prefetch):
     a = synthetic.gaussian_bf16((M, K), 1.0, seed=M * 5 + N)
     w = synthetic.gaussian_bf16((N, K), 0.02, seed=N + K)
     check_full(a, w, f"decode {M}x{N}x{K}")
@@ -117,7 +128,7 @@ def test_prefill_workloads_sampled(idx, dense_pairs):
     check_sampled(a, w, cfg.name)
 
 
-def test_decode_workloads():
+def test_decode_workloads(weight_prefetch):
     for cfg in synthetic.DECODE:
         a, w = synthetic.make_linear_inputs(cfg)
         if cfg.M <= 8:
