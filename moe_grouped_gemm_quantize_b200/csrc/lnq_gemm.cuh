@@ -86,9 +86,12 @@ struct GemmCfg {
     static constexpr int kPBytes = kP * kBK;
     static constexpr int kQRowsPerCta = PAIR ? BNQ / 2 : BNQ;
     static constexpr int kQBytes = kQRowsPerCta * kBK;
-    static constexpr int kScaleStages = SWAP ? 16 : 8;  // scale ring depth (K blocks)
+    // Scale ring depth in K blocks.  Scale copies travel the load/store path and
+    // take several microseconds to land under a full operand stream, so the ring
+    // must hold that many K blocks' worth (32 covers ~6000 cycles at ~200 per block).
+    static constexpr int kScaleStages = 32;
     // scale slot: activation scales (128 rows, or BNQ tokens), then the weight scales
-    static constexpr int kSbOffset = SWAP ? BNQ : 256;
+    static constexpr int kSbOffset = SWAP ? BNQ : 128;
     static constexpr int kScaleSlotFloats = kSbOffset + 4;
     static constexpr int kCW = BNQ / EPI_WG;      // accumulator columns per epilogue thread
     static constexpr int kEpiThreads = 128 * EPI_WG;
