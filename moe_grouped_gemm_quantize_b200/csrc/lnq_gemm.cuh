@@ -94,6 +94,9 @@ struct GemmCfg {
     static constexpr int kSbOffset = SWAP ? BNQ : 128;
     static constexpr int kScaleSlotFloats = kSbOffset + 4;
     static constexpr int kCW = BNQ / EPI_WG;      // accumulator columns per epilogue thread
+    // TMEM columns per load in the promotion (each load issued one chunk ahead)
+    static constexpr int kLdCols = 32;
+    static_assert(kCW % kLdCols == 0, "promotion chunks tile the thread's columns");
     static constexpr int kEpiThreads = 128 * EPI_WG;
     static constexpr int kThreads = 128 + kEpiThreads;
     // TMEM accumulators of BNQ columns each, as many as the 512 columns hold (at
@@ -172,7 +175,7 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32
 
 // One K block of the per-block FP32 promotion: acc += partial * scale, where
 // the partial is this thread's TMEM lane (kCW columns starting at taddr).  The
-// columns are read in chunks of 64 (32 when the slice is narrower); `release`
+// columns are read in chunks of kLdCols; `release`
 // runs as soon as the last chunk has arrived in registers, before its FMAs, so
 // the tensor core may overwrite the slice early.
 //   dense:  scale = sa[row] * sb[column block of this warpgroup]
@@ -204,20 +207,21 @@ __device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint3
         const float sb = slot[C::kSbOffset];
         s2 = make_float2(sb, sb);
     }
-    // 32-column chunks, each load issued one chunk ahead of the FMAs
-    constexpr int NC = C::kCW / 32;
-    uint32_t ra[32], rb[32];
-    tmem_ld32_async(taddr, ra);
+    // chunks of kLdCols columns, each load issued one chunk ahead of the FMAs
+    constexpr int X = C::kLdCols;
+    constexpr int NC = C::kCW / X;
+    uint32_t ra[X], rb[X];
+    tmem_ld_async(taddr, ra);
     tmem_wait_ld(ra);
     if (NC == 1) release();
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
         if (c + 1 < NC) {
-            if (c & 1) tmem_ld32_async(taddr + (c + 1) * 32, ra);
-            else tmem_ld32_async(taddr + (c + 1) * 32, rb);
+            if (c & 1) tmem_ld_async(taddr + (c + 1) * X, ra);
+            else tmem_ld_async(taddr + (c + 1) * X, rb);
         }
-        if (c & 1) promote_chunk<C, 32>(acc, rb, c * 32, slot, s2);
-        else promote_chunk<C, 32>(acc, ra, c * 32, slot, s2);
+        if (c & 1) promote_chunk<C, X>(acc, rb, c * X, slot, s2);
+        else promote_chunk<C, X>(acc, ra, c * X, slot, s2);
         if (c + 1 < NC) {
             if (c & 1) tmem_wait_ld(ra);
             else tmem_wait_ld(rb);
@@ -333,9 +337,13 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     if constexpr (C::kRegSplit) setmaxnreg_dec<56>();
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            tma_prefetch_desc(&map_p);
-            tma_prefetch_desc(&map_q);
+        // The whole warp runs the loop; one elected lane issues the copies.
+        {
+            if (elect_one()) {
+                tma_prefetch_desc(&map_p);
+                tma_prefetch_desc(&map_q);
+            }
+            __syncwarp();
             int stage = 0;
             uint32_t phase = 0;
             uint32_t filled = 0, fill_parity = 0;
@@ -351,15 +359,18 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         const TileCoord tc = tile_coord<C>(args, unit, rank);
                         if (tc.group >= 0 && !C::GROUPED) {
                             prefetched = min(C::STAGES, kb_end - kb_begin);
-                            for (int s = 0; s < prefetched; ++s) {
-                                mbar_arrive_expect_tx(full_bar(s), C::kPBytes + C::kQBytes);
-                                if constexpr (C::SWAP)
-                                    tma_load_2d(sP + s * C::kPBytes, &map_p, full_bar(s), (kb_begin + s) * C::kBK,
-                                                tc.p0);
-                                else
-                                    tma_load_2d(sQ + s * C::kQBytes, &map_q, full_bar(s), (kb_begin + s) * C::kBK,
-                                                tc.q0);
+                            if (elect_one()) {
+                                for (int s = 0; s < prefetched; ++s) {
+                                    mbar_arrive_expect_tx(full_bar(s), C::kPBytes + C::kQBytes);
+                                    if constexpr (C::SWAP)
+                                        tma_load_2d(sP + s * C::kPBytes, &map_p, full_bar(s),
+                                                    (kb_begin + s) * C::kBK, tc.p0);
+                                    else
+                                        tma_load_2d(sQ + s * C::kQBytes, &map_q, full_bar(s),
+                                                    (kb_begin + s) * C::kBK, tc.q0);
+                                }
                             }
+                            __syncwarp();
                         }
                     }
                 }
@@ -380,33 +391,41 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     if (prefetched > 0) {
                         // stage already armed and its weight half in flight: load the activations
                         if constexpr (!C::PAIR) {
-                            if constexpr (C::SWAP)
-                                tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK, q_row);
-                            else
-                                tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK, p_row);
+                            if (elect_one()) {
+                                if constexpr (C::SWAP)
+                                    tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK,
+                                                q_row);
+                                else
+                                    tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK,
+                                                p_row);
+                            }
+                            __syncwarp();
                         }
                         --prefetched;
                     } else {
-                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, wctx)) {
-                        ok = false;
-                        break;
-                    }
-                    if constexpr (C::PAIR) {
-                        // both CTAs' bytes complete on the first CTA's full barrier
-                        if (rank == 0)
-                            mbar_arrive_expect_tx(full_bar(stage), 2 * (C::kPBytes + C::kQBytes));
-                        const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
-                        tma_load_2d_pair(sP + stage * C::kPBytes, &map_p, leader_full, kb * C::kBK, p_row);
-                        // slice h of the tile's N: this CTA holds its kSliceQRows rows of it
+                        if (!mbar_wait_warp(empty_bar(stage), phase ^ 1u, wctx)) {
+                            ok = false;
+                            break;
+                        }
+                        if (elect_one()) {
+                            if constexpr (C::PAIR) {
+                                // both CTAs' bytes complete on the first CTA's full barrier
+                                if (rank == 0)
+                                    mbar_arrive_expect_tx(full_bar(stage), 2 * (C::kPBytes + C::kQBytes));
+                                const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
+                                tma_load_2d_pair(sP + stage * C::kPBytes, &map_p, leader_full, kb * C::kBK, p_row);
+                                // slice h of the tile's N: this CTA holds its kSliceQRows rows of it
 #pragma unroll
-                        for (int h = 0; h < C::kSlices; ++h)
-                            tma_load_2d_pair(sQ + stage * C::kQBytes + h * C::kSliceQRows * C::kBK, &map_q,
-                                             leader_full, kb * C::kBK, q_row + h * C::kSliceN);
-                    } else {
-                        mbar_arrive_expect_tx(full_bar(stage), C::kPBytes + C::kQBytes);
-                        tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK, p_row);
-                        tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK, q_row);
-                    }
+                                for (int h = 0; h < C::kSlices; ++h)
+                                    tma_load_2d_pair(sQ + stage * C::kQBytes + h * C::kSliceQRows * C::kBK, &map_q,
+                                                     leader_full, kb * C::kBK, q_row + h * C::kSliceN);
+                            } else {
+                                mbar_arrive_expect_tx(full_bar(stage), C::kPBytes + C::kQBytes);
+                                tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK, p_row);
+                                tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK, q_row);
+                            }
+                        }
+                        __syncwarp();
                     }
                     filled |= 1u << stage;
                     fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
@@ -426,61 +445,72 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     drain.abort = &never;
                     for (int s = 0; s < C::STAGES; ++s)
                         if (filled & (1u << s))
-                            (void)mbar_wait(full_bar(s), (fill_parity >> s) & 1u, drain);
+                            (void)mbar_wait_warp(full_bar(s), (fill_parity >> s) & 1u, drain);
                     if (C::PAIR) settle_ns(200000);
                 }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0 && rank == 0) {
+        // The whole warp runs the loop (operands stay warp-uniform); one elected
+        // lane issues the MMAs and commits.
+        if (rank == 0) {
             int stage = 0, abuf = 0;
             uint32_t phase = 0, aphase = 0;
             bool ok = true, issued = false;
+            const uint64_t adesc0 = sw128_kmajor_desc(sP);
+            const uint64_t bdesc0 = sw128_kmajor_desc(sQ);
             for (int t = unit; t < args.num_tiles && ok; t += units) {
                 const TileCoord tc = tile_coord<C>(args, t, 0);
                 if (tc.group < 0) continue;
                 for (int kb = kb_begin; kb < kb_end && ok; ++kb) {
-                    if (!mbar_wait(full_bar(stage), phase, wctx)) {
+                    if (!mbar_wait_warp(full_bar(stage), phase, wctx)) {
                         ok = false;
                         break;
                     }
-                    const uint64_t adesc = sw128_kmajor_desc(sP + stage * C::kPBytes);
+                    // descriptor start fields advance by (byte offset >> 4)
+                    const uint64_t adesc = adesc0 + static_cast<uint64_t>((stage * C::kPBytes) >> 4);
 #pragma unroll
                     for (int h = 0; h < C::kSlices; ++h) {
                         const int slot = abuf * C::kSlices + h;
-                        if (!mbar_wait(tempty_bar(slot), aphase ^ 1u, wctx)) {
+                        if (!mbar_wait_warp(tempty_bar(slot), aphase ^ 1u, wctx)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::BNQ + h * C::kSliceN);
                         const uint64_t bdesc =
-                            sw128_kmajor_desc(sQ + stage * C::kQBytes + h * C::kSliceQRows * C::kBK);
-                        if constexpr (C::PAIR) {
+                            bdesc0 + static_cast<uint64_t>((stage * C::kQBytes + h * C::kSliceQRows * C::kBK) >> 4);
+                        if (elect_one()) {
+                            if constexpr (C::PAIR) {
 #pragma unroll
-                            for (int k = 0; k < C::kBK / 32; ++k)
-                                mma_f8f6f4_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
-                                                k > 0 ? 1u : 0u);
-                            mma_commit_pair(mapa_shared(tfull_bar(slot), 0));
-                            mma_commit_pair(mapa_shared(tfull_bar(slot), 1));
-                        } else {
+                                for (int k = 0; k < C::kBK / 32; ++k)
+                                    mma_f8f6f4_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
+                                                    k > 0 ? 1u : 0u);
+                                mma_commit_pair(mapa_shared(tfull_bar(slot), 0));
+                                mma_commit_pair(mapa_shared(tfull_bar(slot), 1));
+                            } else {
 #pragma unroll
-                            for (int k = 0; k < C::kBK / 32; ++k)
-                                mma_f8f6f4(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
-                                           k > 0 ? 1u : 0u);
-                            mma_commit(tfull_bar(slot));
+                                for (int k = 0; k < C::kBK / 32; ++k)
+                                    mma_f8f6f4(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
+                                               k > 0 ? 1u : 0u);
+                                mma_commit(tfull_bar(slot));
+                            }
                         }
+                        __syncwarp();
                         issued = true;
                     }
                     if (!ok) break;
                     // the stage is free once every slice's MMAs have read it
-                    if constexpr (C::PAIR) {
-                        mma_commit_pair(mapa_shared(empty_bar(stage), 0));
-                        mma_commit_pair(mapa_shared(empty_bar(stage), 1));
-                    } else {
-                        mma_commit(empty_bar(stage));
+                    if (elect_one()) {
+                        if constexpr (C::PAIR) {
+                            mma_commit_pair(mapa_shared(empty_bar(stage), 0));
+                            mma_commit_pair(mapa_shared(empty_bar(stage), 1));
+                        } else {
+                            mma_commit(empty_bar(stage));
+                        }
                     }
+                    __syncwarp();
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -492,13 +522,16 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 }
             }
             if (issued) {
-                // every MMA this thread issued completes before TMEM is released
-                if constexpr (C::PAIR) mma_commit_pair(mapa_shared(drain_bar, 0));
-                else mma_commit(drain_bar);
+                // every MMA this warp issued completes before TMEM is released
+                if (elect_one()) {
+                    if constexpr (C::PAIR) mma_commit_pair(mapa_shared(drain_bar, 0));
+                    else mma_commit(drain_bar);
+                }
+                __syncwarp();
                 WaitCtx drain = wctx;
                 uint32_t never = 0u;
                 drain.abort = &never;
-                (void)mbar_wait(drain_bar, 0u, drain);
+                (void)mbar_wait_warp(drain_bar, 0u, drain);
             }
         }
     } else if (warp == 2) {

@@ -102,6 +102,27 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     }
 }
 
+// Every lane of the warp waits; the warp leaves with one common verdict, so that
+// the code after the wait stays warp-uniform.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+    const bool ok = mbar_wait(bar, parity, w);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Elects one lane of the (fully active) warp.  Single-thread asynchronous
+// instructions (tcgen05.mma, commits, TMA) are issued under this predicate from a
+// loop that the whole warp runs, so that their operands stay warp-uniform: issued
+// from a one-lane branch with run-time operands they cost far more issue time.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // ------------------------------------------------- asynchronous global -> shared
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -201,6 +222,27 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
         : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns from tensor memory (see tmem_ld32_async).
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
 // 32 lanes x 32 consecutive 32-bit columns from tensor memory: this thread
 // receives the 32 columns of its own lane.  The load is asynchronous: the
 // registers may be read only after tmem_wait_ld(r) on the same array.
@@ -273,6 +315,11 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[64]) {
                  :
                  : "memory");
 }
+
+// Width-generic forms of the loads above (16, 32 or 64 columns).
+__device__ __forceinline__ void tmem_ld_async(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld16_async(taddr, r); }
+__device__ __forceinline__ void tmem_ld_async(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld32_async(taddr, r); }
+__device__ __forceinline__ void tmem_ld_async(uint32_t taddr, uint32_t (&r)[64]) { tmem_ld64_async(taddr, r); }
 
 // ---------------------------------------------------------------- CTA pairs
 // A cluster of two CTAs running one tcgen05 MMA of M = 256 (cta_group::2):
