@@ -81,6 +81,15 @@ def barrier(dist):
         dist.barrier()
 
 
+def job_throughput(work_per_rank_step: float, steps: int, world: int, ms_max: float,
+                   scale: float) -> float:
+    """Whole-job throughput of a weak-scaling run: every rank processed `steps` steps of
+    `work_per_rank_step` units (FLOPs or bytes) in at most `ms_max` milliseconds (the max
+    over ranks); `scale` converts units per second to the reported unit (1e12 for TFLOP/s,
+    1e9 for GB/s)."""
+    return work_per_rank_step * steps * world / (ms_max * 1e-3) / scale
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -394,10 +403,10 @@ def run_ours(args, world, rank, local):
         barrier(dist)
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
         if is_hbm_bound(args.workload):
-            ev_val = bytes_step * Ke * world / (e_ms * 1e-3) / 1e9
+            ev_val = job_throughput(bytes_step, Ke, world, e_ms, 1e9)
             ev_unit = "GB/s"
         else:
-            ev_val = flops_step * Ke * world / (e_ms * 1e-3) / 1e12
+            ev_val = job_throughput(flops_step, Ke, world, e_ms, 1e12)
             ev_unit = "TFLOP/s"
         e2e = {"value": round(ev_val, 3), "unit": ev_unit, "steps": Ke,
                "h2d_bytes_per_step": int(sum(u.h2d_bytes for u in units)),
@@ -409,14 +418,14 @@ def run_ours(args, world, rank, local):
     peaks, peak_src = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     if is_hbm_bound(args.workload):
-        value = bytes_step * K * world / (ms * 1e-3) / 1e9
+        value = job_throughput(bytes_step, K, world, ms, 1e9)
         unit = "GB/s"
         ach = bytes_step * K / (g_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 4)}
         peak_note = f"HBM copy bandwidth ({peak_src})"
     else:
-        value = flops_step * K * world / (ms * 1e-3) / 1e12
+        value = job_throughput(flops_step, K, world, ms, 1e12)
         unit = "TFLOP/s"
         ach = flops_step * K / (g_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
@@ -474,8 +483,9 @@ def run_ours(args, world, rank, local):
 
 # --------------------------------------------------------------------------- the oracle (CPU)
 
-def oracle_sample(workload: str, rows: int):
-    """Inputs for the oracle on the first `rows` activation rows of each linear."""
+def oracle_inputs(workload: str, max_rows: int):
+    """Oracle inputs for every linear of the workload: up to `max_rows` activation rows
+    (bf16 bits) and the pre-quantized weights of the product."""
     import oracle
     from moe_grouped_gemm_quantize_b200 import synthetic
     cfgs, kind = workload_units(workload)
@@ -483,17 +493,29 @@ def oracle_sample(workload: str, rows: int):
     for c in cfgs:
         if kind == "grouped":
             a, w, m_indices, _ = synthetic.make_moe_inputs(c)
-            r = min(rows, 128)
-            a_bits = synthetic.bf16_bits(a[:r])
+            r = min(max_rows, 128)
             # the first rows belong to group 0: its weights are the product's B
             wq, ws = oracle.quantize_fp8_blocks(synthetic.bf16_bits(w[:c.N]))
-            items.append((a_bits, wq, ws, 2.0 * r * c.N * c.K))
+            items.append((synthetic.bf16_bits(a[:r]), wq, ws, 2.0 * c.N * c.K))
         else:
             a, w = synthetic.make_linear_inputs(c)
-            r = min(rows, c.M)
+            r = min(max_rows, c.M)
             wq, ws = oracle.quantize_fp8_blocks(synthetic.bf16_bits(w))
-            items.append((synthetic.bf16_bits(a[:r]), wq, ws, 2.0 * r * c.N * c.K))
+            items.append((synthetic.bf16_bits(a[:r]), wq, ws, 2.0 * c.N * c.K))
     return items
+
+
+def oracle_sample(items, rows: int, cols: int | None = None):
+    """The first `rows` activation rows of each linear, and of its output columns the
+    first `cols` (a multiple of 128; all when None).  FLOPs are counted for the sample."""
+    out = []
+    for a_bits, wq, ws, flops_per_row in items:
+        r = min(rows, a_bits.shape[0])
+        n = wq.shape[0]
+        if cols is not None and cols < n:
+            wq, ws = wq[:cols], ws[:-(-cols // 128)]
+        out.append((a_bits[:r], wq, ws, flops_per_row * r * wq.shape[0] / n))
+    return out
 
 
 def oracle_step(items):
@@ -503,21 +525,32 @@ def oracle_step(items):
         oracle.gemm_nt(qa, sa, wq, ws)
 
 
+def measure_oracle(items, dt_s: float, steps: int = 1):
+    flops = sum(it[3] for it in items) * steps
+    byts = sum(it[0].size * 3 + it[1].size + 2 * it[0].shape[0] * it[1].shape[0]
+               for it in items) * steps
+    return flops, byts
+
+
 def cpu_baseline(workload: str, target_s: float = 10.0):
-    """The oracle, as it stands, timed on this host on a bounded sample of the workload."""
+    """The oracle, as it stands, timed on this host on a bounded sample of the workload.
+
+    The sample grows (the first r activation rows of every linear) until one timed pass
+    takes at least half of `target_s`; that pass is the reported one."""
     import oracle
-    items = oracle_sample(workload, 1)
-    t = time.perf_counter()
-    oracle_step(items)
-    t1 = time.perf_counter() - t
-    rows = int(max(1, min(64, target_s / max(t1, 1e-3))))
-    items = oracle_sample(workload, rows)
-    t = time.perf_counter()
-    oracle_step(items)
-    dt = time.perf_counter() - t
-    flops = sum(it[3] for it in items)
+    full = oracle_inputs(workload, 2048)
+    max_rows = max(it[0].shape[0] for it in full)
+    rows = 1
+    while True:
+        items = oracle_sample(full, rows)
+        t = time.perf_counter()
+        oracle_step(items)
+        dt = time.perf_counter() - t
+        if dt >= 0.5 * target_s or rows >= max_rows:
+            break
+        rows = min(max_rows, max(2 * rows, int(rows * 0.8 * target_s / max(dt, 1e-3))))
+    flops, byts = measure_oracle(items, dt)
     if is_hbm_bound(workload):
-        byts = sum(it[0].size * 3 + it[1].size + 2 * it[0].shape[0] * it[1].shape[0] for it in items)
         val, unit = byts / dt / 1e9, "GB/s"
     else:
         val, unit = flops / dt / 1e12, "TFLOP/s"
@@ -532,22 +565,22 @@ def run_reference(args, world, rank, local):
         return
     import oracle
     oracle.build()
-    rows = 1
-    items = oracle_sample(args.workload, rows)
+    # each step: the first 16 activation rows x the first 1024 output columns of every
+    # linear of the workload (fewer where the workload has fewer)
+    rows, cols = 16, 1024
+    items = oracle_sample(oracle_inputs(args.workload, rows), rows, cols)
     for _ in range(args.warmup):
         oracle_step(items)
     t = time.perf_counter()
     for _ in range(args.steps):
         oracle_step(items)
     dt = time.perf_counter() - t
-    flops = sum(it[3] for it in items) * args.steps
+    flops, byts = measure_oracle(items, dt, args.steps)
     if is_hbm_bound(args.workload):
-        byts = sum(it[0].size * 3 + it[1].size + 2 * it[0].shape[0] * it[1].shape[0]
-                   for it in items) * args.steps
         val, unit = byts / dt / 1e9, "GB/s"
     else:
         val, unit = flops / dt / 1e12, "TFLOP/s"
-    sample = (f"first {rows} activation row of each linear per step "
+    sample = (f"first {rows} activation rows x first {cols} output columns of each linear per step "
               f"(quantize + FP64 product, weights pre-quantized)")
     out = {
         "impl": "reference",
@@ -582,7 +615,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-weight-prefetch", action="store_true",
                     help="GEMMs wait for the previous kernel before streaming weights")
     ap.add_argument("--cta-pairs", type=int, default=0, choices=[0, 1, 2],
