@@ -86,13 +86,17 @@ struct GemmCfg {
     static constexpr int kPBytes = kP * kBK;
     static constexpr int kQRowsPerCta = PAIR ? BNQ / 2 : BNQ;
     static constexpr int kQBytes = kQRowsPerCta * kBK;
-    // Scale ring depth in K blocks.  Scale copies travel the load/store path and
-    // take several microseconds to land under a full operand stream, so the ring
-    // must hold that many K blocks' worth (32 covers ~6000 cycles at ~200 per block).
-    static constexpr int kScaleStages = 32;
-    // scale slot: activation scales (128 rows, or BNQ tokens), then the weight scales
+    // Scale ring.  Each slot holds the scales of kScaleBatch consecutive K blocks of
+    // a tile, so the epilogue waits on (and releases) a slot once per batch.  Scale
+    // copies travel the load/store path and take several microseconds to land under
+    // a full operand stream, so the ring holds 32 K blocks' worth.
+    static constexpr int kScaleBatch = 4;
+    static constexpr int kScaleStages = 32 / kScaleBatch;
+    // per K block: activation scales (128 rows, or BNQ tokens), then the weight scales
     static constexpr int kSbOffset = SWAP ? BNQ : 128;
-    static constexpr int kScaleSlotFloats = kSbOffset + 4;
+    static constexpr int kScaleKbFloats = kSbOffset + 4;
+    static constexpr int kScaleSlotFloats = kScaleBatch * kScaleKbFloats;
+    static_assert(kScaleKbFloats % 4 == 0, "16-byte aligned scale runs");
     static constexpr int kCW = BNQ / EPI_WG;      // accumulator columns per epilogue thread
     // TMEM columns per load in the promotion (each load issued one chunk ahead)
     static constexpr int kLdCols = 32;
@@ -147,20 +151,13 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32
         c.p0 = (t % a.tiles_p) * C::kP;
         c.q0 = (t / a.tiles_p) * C::BNQ;
         c.group = 0;
-    } else if constexpr (C::GROUPED) {
-        // row-major over (128-row block, column tile): consecutive tiles share
-        // the activation block and walk one group's weights, which stay in L2
-        c.p0 = (t / a.tiles_q) * C::kP;
-        c.q0 = (t % a.tiles_q) * C::BNQ;
-        c.group = __ldg(a.m_indices + c.p0);
-        if (c.group >= a.num_groups) {
-            atomicOr(a.status, kStatusBadGroup);
-            c.group = -1;
-        }
     } else {
-        // bands of row tiles: a wave of tiles shares a band of activation rows
-        // and a few weight column tiles
-        constexpr int kBand = C::PAIR ? 8 : 16;
+        // Bands of row tiles, column-major inside a band: a wave of tiles shares a
+        // band of activation rows and a few weight column tiles.  Grouped: the
+        // 128-row blocks of one group sit next to each other, so a band's blocks of a
+        // group walk that group's weight columns together (a narrow band keeps the
+        // weights of the groups in flight within L2).
+        constexpr int kBand = (C::PAIR || C::GROUPED) ? 8 : 16;
         const int band_tiles = kBand * a.tiles_q;
         const int band = t / band_tiles;
         const int first = band * kBand;
@@ -168,7 +165,15 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32
         const int r = t - band * band_tiles;
         c.p0 = (first + r % rows) * C::kTileM + static_cast<int>(rank) * C::kP;
         c.q0 = (r / rows) * C::BNQ;
-        c.group = 0;
+        if constexpr (C::GROUPED) {
+            c.group = __ldg(a.m_indices + c.p0);
+            if (c.group >= a.num_groups) {
+                atomicOr(a.status, kStatusBadGroup);
+                c.group = -1;
+            }
+        } else {
+            c.group = 0;
+        }
     }
     return c;
 }
@@ -557,14 +562,19 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             const long long sb_row = static_cast<long long>(C::SWAP ? 0 : tc.group) * args.nb + nb_lane;
             const float* sa_src = args.sfa + a_row;
             const float* sb_src = args.sfb + sb_row * args.num_kb;
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
+            for (int kb0 = kb_begin; kb0 < kb_end; kb0 += C::kScaleBatch) {
                 if (!mbar_wait(sempty_bar(sstage), sphase ^ 1u, wctx)) {
                     ok = false;
                     break;
                 }
                 const uint32_t slot = smem_u32(scale_slots + sstage * C::kScaleSlotFloats);
-                if (lane < kSaLanes) cp_async_16(slot + lane * 16, sa_src + static_cast<long long>(kb) * args.M4);
-                if (lane < C::kSbPerTile) cp_async_4(slot + (C::kSbOffset + lane) * 4, sb_src + kb);
+                const int nkb = min(C::kScaleBatch, kb_end - kb0);
+                for (int j = 0; j < nkb; ++j) {
+                    const int kb = kb0 + j;
+                    const uint32_t sub = slot + static_cast<uint32_t>(j * C::kScaleKbFloats * 4);
+                    if (lane < kSaLanes) cp_async_16(sub + lane * 16, sa_src + static_cast<long long>(kb) * args.M4);
+                    if (lane < C::kSbPerTile) cp_async_4(sub + (C::kSbOffset + lane) * 4, sb_src + kb);
+                }
                 cp_async_arrive(sfull_bar(sstage));
                 if (++sstage == C::kScaleStages) {
                     sstage = 0;
@@ -592,21 +602,24 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             float2 acc[C::kCW / 2];
 #pragma unroll
             for (int i = 0; i < C::kCW / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+            int j = 0;  // K block within the scale slot's batch
             for (int kb = kb_begin; kb < kb_end; ++kb) {
+                const bool batch_last = (j == C::kScaleBatch - 1) || (kb + 1 == kb_end);
                 const int slot_id = abuf * C::kSlices + (C::kSlices == 1 ? 0 : wg);
-                if (!mbar_wait(sfull_bar(sstage), sphase, wctx) ||
+                if ((j == 0 && !mbar_wait(sfull_bar(sstage), sphase, wctx)) ||
                     !mbar_wait(tfull_bar(slot_id), aphase, wctx)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const float* slot = scale_slots + sstage * C::kScaleSlotFloats;
+                const float* slot = scale_slots + sstage * C::kScaleSlotFloats + j * C::kScaleKbFloats;
                 const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(abuf * C::BNQ + wg * C::kCW);
                 // the accumulator slice and the scale slot are only read, and each arrival
                 // follows the completion of those reads: no release fence is needed (one
                 // would also wait for this warp's outstanding output stores).  The slice is
                 // released as soon as its last chunk is in registers; the scale slot after
-                // the FMAs, which read per-token scales from it in the decode configuration.
+                // the last K block of its batch (after the FMAs in the decode configuration,
+                // which read per-token scales from it).
                 const uint32_t sempty = sempty_bar(sstage);
                 promote_k_block<C>(acc, taddr, slot, row, wg, [&]() {
                     tc_fence_before();
@@ -615,16 +628,25 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         if constexpr (C::PAIR) mbar_arrive_cluster_relaxed(mapa_shared(tempty_bar(slot_id), 0));
                         else mbar_arrive_relaxed(tempty_bar(slot_id));
                         // dense: the scales were read before the first TMEM load
-                        if constexpr (!C::SWAP) mbar_arrive_relaxed(sempty);
+                        if constexpr (!C::SWAP) {
+                            if (batch_last) mbar_arrive_relaxed(sempty);
+                        }
                     }
                 });
                 if constexpr (C::SWAP) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_relaxed(sempty);
+                    if (batch_last) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_relaxed(sempty);
+                    }
                 }
-                if (++sstage == C::kScaleStages) {
-                    sstage = 0;
-                    sphase ^= 1u;
+                if (batch_last) {
+                    j = 0;
+                    if (++sstage == C::kScaleStages) {
+                        sstage = 0;
+                        sphase ^= 1u;
+                    }
+                } else {
+                    ++j;
                 }
                 if (++abuf == C::kAccBufs) {
                     abuf = 0;
