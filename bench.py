@@ -189,7 +189,7 @@ class ClockSampler:
 class Linear:
     """One dense linear: bf16 activations resident on the device, weights pre-quantized."""
 
-    def __init__(self, cfg, dev):
+    def __init__(self, cfg, dev, split: bool = False):
         import moe_grouped_gemm_quantize_b200 as lnq
         from moe_grouped_gemm_quantize_b200 import synthetic
         self.cfg = cfg
@@ -210,6 +210,8 @@ class Linear:
         self.d2h_bytes = 2 * M * N
         self.host_x = self.x.cpu().pin_memory()
         self.host_d = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        # decode shapes: a workspace lets every SM share the weight stream (K split)
+        self.work = lnq.gemm_workspace(M, N, K, dev) if split else None
 
     def calls(self, stream_ptr):
         """Pre-marshalled C-ABI calls (quantize, gemm)."""
@@ -222,8 +224,11 @@ class Linear:
         qargs = (P(self.x.data_ptr()), c.M, c.K, self.x.stride(0), P(self.q.data_ptr()), c.K,
                  P(self.sfa.data_ptr()), self.M4, s)
         gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), self.M4, P(self.wq.data_ptr()),
-                 P(self.ws.data_ptr()), P(self.d.data_ptr()), c.M, c.N, c.K, s)
-        return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_fp8_block_gemm_nt, gargs)
+                 P(self.ws.data_ptr()), P(self.d.data_ptr()), c.M, c.N, c.K)
+        if self.work is not None:
+            return (L.lnq_quantize_fp8_groups, qargs), \
+                (L.lnq_fp8_block_gemm_nt_ws, gargs + (P(self.work.data_ptr()), self.work.numel(), s))
+        return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_fp8_block_gemm_nt, gargs + (s,))
 
 
 class Grouped:
@@ -314,7 +319,8 @@ def run_ours(args, world, rank, local):
     lnq.lnq_set_weight_prefetch(not args.no_weight_prefetch)
 
     cfgs, kind = workload_units(args.workload)
-    units = [Grouped(c, dev) if kind == "grouped" else Linear(c, dev) for c in cfgs]
+    units = [Grouped(c, dev) if kind == "grouped" else Linear(c, dev, split=args.split)
+             for c in cfgs]
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     calls = [u.calls(sp) for u in units]
@@ -457,6 +463,8 @@ def run_ours(args, world, rank, local):
         "config": {"workload": args.workload, "desc": WORKLOAD_DESC[args.workload],
                    "dense_cta_pairs": args.cta_pairs,
                    "weight_prefetch": not args.no_weight_prefetch,
+                   "decode_k_split": args.split and any(getattr(u, "work", None) is not None
+                                                         for u in units),
                    "parallelism": f"replicas x{world} (independent tokens per rank)",
                    "l2": "working set per step > 126 MB L2; no extra flush"},
         "roofline": roof,
@@ -616,9 +624,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--split", action="store_true",
+                    help="decode GEMMs through the workspace K split (slower than whole weight tiles "
+                         "per CTA at N = 12288 on B200)")
     ap.add_argument("--no-weight-prefetch", action="store_true",
                     help="GEMMs wait for the previous kernel before streaming weights")
-    ap.add_argument("--cta-pairs", type=int, default=0, choices=[0, 1, 2],
+    ap.add_argument("--cta-pairs", type=int, default=1, choices=[0, 1, 2],
                     help="dense GEMMs with M > 128: 0 one CTA per 128x256 tile, 1 CTA pairs on "
                          "256x256 tiles, 2 CTA pairs on 256x128 tiles")
     args = ap.parse_args()

@@ -121,6 +121,44 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
                                  int64_t N, int64_t K, void* stream);
 
 /*
+ * Bytes of workspace that lnq_fp8_block_gemm_nt_ws needs to split the K range of
+ * a decode product (M <= 64) over `num_sms` CTAs, or 0 when the product does not
+ * split (M > 64, K == 128, or at least one weight tile per SM already).  A pure
+ * host computation: no device is touched.
+ */
+int64_t lnq_fp8_block_gemm_nt_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t num_sms);
+
+/*
+ * lnq_fp8_block_gemm_nt with a caller-owned workspace for the decode split.
+ *
+ * Decode products have fewer 128-row weight tiles than the GPU has SMs (96 for
+ * N = 12288).  With a workspace, every SM takes an equal contiguous run of the
+ * (weight tile, 128-wide K block) units; a CTA that covers part of a tile's K
+ * range writes its FP32 partial tile into the workspace and counts itself in the
+ * tile's counter, and the CTA that completes the count adds the tile's partials
+ * in order of their K ranges (a fixed order: the result does not depend on
+ * timing), stores the bf16 tile and resets the counter.  The FP32 promotion per
+ * 128-wide K block is the same as in lnq_fp8_block_gemm_nt; only the grouping of
+ * the block sums differs, so results agree within FP32 rounding.
+ *
+ *   workspace        device memory of at least
+ *                    lnq_fp8_block_gemm_nt_workspace_bytes(M, N, K, SMs of the
+ *                    current device) bytes, 256-byte aligned, ZEROED before its
+ *                    first use; every call leaves its counters zero again.  The
+ *                    caller owns it.  Calls that share a workspace must be ordered
+ *                    (one stream); after an error (LNQ_ERR_TIMEOUT) zero it again.
+ *   workspace_bytes  its size.
+ *   Other arguments and requirements as lnq_fp8_block_gemm_nt.  With workspace ==
+ *   NULL, or for products that do not split, this is lnq_fp8_block_gemm_nt.  A
+ *   workspace smaller than needed returns LNQ_ERR_INVALID_ARG, a misaligned one
+ *   LNQ_ERR_MISALIGNED, before any launch.
+ */
+lnq_status lnq_fp8_block_gemm_nt_ws(const void* a_e4m3, const float* sfa, int64_t M4,
+                                    const void* b_e4m3, const float* sfb, void* d_bf16, int64_t M,
+                                    int64_t N, int64_t K, void* workspace, int64_t workspace_bytes,
+                                    void* stream);
+
+/*
  * M-grouped contiguous block-scaled FP8 GEMM (MoE experts): tokens of all
  * groups concatenated along M, every group starting at a multiple of 128
  * rows, a per-row group id (deepgemm-rust README, "Grouped (contiguous) MoE
@@ -172,10 +210,11 @@ lnq_status lnq_get_last_device_error(void* stream);
 lnq_status lnq_selftest_wait_timeout(int64_t timeout_ns, void* stream);
 
 /*
- * Tuning knob (process-wide, default 0) for dense GEMMs with M > 128:
+ * Tuning knob (process-wide, default 1) for dense GEMMs with M > 128:
  *   0  one CTA per 128 x 256 tile (N >= 256);
  *   1  pairs of CTAs (a cluster of two sharing one tcgen05 MMA) on 256 x 256
- *      tiles, each CTA loading half of the weight tile (N >= 256);
+ *      tiles, each CTA loading half of the weight tile (N >= 256); the
+ *      default: it halves the weight bytes each SM loads per K block;
  *   2  pairs of CTAs on 256 x 128 tiles with four accumulators per CTA
  *      (N >= 128).
  * Other values select 0.  Results are the same up to FP32 summation order.

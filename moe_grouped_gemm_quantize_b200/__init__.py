@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
             "lnq_quantize_fp8_groups": [P, I64, I64, I64, P, I64, P, I64, P],
             "lnq_quantize_fp8_blocks": [P, I64, I64, P, P, P],
             "lnq_fp8_block_gemm_nt": [P, P, I64, P, P, P, I64, I64, I64, P],
+            "lnq_fp8_block_gemm_nt_ws": [P, P, I64, P, P, P, I64, I64, I64, P, I64, P],
             "lnq_m_grouped_fp8_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
             "lnq_get_last_device_error": [P],
             "lnq_selftest_wait_timeout": [I64, P],
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.lnq_status_string.argtypes = [ctypes.c_int]
         L.lnq_status_string.restype = ctypes.c_char_p
         L.lnq_abi_version.restype = ctypes.c_int32
+        L.lnq_fp8_block_gemm_nt_workspace_bytes.argtypes = [I64, I64, I64, I32]
+        L.lnq_fp8_block_gemm_nt_workspace_bytes.restype = I64
         for knob in ("lnq_set_dense_cta_pairs", "lnq_set_weight_prefetch"):
             getattr(L, knob).argtypes = [ctypes.c_int32]
             getattr(L, knob).restype = ctypes.c_int32
@@ -164,6 +167,47 @@ def lnq_fp8_block_gemm_nt(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, s
         raise ValueError("inconsistent shapes")
     _check(lib().lnq_fp8_block_gemm_nt(_ptr(a), _ptr(sfa), sfa.shape[1], _ptr(b), _ptr(sfb), _ptr(d),
                                        M, N, K, _stream(stream)), "lnq_fp8_block_gemm_nt")
+
+
+def lnq_fp8_block_gemm_nt_workspace_bytes(M: int, N: int, K: int, num_sms: int) -> int:
+    """Workspace bytes for the decode K split over num_sms CTAs (0: the product does not split)."""
+    return int(lib().lnq_fp8_block_gemm_nt_workspace_bytes(M, N, K, num_sms))
+
+
+def gemm_workspace(M: int, N: int, K: int, device) -> torch.Tensor | None:
+    """A zeroed workspace for lnq_fp8_block_gemm_nt_ws on `device`, or None when the
+    product does not split.  The library leaves it zeroed after every call."""
+    dev = torch.device(device)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    n = lnq_fp8_block_gemm_nt_workspace_bytes(M, N, K, sms)
+    if n == 0:
+        return None
+    return torch.zeros(n, dtype=torch.uint8, device=dev)
+
+
+def lnq_fp8_block_gemm_nt_ws(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                             d: torch.Tensor, workspace: torch.Tensor | None, stream=None) -> None:
+    """lnq_fp8_block_gemm_nt with the decode K split over a caller-owned workspace
+    (uint8 tensor from gemm_workspace, or None for the unsplit product)."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.float32 or \
+            sfb.dtype != torch.float32 or d.dtype != torch.bfloat16:
+        raise TypeError("a, b float8_e4m3fn/uint8; sfa, sfb float32; d bf16")
+    M, K = a.shape
+    N = b.shape[0]
+    for t in (a, sfa, b, sfb, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    if b.shape[1] != K or tuple(d.shape) != (M, N) or sfa.shape[0] != K // 128 or \
+            tuple(sfb.shape) != (-(-N // 128), K // 128):
+        raise ValueError("inconsistent shapes")
+    if workspace is None:
+        ws, ws_bytes = ctypes.c_void_p(0), 0
+    else:
+        if workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+            raise TypeError("workspace: contiguous uint8 tensor")
+        ws, ws_bytes = _ptr(workspace), workspace.numel()
+    _check(lib().lnq_fp8_block_gemm_nt_ws(_ptr(a), _ptr(sfa), sfa.shape[1], _ptr(b), _ptr(sfb), _ptr(d),
+                                          M, N, K, ws, ws_bytes, _stream(stream)), "lnq_fp8_block_gemm_nt_ws")
 
 
 def lnq_m_grouped_fp8_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,

@@ -41,7 +41,7 @@ struct DeviceInfo {
 
 std::mutex g_mutex;
 // Dense GEMMs with M > 128 run on CTA pairs when set (1: 256x256, 2: 256x128 tiles).
-std::atomic<int> g_dense_pairs{0};
+std::atomic<int> g_dense_pairs{1};
 // GEMMs may start streaming weights before the prior kernel completes.
 std::atomic<int> g_weight_prefetch{0};
 DeviceInfo g_devices[kMaxDevices];
@@ -159,7 +159,9 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
             return LNQ_ERR_CUDA;
         return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
     }
-    const int grid = args.num_tiles < dev.sm_count ? args.num_tiles : dev.sm_count;
+    // whole tiles per CTA, or (split) every CTA a run of the (tile, K block) units
+    const long long work = C::SPLITK ? static_cast<long long>(args.num_tiles) * args.num_kb : args.num_tiles;
+    const int grid = static_cast<int>(work < dev.sm_count ? work : dev.sm_count);
     if (grid <= 0) return LNQ_OK;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -186,6 +188,8 @@ using CfgGrouped256 = GemmCfg<256, 4, 2, false, true>;
 using CfgGrouped128 = GemmCfg<128, 6, 2, false, true>;
 using CfgSwap32 = GemmCfg<32, 10, 1, true, false>;
 using CfgSwap64 = GemmCfg<64, 8, 1, true, false>;
+using CfgSwap32Split = GemmCfg<32, 10, 1, true, false, false, 1, true>;
+using CfgSwap64Split = GemmCfg<64, 8, 1, true, false, false, 1, true>;
 
 constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
 
@@ -306,9 +310,43 @@ lnq_status lnq_quantize_fp8_blocks(const void* w_bf16, int64_t N, int64_t K, voi
     return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
 }
 
-lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4,
-                                 const void* b_e4m3, const float* sfb, void* d_bf16, int64_t M,
-                                 int64_t N, int64_t K, void* stream) {
+namespace {
+
+// Layout of the split workspace for one decode product, or need_bytes == 0 when the
+// product does not split: [partials: tiles * max_slots * 128 * BNQ fp32][counters:
+// tiles int32], each part starting on a 256-byte boundary.
+struct SplitPlan {
+    int64_t need_bytes = 0;
+    int64_t counters_offset = 0;
+    int max_slots = 0;
+};
+
+SplitPlan plan_split(int64_t M, int64_t N, int64_t K, int64_t num_sms) {
+    SplitPlan plan;
+    if (M <= 0 || M > 64 || N <= 0 || K <= 0 || K % 128 != 0 || num_sms <= 0) return plan;
+    const int64_t bnq = M <= 32 ? 32 : 64;
+    const int64_t tiles = ((N + 127) / 128) * ((M + bnq - 1) / bnq);
+    const int64_t nkb = K / 128;
+    // only where whole tiles would leave SMs idle and a tile has K blocks to share
+    if (tiles >= num_sms || nkb < 2) return plan;
+    const int64_t U = tiles * nkb;
+    const int64_t G = U < num_sms ? U : num_sms;
+    auto owner = [&](int64_t x) { return ((x + 1) * G + U - 1) / U - 1; };
+    int64_t slots = 0;
+    for (int64_t t = 0; t < tiles; ++t) {
+        const int64_t n = owner((t + 1) * nkb - 1) - owner(t * nkb) + 1;
+        if (n > slots) slots = n;
+    }
+    auto round256 = [](int64_t b) { return (b + 255) / 256 * 256; };
+    plan.max_slots = static_cast<int>(slots);
+    plan.counters_offset = round256(tiles * slots * 128 * bnq * 4);
+    plan.need_bytes = plan.counters_offset + round256(tiles * 4);
+    return plan;
+}
+
+lnq_status gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4, const void* b_e4m3,
+                   const float* sfb, void* d_bf16, int64_t M, int64_t N, int64_t K,
+                   void* workspace, int64_t workspace_bytes, void* stream) {
     if (M <= 0 || N <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
     if (K % 128 != 0 || N % 16 != 0 || N < 16 || M > kMaxRows || N > kMaxRows ||
         K > (int64_t{1} << 31))
@@ -336,6 +374,23 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
     if (M <= 64) {
         // decode: weights in the MMA's 128-row slot, tokens padded to 32 or 64
         args.tiles_p = static_cast<int>((N + 127) / 128);
+        const SplitPlan plan = plan_split(M, N, K, dev->sm_count);
+        if (workspace != nullptr && plan.need_bytes > 0) {
+            if (workspace_bytes < plan.need_bytes) return LNQ_ERR_INVALID_ARG;
+            if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return LNQ_ERR_MISALIGNED;
+            // all SMs share the (tile, K block) units; partial tiles meet in the workspace
+            args.partials = static_cast<float*>(workspace);
+            args.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + plan.counters_offset);
+            args.max_slots = plan.max_slots;
+            if (M <= 32) {
+                args.tiles_q = static_cast<int>((M + 31) / 32);
+                args.num_tiles = args.tiles_p * args.tiles_q;
+                return launch_gemm<CfgSwap32Split>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
+            }
+            args.tiles_q = static_cast<int>((M + 63) / 64);
+            args.num_tiles = args.tiles_p * args.tiles_q;
+            return launch_gemm<CfgSwap64Split>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
+        }
         if (M <= 32) {
             args.tiles_q = static_cast<int>((M + 31) / 32);
             args.num_tiles = args.tiles_p * args.tiles_q;
@@ -369,6 +424,26 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
     args.tiles_q = static_cast<int>((N + 127) / 128);
     args.num_tiles = args.tiles_p * args.tiles_q;
     return launch_gemm<CfgDense128>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
+}
+
+}  // namespace
+
+lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4,
+                                 const void* b_e4m3, const float* sfb, void* d_bf16, int64_t M,
+                                 int64_t N, int64_t K, void* stream) {
+    return gemm_nt(a_e4m3, sfa, M4, b_e4m3, sfb, d_bf16, M, N, K, nullptr, 0, stream);
+}
+
+int64_t lnq_fp8_block_gemm_nt_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t num_sms) {
+    return plan_split(M, N, K, num_sms).need_bytes;
+}
+
+lnq_status lnq_fp8_block_gemm_nt_ws(const void* a_e4m3, const float* sfa, int64_t M4,
+                                    const void* b_e4m3, const float* sfb, void* d_bf16, int64_t M,
+                                    int64_t N, int64_t K, void* workspace, int64_t workspace_bytes,
+                                    void* stream) {
+    if (workspace_bytes < 0) return LNQ_ERR_INVALID_ARG;
+    return gemm_nt(a_e4m3, sfa, M4, b_e4m3, sfb, d_bf16, M, N, K, workspace, workspace_bytes, stream);
 }
 
 lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sfa,

@@ -60,12 +60,18 @@ struct GemmArgs {
     int tiles_q;      // tiles along the MMA N slot
     int num_tiles;
     int prefetch_weights;  // issue the first weight stages before waiting on the prior kernel
+    // Split configuration only: the grid's CTAs share the num_tiles * num_kb (tile, K
+    // block) units in contiguous runs; a CTA that covers part of a tile leaves an FP32
+    // partial tile in `partials` and counts itself in `counters`.
+    float* partials;  // [num_tiles][max_slots][128][BNQ]
+    int* counters;    // [num_tiles], zero before and after every launch
+    int max_slots;    // most CTAs sharing one tile
 };
 
 constexpr unsigned int kStatusBadGroup = 2u;
 
 template <int BNQ_, int STAGES_, int EPI_WG_, bool SWAP_, bool GROUPED_, bool PAIR_ = false,
-          int SLICES_ = 1>
+          int SLICES_ = 1, bool SPLITK_ = false>
 struct GemmCfg {
     static constexpr int BNQ = BNQ_;   // MMA N (the whole pair's N for PAIR)
     static constexpr int STAGES = STAGES_;
@@ -73,6 +79,9 @@ struct GemmCfg {
     static constexpr bool SWAP = SWAP_;
     static constexpr bool GROUPED = GROUPED_;
     static constexpr bool PAIR = PAIR_;
+    // decode only: (tile, K block) units shared in contiguous runs by all CTAs
+    static constexpr bool SPLITK = SPLITK_;
+    static_assert(!SPLITK || SWAP, "the K split serves the decode configuration");
     static_assert(!(SWAP && GROUPED), "decode configuration is dense only");
     static_assert(!(PAIR && (SWAP || GROUPED)), "CTA pairs serve the dense configuration");
     static_assert(BNQ % 16 == 0 && BNQ >= 16 && BNQ <= 256, "MMA N for M=128/256");
@@ -128,7 +137,7 @@ struct GemmCfg {
     static constexpr int kOffQ = kOffP + STAGES * kPBytes;
     static constexpr int kOffScale = kOffQ + STAGES * kQBytes;
     static constexpr int kOffBar = kOffScale + kScaleStages * kScaleSlotFloats * 4;
-    static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs * kSlices + 2 * kScaleStages + 1;
+    static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs * kSlices + 2 * kScaleStages + 1 + (SPLITK ? 2 : 0);
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -136,6 +145,44 @@ struct GemmCfg {
                   "TMEM allocation is a power of two between 32 and 512 columns");
     static_assert(kQBytes % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
 };
+
+// A run of K blocks [kb_lo, kb_hi) of tile t.  Without the split each CTA takes
+// whole tiles unit, unit + units, ...; with it, CTA `unit` of `units` takes the
+// (tile, K block) units [unit*U/units, (unit+1)*U/units), U = num_tiles * num_kb,
+// which covers at most two tiles partly.
+struct Segment {
+    int t;
+    int kb_lo;
+    int kb_hi;
+};
+
+template <class C>
+__device__ __forceinline__ bool segment(const GemmArgs& a, int unit, int units, int i, Segment& s) {
+    if constexpr (C::SPLITK) {
+        const long long nkb = a.num_kb;
+        const long long U = static_cast<long long>(a.num_tiles) * nkb;
+        const long long u0 = static_cast<long long>(unit) * U / units;
+        const long long u1 = static_cast<long long>(unit + 1) * U / units;
+        const long long t = u0 / nkb + i;
+        if (t * nkb >= u1) return false;
+        s.t = static_cast<int>(t);
+        s.kb_lo = static_cast<int>(u0 > t * nkb ? u0 - t * nkb : 0);
+        s.kb_hi = static_cast<int>(u1 - t * nkb < nkb ? u1 - t * nkb : nkb);
+        return true;
+    } else {
+        const int t = unit + i * units;
+        if (t >= a.num_tiles) return false;
+        s.t = t;
+        s.kb_lo = 0;
+        s.kb_hi = a.num_kb;
+        return true;
+    }
+}
+
+// The CTA whose run holds unit x: the largest c with floor(c*U/units) <= x.
+__device__ __forceinline__ int unit_owner(long long x, long long U, int units) {
+    return static_cast<int>(((x + 1) * units + U - 1) / U) - 1;
+}
 
 struct TileCoord {
     int p0;     // first row of this CTA's P operand (activation row, or weight row for SWAP)
@@ -283,6 +330,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         return bars + 8u * (2 * C::STAGES + 2 * kSlots + C::kScaleStages + s);
     };
     const uint32_t drain_bar = bars + 8u * (2 * C::STAGES + 2 * kSlots + 2 * C::kScaleStages);
+    // split configuration: partial tile written by every epilogue warp; count taken
+    const uint32_t fix_bar = drain_bar + 8u;
+    const uint32_t dec_bar = drain_bar + 16u;
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile uint32_t* abort_flag = misc + 1;
 
@@ -292,8 +342,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;
     const int unit = C::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int units = C::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
-    const int kb_begin = 0;
-    const int kb_end = args.num_kb;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -309,6 +357,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             mbar_init(sempty_bar(s), C::kEpiThreads / 32);
         }
         mbar_init(drain_bar, 1);
+        if constexpr (C::SPLITK) {
+            mbar_init(fix_bar, C::kEpiThreads / 32);
+            mbar_init(dec_bar, 1);
+        }
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -330,7 +382,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     // own, and this one waits for the previous kernel before reading any input
     // (the producer may first prefetch weights, see below)
     launch_dependents();
-    if (!(args.prefetch_weights && warp == 0)) wait_prior_grids();
+    if (!(args.prefetch_weights && (warp == 0 || warp == 3))) wait_prior_grids();
 
     WaitCtx wctx;
     wctx.abort = abort_flag;
@@ -340,10 +392,15 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     if (warp < 4) {
     // control warpgroup: registers handed to the epilogue warpgroups
     if constexpr (C::kRegSplit) setmaxnreg_dec<56>();
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        // The whole warp runs the loop; one elected lane issues the copies.
-        {
+    if (warp == 0 || warp == 3) {
+        // ------------------------------------------------------------ TMA producers
+        // Two warps share the ring, warp 0 filling the even stages and warp 3 the odd
+        // ones: issuing one stage (a wait, an expect-tx arrival and the copies) keeps
+        // a warp busy for several hundred cycles, more than one K block's MMA on the
+        // smaller tiles.  Each warp runs its loop whole and one elected lane issues.
+        const int pidx = (warp == 0) ? 0 : 1;
+        constexpr int kProducers = (C::STAGES % 2 == 0) ? 2 : 1;
+        if (pidx < kProducers) {
             if (elect_one()) {
                 tma_prefetch_desc(&map_p);
                 tma_prefetch_desc(&map_q);
@@ -360,19 +417,20 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             int prefetched = 0;
             if (args.prefetch_weights) {
                 if constexpr (!C::PAIR) {
-                    if (unit < args.num_tiles) {
-                        const TileCoord tc = tile_coord<C>(args, unit, rank);
+                    Segment sg0;
+                    if (segment<C>(args, unit, units, 0, sg0)) {
+                        const TileCoord tc = tile_coord<C>(args, sg0.t, rank);
                         if (tc.group >= 0 && !C::GROUPED) {
-                            prefetched = min(C::STAGES, kb_end - kb_begin);
+                            prefetched = min(C::STAGES, sg0.kb_hi - sg0.kb_lo);
                             if (elect_one()) {
-                                for (int s = 0; s < prefetched; ++s) {
+                                for (int s = pidx; s < prefetched; s += kProducers) {
                                     mbar_arrive_expect_tx(full_bar(s), C::kPBytes + C::kQBytes);
                                     if constexpr (C::SWAP)
                                         tma_load_2d(sP + s * C::kPBytes, &map_p, full_bar(s),
-                                                    (kb_begin + s) * C::kBK, tc.p0);
+                                                    (sg0.kb_lo + s) * C::kBK, tc.p0);
                                     else
                                         tma_load_2d(sQ + s * C::kQBytes, &map_q, full_bar(s),
-                                                    (kb_begin + s) * C::kBK, tc.q0);
+                                                    (sg0.kb_lo + s) * C::kBK, tc.q0);
                                 }
                             }
                             __syncwarp();
@@ -381,8 +439,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 }
                 wait_prior_grids();
             }
-            for (int t = unit; t < args.num_tiles && ok; t += units) {
-                const TileCoord tc = tile_coord<C>(args, t, rank);
+            Segment sg;
+            for (int i = 0; ok && segment<C>(args, unit, units, i, sg); ++i) {
+                const TileCoord tc = tile_coord<C>(args, sg.t, rank);
                 if (tc.group < 0) continue;
                 int p_row, q_row;
                 if constexpr (C::SWAP) {
@@ -392,8 +451,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     p_row = tc.p0;
                     q_row = tc.group * args.N + tc.q0 + static_cast<int>(rank) * C::kSliceQRows;
                 }
-                for (int kb = kb_begin; kb < kb_end; ++kb) {
-                    if (prefetched > 0) {
+                for (int kb = sg.kb_lo; kb < sg.kb_hi; ++kb) {
+                    if (stage % kProducers != pidx) {
+                        // the other producer's stage
+                        if (prefetched > 0) --prefetched;
+                    } else if (prefetched > 0) {
                         // stage already armed and its weight half in flight: load the activations
                         if constexpr (!C::PAIR) {
                             if (elect_one()) {
@@ -432,8 +494,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         }
                         __syncwarp();
                     }
-                    filled |= 1u << stage;
-                    fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+                    if (stage % kProducers == pidx) {
+                        filled |= 1u << stage;
+                        fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+                    }
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -465,10 +529,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             bool ok = true, issued = false;
             const uint64_t adesc0 = sw128_kmajor_desc(sP);
             const uint64_t bdesc0 = sw128_kmajor_desc(sQ);
-            for (int t = unit; t < args.num_tiles && ok; t += units) {
-                const TileCoord tc = tile_coord<C>(args, t, 0);
+            Segment sg;
+            for (int i = 0; ok && segment<C>(args, unit, units, i, sg); ++i) {
+                const TileCoord tc = tile_coord<C>(args, sg.t, 0);
                 if (tc.group < 0) continue;
-                for (int kb = kb_begin; kb < kb_end && ok; ++kb) {
+                for (int kb = sg.kb_lo; kb < sg.kb_hi && ok; ++kb) {
                     if (!mbar_wait_warp(full_bar(stage), phase, wctx)) {
                         ok = false;
                         break;
@@ -551,8 +616,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         uint32_t sphase = 0;
         bool ok = true;
         constexpr int kSaLanes = C::kSaPerTile / 4;  // lanes that copy 16 bytes of sa
-        for (int t = unit; t < args.num_tiles && ok; t += units) {
-            const TileCoord tc = tile_coord<C>(args, t, rank);
+        Segment sg;
+        for (int i = 0; ok && segment<C>(args, unit, units, i, sg); ++i) {
+            const TileCoord tc = tile_coord<C>(args, sg.t, rank);
             if (tc.group < 0) continue;
             // activation rows of the tile (tokens for SWAP) and weight scale rows
             long long a_row = (C::SWAP ? tc.q0 : tc.p0) + lane * 4;
@@ -562,13 +628,13 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             const long long sb_row = static_cast<long long>(C::SWAP ? 0 : tc.group) * args.nb + nb_lane;
             const float* sa_src = args.sfa + a_row;
             const float* sb_src = args.sfb + sb_row * args.num_kb;
-            for (int kb0 = kb_begin; kb0 < kb_end; kb0 += C::kScaleBatch) {
+            for (int kb0 = sg.kb_lo; kb0 < sg.kb_hi; kb0 += C::kScaleBatch) {
                 if (!mbar_wait(sempty_bar(sstage), sphase ^ 1u, wctx)) {
                     ok = false;
                     break;
                 }
                 const uint32_t slot = smem_u32(scale_slots + sstage * C::kScaleSlotFloats);
-                const int nkb = min(C::kScaleBatch, kb_end - kb0);
+                const int nkb = min(C::kScaleBatch, sg.kb_hi - kb0);
                 for (int j = 0; j < nkb; ++j) {
                     const int kb = kb0 + j;
                     const uint32_t sub = slot + static_cast<uint32_t>(j * C::kScaleKbFloats * 4);
@@ -595,16 +661,18 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
         int sstage = 0, abuf = 0;
         uint32_t sphase = 0, aphase = 0;
+        uint32_t fix_phase = 0;
         bool ok = true;
-        for (int t = unit; t < args.num_tiles && ok; t += units) {
-            const TileCoord tc = tile_coord<C>(args, t, rank);
+        Segment sg;
+        for (int i = 0; ok && segment<C>(args, unit, units, i, sg); ++i) {
+            const TileCoord tc = tile_coord<C>(args, sg.t, rank);
             if (tc.group < 0) continue;
             float2 acc[C::kCW / 2];
 #pragma unroll
             for (int i = 0; i < C::kCW / 2; ++i) acc[i] = make_float2(0.f, 0.f);
             int j = 0;  // K block within the scale slot's batch
-            for (int kb = kb_begin; kb < kb_end; ++kb) {
-                const bool batch_last = (j == C::kScaleBatch - 1) || (kb + 1 == kb_end);
+            for (int kb = sg.kb_lo; kb < sg.kb_hi; ++kb) {
+                const bool batch_last = (j == C::kScaleBatch - 1) || (kb + 1 == sg.kb_hi);
                 const int slot_id = abuf * C::kSlices + (C::kSlices == 1 ? 0 : wg);
                 if ((j == 0 && !mbar_wait(sfull_bar(sstage), sphase, wctx)) ||
                     !mbar_wait(tfull_bar(slot_id), aphase, wctx)) {
@@ -654,6 +722,68 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 }
             }
             if (!ok) break;
+            if constexpr (C::SPLITK) {
+                if (sg.kb_lo != 0 || sg.kb_hi != args.num_kb) {
+                    // Part of the tile's K range: leave the FP32 partial in this CTA's slot
+                    // of the tile and count it; the CTA that completes the count sums the
+                    // slots in order of their K ranges (so the result does not depend on
+                    // which CTA finishes last), stores the tile and rezeroes the count.
+                    const long long nkb = args.num_kb;
+                    const long long U = static_cast<long long>(args.num_tiles) * nkb;
+                    const int first = unit_owner(static_cast<long long>(sg.t) * nkb, U, units);
+                    const int last = unit_owner(static_cast<long long>(sg.t + 1) * nkb - 1, U, units);
+                    const int n_parts = last - first + 1;
+                    const int slot = unit - first;
+                    auto part = [&](int sl) {
+                        return reinterpret_cast<float4*>(
+                            args.partials +
+                            ((static_cast<long long>(sg.t) * args.max_slots + sl) * C::kP + row) * C::kCW);
+                    };
+                    float4* mine = part(slot);
+#pragma unroll
+                    for (int i4 = 0; i4 < C::kCW / 4; ++i4)
+                        mine[i4] = make_float4(acc[2 * i4].x, acc[2 * i4].y, acc[2 * i4 + 1].x, acc[2 * i4 + 1].y);
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(fix_bar);
+                    if (ew == 0) {
+                        // every epilogue warp has written and fenced its rows: count this CTA
+                        if (mbar_wait_warp(fix_bar, fix_phase, wctx)) {
+                            if (lane == 0) {
+                                const int before = atomicAdd(args.counters + sg.t, 1);
+                                const bool completes = (before == n_parts - 1);
+                                if (completes) args.counters[sg.t] = 0;
+                                misc[2] = completes ? 1u : 0u;
+                                __threadfence();
+                            }
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(dec_bar);
+                        } else {
+                            ok = false;
+                        }
+                    }
+                    if (ok) ok = mbar_wait(dec_bar, fix_phase, wctx);
+                    fix_phase ^= 1u;
+                    if (!ok) break;
+                    if (*reinterpret_cast<volatile uint32_t*>(misc + 2) == 0u) continue;  // another CTA stores
+                    __threadfence();
+                    // every slot of the tile, in order of K
+                    for (int sl = 0; sl < n_parts; ++sl) {
+                        const float4* p = part(sl);
+#pragma unroll
+                        for (int i4 = 0; i4 < C::kCW / 4; ++i4) {
+                            const float4 v = __ldcg(p + i4);
+                            if (sl == 0) {
+                                acc[2 * i4] = make_float2(v.x, v.y);
+                                acc[2 * i4 + 1] = make_float2(v.z, v.w);
+                            } else {
+                                acc[2 * i4] = __fadd2_rn(acc[2 * i4], make_float2(v.x, v.y));
+                                acc[2 * i4 + 1] = __fadd2_rn(acc[2 * i4 + 1], make_float2(v.z, v.w));
+                            }
+                        }
+                    }
+                }
+            }
             // ---- store the tile
             if constexpr (!C::SWAP) {
                 const int m = tc.p0 + row;

@@ -34,7 +34,7 @@ def L():
 
 def declared_functions():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:lnq_status|const char\*|int32_t)\s+(lnq_\w+)\s*\(", text,
+    return sorted(set(re.findall(r"^\s*(?:lnq_status|const char\*|int32_t|int64_t)\s+(lnq_\w+)\s*\(", text,
                                  flags=re.M)))
 
 

@@ -151,3 +151,104 @@ def test_timeout_path_reports_and_recovers():
     assert lnq.lnq_get_last_device_error() == 0
     a, w = synthetic.make_linear_inputs(synthetic.TINY)
     check_full(a, w, "tiny after timeout")
+
+
+# ---------------------------------------------------------------- decode K split
+
+def gpu_linear_split(a: torch.Tensor, w: torch.Tensor):
+    wq, ws = lnq.quantize_weights(w.to(DEV))
+    aq, sa = lnq.quantize_activations(a.to(DEV))
+    M, N, K = a.shape[0], w.shape[0], a.shape[1]
+    work = lnq.gemm_workspace(M, N, K, DEV)
+    d = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lnq.lnq_fp8_block_gemm_nt_ws(aq, sa, wq, ws, d, work)
+    assert lnq.lnq_get_last_device_error() == 0
+    return d, work, (aq, sa, wq, ws)
+
+
+def counters_zero(work: torch.Tensor, M: int, N: int) -> bool:
+    # the counters sit after the partial tiles, one int32 per weight tile
+    bnq = 32 if M <= 32 else 64
+    tiles = -(-N // 128) * -(-M // bnq)
+    tail = -(-(tiles * 4) // 256) * 256
+    counters = work[work.numel() - tail:].view(torch.int32)[:tiles]
+    return bool((counters == 0).all())
+
+
+@pytest.mark.parametrize("M", [1, 5, 32, 33, 64])
+@pytest.mark.parametrize("N,K", [(256, 1024), (400, 2048), (1152, 4096)])
+def test_decode_split_elementwise(M, N, K, weight_prefetch):
+    a = synthetic.gaussian_bf16((M, K), 1.0, seed=3 * M + N)
+    w = synthetic.gaussian_bf16((N, K), 0.02, seed=N + 7 * K)
+    d, work, _ = gpu_linear_split(a, w)
+    assert work is not None, "this product must take the split path"
+    ref, _ = oracle_linear(a, w)
+    assert_gemm_close(to_f64(d), ref, f"split {M}x{N}x{K}")
+    torch.cuda.synchronize()
+    assert counters_zero(work, M, N)
+
+
+def test_decode_split_is_deterministic_and_reuses_its_workspace():
+    M, N, K = 64, 1152, 4096
+    a = synthetic.gaussian_bf16((M, K), 1.0, 11)
+    w = synthetic.gaussian_bf16((N, K), 0.02, 12)
+    d1, work, (aq, sa, wq, ws) = gpu_linear_split(a, w)
+    d2 = torch.empty_like(d1)
+    for _ in range(3):
+        lnq.lnq_fp8_block_gemm_nt_ws(aq, sa, wq, ws, d2, work)
+    torch.cuda.synchronize()
+    assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+    assert counters_zero(work, M, N)
+
+
+def test_decode_split_workloads(weight_prefetch):
+    for cfg in synthetic.DECODE:
+        a, w = synthetic.make_linear_inputs(cfg)
+        d, work, (aq, sa, wq, ws) = gpu_linear_split(a, w)
+        assert work is not None
+        qa, sao = oracle_quantize_a(a)
+        qb, sbo = oracle_quantize_w(w)
+        if cfg.M <= 8:
+            ref = oracle.gemm_nt(qa, sao, qb, sbo)
+            assert_gemm_close(to_f64(d), ref, cfg.name + " split")
+        else:
+            rows, cols = sample_points(cfg.M, cfg.N, 20000, 0, full_row=cfg.M - 1, full_col=cfg.N // 2 + 1)
+            ref = oracle.gemm_nt_points(qa, sao, qb, sbo, rows, cols)
+            assert_gemm_close(to_f64(d)[rows, cols], ref, cfg.name + " split")
+        torch.cuda.synchronize()
+        assert counters_zero(work, cfg.M, cfg.N)
+
+
+def test_workspace_call_without_a_split_is_the_plain_product():
+    # no workspace, or a product that does not split, takes the unsplit kernel
+    a = synthetic.gaussian_bf16((64, 1024), 1.0, 21)
+    w = synthetic.gaussian_bf16((256, 1024), 0.02, 22)
+    d_plain, (aq, sa, wq, ws) = gpu_linear(a, w)
+    d = torch.empty_like(d_plain)
+    lnq.lnq_fp8_block_gemm_nt_ws(aq, sa, wq, ws, d, None)
+    torch.cuda.synchronize()
+    assert torch.equal(d.view(torch.int16), d_plain.view(torch.int16))
+    a2 = synthetic.gaussian_bf16((200, 512), 1.0, 23)
+    w2 = synthetic.gaussian_bf16((256, 512), 0.02, 24)
+    assert lnq.gemm_workspace(200, 256, 512, DEV) is None
+    d2_plain, (aq2, sa2, wq2, ws2) = gpu_linear(a2, w2)
+    d2 = torch.empty_like(d2_plain)
+    lnq.lnq_fp8_block_gemm_nt_ws(aq2, sa2, wq2, ws2, d2, torch.zeros(256, dtype=torch.uint8, device=DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(d2.view(torch.int16), d2_plain.view(torch.int16))
+
+
+def test_workspace_errors_are_reported_before_launch():
+    a = synthetic.gaussian_bf16((8, 1024), 1.0, 31)
+    w = synthetic.gaussian_bf16((256, 1024), 0.02, 32)
+    _, (aq, sa, wq, ws) = gpu_linear(a, w)
+    d = torch.empty((8, 256), dtype=torch.bfloat16, device=DEV)
+    need = lnq.lnq_fp8_block_gemm_nt_workspace_bytes(8, 256, 1024, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert need > 0
+    small = torch.zeros(need - 256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(lnq.LnqError):
+        lnq.lnq_fp8_block_gemm_nt_ws(aq, sa, wq, ws, d, small)
+    big = torch.zeros(need + 256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(lnq.LnqError):
+        lnq.lnq_fp8_block_gemm_nt_ws(aq, sa, wq, ws, d, big[16:])   # not 256-byte aligned
+    assert lnq.lnq_get_last_device_error() == 0
