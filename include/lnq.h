@@ -144,9 +144,12 @@ int64_t lnq_fp8_block_gemm_nt_workspace_bytes(int64_t M, int64_t N, int64_t K, i
  *   workspace        device memory of at least
  *                    lnq_fp8_block_gemm_nt_workspace_bytes(M, N, K, SMs of the
  *                    current device) bytes, 256-byte aligned, ZEROED before its
- *                    first use; every call leaves its counters zero again.  The
- *                    caller owns it.  Calls that share a workspace must be ordered
- *                    (one stream); after an error (LNQ_ERR_TIMEOUT) zero it again.
+ *                    first use.  Its first 4 KiB hold one counter per weight tile
+ *                    and every call leaves them zero again; the partial tiles
+ *                    follow.  So one workspace, sized for the largest product, serves
+ *                    any sequence of products.  The caller owns it.  Calls that share
+ *                    a workspace must be ordered (one stream); after an error
+ *                    (LNQ_ERR_TIMEOUT) zero it again.
  *   workspace_bytes  its size.
  *   Other arguments and requirements as lnq_fp8_block_gemm_nt.  With workspace ==
  *   NULL, or for products that do not split, this is lnq_fp8_block_gemm_nt.  A

@@ -198,6 +198,7 @@ constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
 
 using namespace lnq;
 
+
 extern "C" {
 
 int32_t lnq_abi_version(void) { return 10000; }
@@ -313,11 +314,15 @@ lnq_status lnq_quantize_fp8_blocks(const void* w_bf16, int64_t N, int64_t K, voi
 namespace {
 
 // Layout of the split workspace for one decode product, or need_bytes == 0 when the
-// product does not split: [partials: tiles * max_slots * 128 * BNQ fp32][counters:
-// tiles int32], each part starting on a 256-byte boundary.
+// product does not split: [counters: one int32 per tile in a fixed 4 KiB region]
+// [partials: tiles * max_slots * 128 * BNQ fp32 from byte 4096].  The counters sit
+// at the same place for every shape, so one workspace (zeroed once) serves any
+// sequence of products: each call rezeroes the counters it used, and no call writes
+// partial tiles over another shape's counters.
+constexpr int64_t kSplitCounterBytes = 4096;
 struct SplitPlan {
     int64_t need_bytes = 0;
-    int64_t counters_offset = 0;
+    int64_t partials_offset = kSplitCounterBytes;
     int max_slots = 0;
 };
 
@@ -328,7 +333,7 @@ SplitPlan plan_split(int64_t M, int64_t N, int64_t K, int64_t num_sms) {
     const int64_t tiles = ((N + 127) / 128) * ((M + bnq - 1) / bnq);
     const int64_t nkb = K / 128;
     // only where whole tiles would leave SMs idle and a tile has K blocks to share
-    if (tiles >= num_sms || nkb < 2) return plan;
+    if (tiles >= num_sms || nkb < 2 || tiles * 4 > kSplitCounterBytes) return plan;
     const int64_t U = tiles * nkb;
     const int64_t G = U < num_sms ? U : num_sms;
     auto owner = [&](int64_t x) { return ((x + 1) * G + U - 1) / U - 1; };
@@ -339,8 +344,7 @@ SplitPlan plan_split(int64_t M, int64_t N, int64_t K, int64_t num_sms) {
     }
     auto round256 = [](int64_t b) { return (b + 255) / 256 * 256; };
     plan.max_slots = static_cast<int>(slots);
-    plan.counters_offset = round256(tiles * slots * 128 * bnq * 4);
-    plan.need_bytes = plan.counters_offset + round256(tiles * 4);
+    plan.need_bytes = kSplitCounterBytes + round256(tiles * slots * 128 * bnq * 4);
     return plan;
 }
 
@@ -379,8 +383,8 @@ lnq_status gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4, const void*
             if (workspace_bytes < plan.need_bytes) return LNQ_ERR_INVALID_ARG;
             if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return LNQ_ERR_MISALIGNED;
             // all SMs share the (tile, K block) units; partial tiles meet in the workspace
-            args.partials = static_cast<float*>(workspace);
-            args.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + plan.counters_offset);
+            args.counters = static_cast<int*>(workspace);
+            args.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.partials_offset);
             args.max_slots = plan.max_slots;
             if (M <= 32) {
                 args.tiles_q = static_cast<int>((M + 31) / 32);

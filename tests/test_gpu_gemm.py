@@ -167,12 +167,8 @@ def gpu_linear_split(a: torch.Tensor, w: torch.Tensor):
 
 
 def counters_zero(work: torch.Tensor, M: int, N: int) -> bool:
-    # the counters sit after the partial tiles, one int32 per weight tile
-    bnq = 32 if M <= 32 else 64
-    tiles = -(-N // 128) * -(-M // bnq)
-    tail = -(-(tiles * 4) // 256) * 256
-    counters = work[work.numel() - tail:].view(torch.int32)[:tiles]
-    return bool((counters == 0).all())
+    # the counters fill the workspace's first 4 KiB, one int32 per weight tile
+    return bool((work[:4096].view(torch.int32) == 0).all())
 
 
 @pytest.mark.parametrize("M", [1, 5, 32, 33, 64])
@@ -252,3 +248,27 @@ def test_workspace_errors_are_reported_before_launch():
     with pytest.raises(lnq.LnqError):
         lnq.lnq_fp8_block_gemm_nt_ws(aq, sa, wq, ws, d, big[16:])   # not 256-byte aligned
     assert lnq.lnq_get_last_device_error() == 0
+
+
+def test_one_workspace_serves_products_of_different_shapes():
+    # sized for the largest product, zeroed once, then used by products whose
+    # partial tiles and counters have other extents
+    shapes = [(64, 12288, 4096), (8, 1152, 4096), (33, 400, 2048), (1, 2048, 8192), (64, 12288, 4096)]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    size = max(lnq.lnq_fp8_block_gemm_nt_workspace_bytes(M, N, K, sms) for M, N, K in shapes)
+    work = torch.zeros(size, dtype=torch.uint8, device=DEV)
+    for i, (M, N, K) in enumerate(shapes):
+        a = synthetic.gaussian_bf16((M, K), 1.0, seed=100 + i)
+        w = synthetic.gaussian_bf16((N, K), 0.02, seed=200 + i)
+        wq, ws = lnq.quantize_weights(w.to(DEV))
+        aq, sa = lnq.quantize_activations(a.to(DEV))
+        d = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+        lnq.lnq_fp8_block_gemm_nt_ws(aq, sa, wq, ws, d, work)
+        torch.cuda.synchronize()
+        assert lnq.lnq_get_last_device_error() == 0
+        qa, sao = oracle_quantize_a(a)
+        qb, sbo = oracle_quantize_w(w)
+        rows, cols = sample_points(M, N, 4000, i, full_row=M - 1, full_col=N // 2)
+        ref = oracle.gemm_nt_points(qa, sao, qb, sbo, rows, cols)
+        assert_gemm_close(to_f64(d)[rows, cols], ref, f"shared workspace {M}x{N}x{K}")
+        assert counters_zero(work, M, N)
