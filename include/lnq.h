@@ -162,6 +162,28 @@ lnq_status lnq_fp8_block_gemm_nt_ws(const void* a_e4m3, const float* sfa, int64_
                                     void* stream);
 
 /*
+ * lnq_fp8_block_gemm_nt_ws with the library's own fixed scratch instead of a
+ * caller's workspace: this entry point allocates nothing.  The pages have no
+ * counterpart; it exists for callers that may not allocate device memory around
+ * the call.
+ *
+ * The scratch is one file-scope device array of 10 MiB (10485760 bytes) per
+ * device, whose address is looked up once per device.  Products whose split needs
+ * more (lnq_fp8_block_gemm_nt_workspace_bytes above 10 MiB; M = 64, N = 12288,
+ * K = 4096 needs 9.0 MiB) return LNQ_ERR_UNSUPPORTED_SHAPE before any launch;
+ * products that do not split run lnq_fp8_block_gemm_nt.
+ *
+ * The array is shared by every call on the device: calls that overlap in time (on
+ * different streams, or from several threads without ordering) race on it and
+ * must not be issued.  After a call the array keeps that call's partial tiles
+ * (its counters are zero again); after LNQ_ERR_TIMEOUT the counters may not be
+ * zero and later results of this entry point are undefined.
+ */
+lnq_status lnq_fp8_block_gemm_nt_static_ws(const void* a_e4m3, const float* sfa, int64_t M4,
+                                           const void* b_e4m3, const float* sfb, void* d_bf16,
+                                           int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
  * M-grouped contiguous block-scaled FP8 GEMM (MoE experts): tokens of all
  * groups concatenated along M, every group starting at a multiple of 128
  * rows, a per-row group id (deepgemm-rust README, "Grouped (contiguous) MoE

@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "lnq_quantize_fp8_blocks": [P, I64, I64, P, P, P],
             "lnq_fp8_block_gemm_nt": [P, P, I64, P, P, P, I64, I64, I64, P],
             "lnq_fp8_block_gemm_nt_ws": [P, P, I64, P, P, P, I64, I64, I64, P, I64, P],
+            "lnq_fp8_block_gemm_nt_static_ws": [P, P, I64, P, P, P, I64, I64, I64, P],
             "lnq_m_grouped_fp8_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
             "lnq_get_last_device_error": [P],
             "lnq_selftest_wait_timeout": [I64, P],
@@ -183,6 +184,26 @@ def gemm_workspace(M: int, N: int, K: int, device) -> torch.Tensor | None:
     if n == 0:
         return None
     return torch.zeros(n, dtype=torch.uint8, device=dev)
+
+
+def lnq_fp8_block_gemm_nt_static_ws(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                                    d: torch.Tensor, stream=None) -> None:
+    """lnq_fp8_block_gemm_nt_ws with the library's fixed 10 MiB device scratch (no allocation;
+    calls must not overlap in time)."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.float32 or \
+            sfb.dtype != torch.float32 or d.dtype != torch.bfloat16:
+        raise TypeError("a, b float8_e4m3fn/uint8; sfa, sfb float32; d bf16")
+    M, K = a.shape
+    N = b.shape[0]
+    for t in (a, sfa, b, sfb, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    if b.shape[1] != K or tuple(d.shape) != (M, N) or sfa.shape[0] != K // 128 or \
+            tuple(sfb.shape) != (-(-N // 128), K // 128):
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_fp8_block_gemm_nt_static_ws(_ptr(a), _ptr(sfa), sfa.shape[1], _ptr(b), _ptr(sfb),
+                                                 _ptr(d), M, N, K, _stream(stream)),
+           "lnq_fp8_block_gemm_nt_static_ws")
 
 
 def lnq_fp8_block_gemm_nt_ws(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,

@@ -198,6 +198,14 @@ constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
 
 using namespace lnq;
 
+// Scratch of lnq_fp8_block_gemm_nt_static_ws: the decode K split's partial tiles and
+// counters in a fixed device array (zero when the module loads; every call leaves the
+// counters zero), so that entry point allocates nothing.  Calls on several streams
+// would share it: they must not overlap.
+static constexpr int64_t kStaticSplitBytes = int64_t{10} << 20;
+static __device__ __align__(256) unsigned char g_static_split_scratch[kStaticSplitBytes];
+static void* g_static_split_addr[64] = {};
+static std::mutex g_static_split_mutex;
 
 extern "C" {
 
@@ -448,6 +456,31 @@ lnq_status lnq_fp8_block_gemm_nt_ws(const void* a_e4m3, const float* sfa, int64_
                                     void* stream) {
     if (workspace_bytes < 0) return LNQ_ERR_INVALID_ARG;
     return gemm_nt(a_e4m3, sfa, M4, b_e4m3, sfb, d_bf16, M, N, K, workspace, workspace_bytes, stream);
+}
+
+lnq_status lnq_fp8_block_gemm_nt_static_ws(const void* a_e4m3, const float* sfa, int64_t M4,
+                                           const void* b_e4m3, const float* sfb, void* d_bf16,
+                                           int64_t M, int64_t N, int64_t K, void* stream) {
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    int devno = 0;
+    if (cudaGetDevice(&devno) != cudaSuccess) return LNQ_ERR_CUDA;
+    const int64_t need = plan_split(M, N, K, dev->sm_count).need_bytes;
+    if (need > kStaticSplitBytes) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    void* ws = nullptr;
+    if (need > 0) {
+        std::lock_guard<std::mutex> lock(g_static_split_mutex);
+        if (g_static_split_addr[devno] == nullptr) {
+            // the device address of the file-scope scratch array, once per device
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_static_split_scratch) != cudaSuccess || p == nullptr)
+                return LNQ_ERR_CUDA;
+            g_static_split_addr[devno] = p;
+        }
+        ws = g_static_split_addr[devno];
+    }
+    return gemm_nt(a_e4m3, sfa, M4, b_e4m3, sfb, d_bf16, M, N, K, ws, kStaticSplitBytes, stream);
 }
 
 lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sfa,
