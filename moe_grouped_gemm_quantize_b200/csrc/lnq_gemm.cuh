@@ -81,6 +81,8 @@ struct GemmCfg {
     static constexpr bool PAIR = PAIR_;
     // decode only: (tile, K block) units shared in contiguous runs by all CTAs
     static constexpr bool SPLITK = SPLITK_;
+    // decode: two warps issue MMAs (alternate K blocks), one produces
+    static constexpr bool kDualMma = SWAP;
     static_assert(!SPLITK || SWAP, "the K split serves the decode configuration");
     static_assert(!(SWAP && GROUPED), "decode configuration is dense only");
     static_assert(!(PAIR && (SWAP || GROUPED)), "CTA pairs serve the dense configuration");
@@ -356,7 +358,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             mbar_init(sfull_bar(s), 32);
             mbar_init(sempty_bar(s), C::kEpiThreads / 32);
         }
-        mbar_init(drain_bar, 1);
+        mbar_init(drain_bar, C::kDualMma ? 2 : 1);
         if constexpr (C::SPLITK) {
             mbar_init(fix_bar, C::kEpiThreads / 32);
             mbar_init(dec_bar, 1);
@@ -392,14 +394,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     if (warp < 4) {
     // control warpgroup: registers handed to the epilogue warpgroups
     if constexpr (C::kRegSplit) setmaxnreg_dec<56>();
-    if (warp == 0 || warp == 3) {
+    if (warp == 0 || (warp == 3 && !C::kDualMma)) {
         // ------------------------------------------------------------ TMA producers
         // Two warps share the ring, warp 0 filling the even stages and warp 3 the odd
         // ones: issuing one stage (a wait, an expect-tx arrival and the copies) keeps
-        // a warp busy for several hundred cycles, more than one K block's MMA on the
-        // smaller tiles.  Each warp runs its loop whole and one elected lane issues.
+        // a warp busy for several hundred cycles.  Each warp runs its loop whole and
+        // one elected lane issues.  (Decode: warp 3 issues MMAs instead.)
         const int pidx = (warp == 0) ? 0 : 1;
-        constexpr int kProducers = (C::STAGES % 2 == 0) ? 2 : 1;
+        constexpr int kProducers = (C::STAGES % 2 == 0 && !C::kDualMma) ? 2 : 1;
         if (pidx < kProducers) {
             if (elect_one()) {
                 tma_prefetch_desc(&map_p);
@@ -519,12 +521,18 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 }
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || (warp == 3 && C::kDualMma)) {
+        // ------------------------------------------------------------ MMA issuer(s)
         // The whole warp runs the loop (operands stay warp-uniform); one elected
-        // lane issues the MMAs and commits.
+        // lane issues the MMAs and commits.  Decode tiles are so narrow that issuing a
+        // K block's MMAs and commits takes longer than the tensor core needs for them:
+        // there warps 1 and 3 take alternate K blocks (each K block has its own stage
+        // and accumulator, so the two streams are independent).
+        const int midx = (warp == 1) ? 0 : 1;
+        constexpr int kIssuers = C::kDualMma ? 2 : 1;
         if (rank == 0) {
             int stage = 0, abuf = 0;
+            int gk = 0;  // K blocks seen, for the alternation
             uint32_t phase = 0, aphase = 0;
             bool ok = true, issued = false;
             const uint64_t adesc0 = sw128_kmajor_desc(sP);
@@ -534,6 +542,18 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 const TileCoord tc = tile_coord<C>(args, sg.t, 0);
                 if (tc.group < 0) continue;
                 for (int kb = sg.kb_lo; kb < sg.kb_hi && ok; ++kb) {
+                    if (gk++ % kIssuers != midx) {
+                        // the other issuer's K block
+                        if (++stage == C::STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                        if (++abuf == C::kAccBufs) {
+                            abuf = 0;
+                            aphase ^= 1u;
+                        }
+                        continue;
+                    }
                     if (!mbar_wait_warp(full_bar(stage), phase, wctx)) {
                         ok = false;
                         break;
@@ -591,8 +611,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     }
                 }
             }
-            if (issued) {
-                // every MMA this warp issued completes before TMEM is released
+            if (issued || kIssuers > 1) {
+                // every MMA this warp issued completes before TMEM is released (with two
+                // issuers both always commit: the barrier counts two arrivals)
                 if (elect_one()) {
                     if constexpr (C::PAIR) mma_commit_pair(mapa_shared(drain_bar, 0));
                     else mma_commit(drain_bar);
