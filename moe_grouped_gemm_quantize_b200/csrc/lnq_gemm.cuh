@@ -81,8 +81,6 @@ struct GemmCfg {
     static constexpr bool PAIR = PAIR_;
     // decode only: (tile, K block) units shared in contiguous runs by all CTAs
     static constexpr bool SPLITK = SPLITK_;
-    // decode: two warps issue MMAs (alternate K blocks), one produces
-    static constexpr bool kDualMma = SWAP;
     static_assert(!SPLITK || SWAP, "the K split serves the decode configuration");
     static_assert(!(SWAP && GROUPED), "decode configuration is dense only");
     static_assert(!(PAIR && (SWAP || GROUPED)), "CTA pairs serve the dense configuration");
@@ -358,7 +356,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             mbar_init(sfull_bar(s), 32);
             mbar_init(sempty_bar(s), C::kEpiThreads / 32);
         }
-        mbar_init(drain_bar, C::kDualMma ? 2 : 1);
+        mbar_init(drain_bar, 2);
         if constexpr (C::SPLITK) {
             mbar_init(fix_bar, C::kEpiThreads / 32);
             mbar_init(dec_bar, 1);
@@ -384,7 +382,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     // own, and this one waits for the previous kernel before reading any input
     // (the producer may first prefetch weights, see below)
     launch_dependents();
-    if (!(args.prefetch_weights && (warp == 0 || warp == 3))) wait_prior_grids();
+    if (!(args.prefetch_weights && warp == 0)) wait_prior_grids();
 
     WaitCtx wctx;
     wctx.abort = abort_flag;
@@ -394,15 +392,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     if (warp < 4) {
     // control warpgroup: registers handed to the epilogue warpgroups
     if constexpr (C::kRegSplit) setmaxnreg_dec<56>();
-    if (warp == 0 || (warp == 3 && !C::kDualMma)) {
-        // ------------------------------------------------------------ TMA producers
-        // Two warps share the ring, warp 0 filling the even stages and warp 3 the odd
-        // ones: issuing one stage (a wait, an expect-tx arrival and the copies) keeps
-        // a warp busy for several hundred cycles.  Each warp runs its loop whole and
-        // one elected lane issues.  (Decode: warp 3 issues MMAs instead.)
-        const int pidx = (warp == 0) ? 0 : 1;
-        constexpr int kProducers = (C::STAGES % 2 == 0 && !C::kDualMma) ? 2 : 1;
-        if (pidx < kProducers) {
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        // The whole warp runs the loop; one elected lane issues the copies.
+        {
             if (elect_one()) {
                 tma_prefetch_desc(&map_p);
                 tma_prefetch_desc(&map_q);
@@ -425,7 +418,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         if (tc.group >= 0 && !C::GROUPED) {
                             prefetched = min(C::STAGES, sg0.kb_hi - sg0.kb_lo);
                             if (elect_one()) {
-                                for (int s = pidx; s < prefetched; s += kProducers) {
+                                for (int s = 0; s < prefetched; ++s) {
                                     mbar_arrive_expect_tx(full_bar(s), C::kPBytes + C::kQBytes);
                                     if constexpr (C::SWAP)
                                         tma_load_2d(sP + s * C::kPBytes, &map_p, full_bar(s),
@@ -454,10 +447,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     q_row = tc.group * args.N + tc.q0 + static_cast<int>(rank) * C::kSliceQRows;
                 }
                 for (int kb = sg.kb_lo; kb < sg.kb_hi; ++kb) {
-                    if (stage % kProducers != pidx) {
-                        // the other producer's stage
-                        if (prefetched > 0) --prefetched;
-                    } else if (prefetched > 0) {
+                    if (prefetched > 0) {
                         // stage already armed and its weight half in flight: load the activations
                         if constexpr (!C::PAIR) {
                             if (elect_one()) {
@@ -496,10 +486,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         }
                         __syncwarp();
                     }
-                    if (stage % kProducers == pidx) {
-                        filled |= 1u << stage;
-                        fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
-                    }
+                    filled |= 1u << stage;
+                    fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -521,20 +509,21 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 }
             }
         }
-    } else if (warp == 1 || (warp == 3 && C::kDualMma)) {
-        // ------------------------------------------------------------ MMA issuer(s)
+    } else if (warp == 1 || warp == 3) {
+        // ------------------------------------------------------------ MMA issuers
         // The whole warp runs the loop (operands stay warp-uniform); one elected
-        // lane issues the MMAs and commits.  Decode tiles are so narrow that issuing a
-        // K block's MMAs and commits takes longer than the tensor core needs for them:
-        // there warps 1 and 3 take alternate K blocks (each K block has its own stage
-        // and accumulator, so the two streams are independent).
+        // lane issues the MMAs and commits.  Issuing a K block (two barrier waits,
+        // four MMAs, two commits) keeps a warp busy about as long as the tensor core
+        // needs for a 128 x 256 K block, and longer for the narrow decode tiles, so
+        // warps 1 and 3 take alternate K blocks (each K block has its own stage and
+        // accumulator: the two streams are independent).
         const int midx = (warp == 1) ? 0 : 1;
-        constexpr int kIssuers = C::kDualMma ? 2 : 1;
+        constexpr int kIssuers = 2;
         if (rank == 0) {
             int stage = 0, abuf = 0;
             int gk = 0;  // K blocks seen, for the alternation
             uint32_t phase = 0, aphase = 0;
-            bool ok = true, issued = false;
+            bool ok = true;
             const uint64_t adesc0 = sw128_kmajor_desc(sP);
             const uint64_t bdesc0 = sw128_kmajor_desc(sQ);
             Segment sg;
@@ -588,7 +577,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                             }
                         }
                         __syncwarp();
-                        issued = true;
                     }
                     if (!ok) break;
                     // the stage is free once every slice's MMAs have read it
@@ -611,9 +599,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     }
                 }
             }
-            if (issued || kIssuers > 1) {
-                // every MMA this warp issued completes before TMEM is released (with two
-                // issuers both always commit: the barrier counts two arrivals)
+            {
+                // every MMA this warp issued completes before TMEM is released (both
+                // issuers always commit: the barrier counts two arrivals)
                 if (elect_one()) {
                     if constexpr (C::PAIR) mma_commit_pair(mapa_shared(drain_bar, 0));
                     else mma_commit(drain_bar);
