@@ -72,6 +72,11 @@ def _load():
         lib.oracle_m_grouped_gemm_points.restype = ctypes.c_int
         lib.oracle_m_grouped_gemm_points.argtypes = [
             P, P, P, P, P, ctypes.c_int32, I64, I64, I64, P, P, I64, P]
+        lib.oracle_m_grouped_gemm_masked.restype = ctypes.c_int
+        lib.oracle_m_grouped_gemm_masked.argtypes = [P, P, I64, P, P, P, ctypes.c_int32, I64, I64, I64, P]
+        lib.oracle_m_grouped_gemm_masked_points.restype = ctypes.c_int
+        lib.oracle_m_grouped_gemm_masked_points.argtypes = [
+            P, P, I64, P, P, P, ctypes.c_int32, I64, I64, I64, P, P, I64, P]
         _lib = lib
         return lib
 
@@ -206,4 +211,43 @@ def m_grouped_gemm_points(qa, sfa, qb, sfb, m_indices, num_groups: int, rows, co
     _check(_load().oracle_m_grouped_gemm_points(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(mi),
                                                 num_groups, M_total, N, K, _ptr(rows), _ptr(cols),
                                                 rows.size, _ptr(out)), "m_grouped_gemm_points")
+    return out
+
+
+def m_grouped_gemm_masked(qa, sfa, qb, sfb, masked_m, M_max: int) -> np.ndarray:
+    """FP64 D [G*M_max, N] of the masked grouped product: group g's first masked_m[g]
+    rows (rows g*M_max ...) against group g's weights; other rows are NaN.  qa is
+    [G*M_max, K], sfa [K/128, M4] over those rows, qb [G*N, K]."""
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    sfa = _c(sfa, np.float32)
+    sfb = _c(sfb, np.float32)
+    mm = _c(np.asarray(masked_m, dtype=np.int32), np.int32)
+    G = mm.size
+    total, K = qa.shape
+    if total != G * M_max:
+        raise ValueError("qa must hold G * M_max rows")
+    N = qb.shape[0] // G
+    D = np.full((total, N), np.nan, dtype=np.float64)
+    _check(_load().oracle_m_grouped_gemm_masked(_ptr(qa), _ptr(sfa), sfa.shape[1], _ptr(qb), _ptr(sfb),
+                                                _ptr(mm), G, M_max, N, K, _ptr(D)), "m_grouped_gemm_masked")
+    return D
+
+
+def m_grouped_gemm_masked_points(qa, sfa, qb, sfb, masked_m, M_max: int, rows, cols) -> np.ndarray:
+    """The masked grouped product at (rows[i], cols[i]); NaN past a group's count."""
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    sfa = _c(sfa, np.float32)
+    sfb = _c(sfb, np.float32)
+    mm = _c(np.asarray(masked_m, dtype=np.int32), np.int32)
+    rows = _c(np.asarray(rows, dtype=np.int64), np.int64)
+    cols = _c(np.asarray(cols, dtype=np.int64), np.int64)
+    G = mm.size
+    total, K = qa.shape
+    N = qb.shape[0] // G
+    out = np.empty(rows.shape, dtype=np.float64)
+    _check(_load().oracle_m_grouped_gemm_masked_points(_ptr(qa), _ptr(sfa), sfa.shape[1], _ptr(qb), _ptr(sfb),
+                                                       _ptr(mm), G, M_max, N, K, _ptr(rows), _ptr(cols),
+                                                       rows.size, _ptr(out)), "m_grouped_gemm_masked_points")
     return out

@@ -32,6 +32,12 @@
  *     (G*n, k) and weight scales (G*ceil(n/128), ceil(k/128)): deepgemm-rust
  *     README, "Grouped (contiguous) MoE GEMM" and "What's implemented";
  *     Triton_Grouped_GEMM README, "Example DeepGEMM layout creation".
+ *   - M-grouped masked layout (the per-expert output of a token dispatch):
+ *     group g owns rows g*M_max .. g*M_max + M_max - 1 of A and D, of which
+ *     only the first masked_m[g] are real; the counts stay on the device:
+ *     deepgemm-rust README, "What's implemented", m_grouped_fp8_gemm_nt_masked
+ *     (masked_m scheduler, DeepEP-style dispatch output, zero CPU sync).  The
+ *     weights and their scales are laid out as in the contiguous variant.
  *   - E4M3 round-to-nearest-even with saturation at 448, scale = amax/448:
  *     the benchmark spec's numerics (the pages never print 448; the encoder
  *     below is written from the OCP FP8 E4M3 format definition: bias 7,
@@ -405,6 +411,90 @@ int oracle_m_grouped_gemm_points(const uint8_t* qa, const float* sfa, const uint
             }
             dequant_a_row(qa, sfa, M_total, K, rows[i], ad);
             dequant_b_row(qb, sfb, K, g * N + n, g * NB + n / ORACLE_GROUP, bd);
+            out[i] = dot(ad, bd, K);
+        }
+        free(ad);
+        free(bd);
+    }
+    return 0;
+}
+
+/* M-grouped masked product: for each group g and each of its first masked_m[g]
+ * rows m, D[g*M_max + m][n] = sum_k (value(qa[row,k]) * sfa[k/128][row]) *
+ * (value(qb[g*N + n, k]) * sfb[g*ceil(N/128) + n/128][k/128]), row = g*M_max + m,
+ * in FP64.  qa is [G*M_max][K]; sfa is [K/128][M4] over those G*M_max rows (M4 >=
+ * G*M_max).  Rows past masked_m[g] are not written.  Returns -1 if a count lies
+ * outside [0, M_max]. */
+int oracle_m_grouped_gemm_masked(const uint8_t* qa, const float* sfa, int64_t M4, const uint8_t* qb,
+                                 const float* sfb, const int32_t* masked_m, int32_t G, int64_t M_max,
+                                 int64_t N, int64_t K, double* D)
+{
+    int64_t g, NB, total;
+    if (G <= 0 || M_max <= 0 || N <= 0 || K <= 0 || K % ORACLE_GROUP != 0 || M4 < G * M_max)
+        return -1;
+    for (g = 0; g < G; ++g)
+        if (masked_m[g] < 0 || masked_m[g] > M_max)
+            return -1;
+    NB = (N + ORACLE_GROUP - 1) / ORACLE_GROUP;
+    total = G * M_max;
+#pragma omp parallel
+    {
+        double* ad = (double*)malloc(sizeof(double) * (size_t)K);
+        double* bd = (double*)malloc(sizeof(double) * (size_t)K);
+        int64_t r;
+#pragma omp for schedule(dynamic, 1)
+        for (r = 0; r < total; ++r) {
+            int64_t n, gr = r / M_max, m = r % M_max;
+            if (m >= masked_m[gr] || !ad || !bd)
+                continue;
+            dequant_a_row(qa, sfa, M4, K, r, ad);
+            for (n = 0; n < N; ++n) {
+                dequant_b_row(qb, sfb, K, gr * N + n, gr * NB + n / ORACLE_GROUP, bd);
+                D[r * N + n] = dot(ad, bd, K);
+            }
+        }
+        free(ad);
+        free(bd);
+    }
+    return 0;
+}
+
+/* The masked product at chosen points (rows index the G*M_max rows); a point on a
+ * row past its group's count yields NaN. */
+int oracle_m_grouped_gemm_masked_points(const uint8_t* qa, const float* sfa, int64_t M4,
+                                        const uint8_t* qb, const float* sfb,
+                                        const int32_t* masked_m, int32_t G, int64_t M_max,
+                                        int64_t N, int64_t K, const int64_t* rows,
+                                        const int64_t* cols, int64_t count, double* out)
+{
+    int64_t i, g, NB;
+    int bad = 0;
+    if (G <= 0 || M_max <= 0 || N <= 0 || K <= 0 || K % ORACLE_GROUP != 0 || M4 < G * M_max)
+        return -1;
+    for (g = 0; g < G; ++g)
+        if (masked_m[g] < 0 || masked_m[g] > M_max)
+            return -1;
+    for (i = 0; i < count; ++i)
+        if (rows[i] < 0 || rows[i] >= G * M_max || cols[i] < 0 || cols[i] >= N)
+            bad = 1;
+    if (bad)
+        return -1;
+    NB = (N + ORACLE_GROUP - 1) / ORACLE_GROUP;
+#pragma omp parallel
+    {
+        double* ad = (double*)malloc(sizeof(double) * (size_t)K);
+        double* bd = (double*)malloc(sizeof(double) * (size_t)K);
+#pragma omp for schedule(dynamic, 16)
+        for (i = 0; i < count; ++i) {
+            int64_t gr = rows[i] / M_max, m = rows[i] % M_max, n = cols[i];
+            if (!ad || !bd)
+                continue;
+            if (m >= masked_m[gr]) {
+                out[i] = NAN;
+                continue;
+            }
+            dequant_a_row(qa, sfa, M4, K, rows[i], ad);
+            dequant_b_row(qb, sfb, K, gr * N + n, gr * NB + n / ORACLE_GROUP, bd);
             out[i] = dot(ad, bd, K);
         }
         free(ad);
