@@ -272,6 +272,51 @@ class Grouped:
         return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_m_grouped_fp8_gemm_contiguous, gargs)
 
 
+class Masked:
+    """The M-grouped masked MoE GEMM: 32 expert buffers of 128 rows, 2048 routed tokens."""
+
+    def __init__(self, cfg, dev):
+        import moe_grouped_gemm_quantize_b200 as lnq
+        from moe_grouped_gemm_quantize_b200 import synthetic
+        self.cfg = cfg
+        a, w, counts = synthetic.make_moe_masked_inputs(cfg)
+        G, Mm, N, K = cfg.groups, cfg.m_max, cfg.N, cfg.K
+        self.M = G * Mm
+        self.x = a.to(dev)
+        self.wq, self.ws = lnq.quantize_weights_grouped(w.to(dev), G)
+        del w
+        self.mm = torch.from_numpy(counts).to(dev)
+        real = int(counts.sum())
+        busy = int((counts > 0).sum())
+        self.q = torch.empty((self.M, K), dtype=torch.float8_e4m3fn, device=dev)
+        self.sfa = torch.empty((K // 128, self.M), dtype=torch.float32, device=dev)
+        self.d = torch.empty((self.M, N), dtype=torch.bfloat16, device=dev)
+        self.flops = cfg.flops   # real rows only
+        # algorithmic: real activation rows and their scales, the weights and weight
+        # scales of the experts with tokens, the real output rows, the counts
+        self.gemm_bytes = (real * K + 4 * (K // 128) * real + busy * N * K
+                           + 4 * busy * (-(-N // 128)) * (K // 128) + 2 * real * N + 4 * G)
+        self.quant_bytes = 3 * self.M * K + 4 * (K // 128) * self.M
+        self.h2d_bytes = 2 * self.M * K
+        self.d2h_bytes = 2 * self.M * N
+        self.host_x = self.x.cpu().pin_memory()
+        self.host_d = torch.empty((self.M, N), dtype=torch.bfloat16).pin_memory()
+
+    def calls(self, stream_ptr):
+        import ctypes
+        import moe_grouped_gemm_quantize_b200 as lnq
+        L = lnq.lib()
+        P = ctypes.c_void_p
+        c = self.cfg
+        s = P(stream_ptr)
+        qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K,
+                 P(self.sfa.data_ptr()), self.M, s)
+        gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), P(self.wq.data_ptr()),
+                 P(self.ws.data_ptr()), P(self.mm.data_ptr()), c.groups, c.m_max,
+                 c.tokens // c.groups, P(self.d.data_ptr()), c.N, c.K, s)
+        return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_m_grouped_fp8_gemm_masked, gargs)
+
+
 def workload_units(name: str):
     from moe_grouped_gemm_quantize_b200 import synthetic
     if name == "prefill":
@@ -284,6 +329,8 @@ def workload_units(name: str):
         return [synthetic.TINY], "linear"
     if name == "moe":
         return [synthetic.MOE], "grouped"
+    if name == "moe_masked":
+        return [synthetic.MOE_MASKED], "masked"
     raise ValueError(name)
 
 
@@ -293,11 +340,13 @@ WORKLOAD_DESC = {
     "moe": "M-grouped contiguous MoE: 16384 rows over 32 experts (multinomial seed 0), N=4096, K=7168",
     "square": "square 8192^3 with 5% outlier 1x128 groups (x100)",
     "tiny": "tiny 128x256x512",
+    "moe_masked": "M-grouped masked MoE: 32 expert buffers of 128 rows, 2048 routed tokens "
+                  "(multinomial seed 3), N=4096, K=7168",
 }
 
 
 def is_hbm_bound(name: str) -> bool:
-    return name == "decode"
+    return name in ("decode", "moe_masked")
 
 
 # --------------------------------------------------------------------------- our arm
@@ -319,8 +368,8 @@ def run_ours(args, world, rank, local):
     lnq.lnq_set_weight_prefetch(not args.no_weight_prefetch)
 
     cfgs, kind = workload_units(args.workload)
-    units = [Grouped(c, dev) if kind == "grouped" else Linear(c, dev, split=args.split)
-             for c in cfgs]
+    units = [Grouped(c, dev) if kind == "grouped" else Masked(c, dev) if kind == "masked"
+             else Linear(c, dev, split=args.split) for c in cfgs]
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     calls = [u.calls(sp) for u in units]
@@ -499,7 +548,13 @@ def oracle_inputs(workload: str, max_rows: int):
     cfgs, kind = workload_units(workload)
     items = []
     for c in cfgs:
-        if kind == "grouped":
+        if kind == "masked":
+            a, w, counts = synthetic.make_moe_masked_inputs(c)
+            r = min(max_rows, int(counts[0]))
+            # group 0's real rows against group 0's weights
+            wq, ws = oracle.quantize_fp8_blocks(synthetic.bf16_bits(w[:c.N]))
+            items.append((synthetic.bf16_bits(a[:r]), wq, ws, 2.0 * c.N * c.K))
+        elif kind == "grouped":
             a, w, m_indices, _ = synthetic.make_moe_inputs(c)
             r = min(max_rows, 128)
             # the first rows belong to group 0: its weights are the product's B
@@ -618,7 +673,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "decode", "moe", "square", "tiny"],
+    ap.add_argument("--workload", choices=["prefill", "decode", "moe", "moe_masked", "square", "tiny"],
                     default="prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

@@ -213,6 +213,35 @@ lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sf
                                              void* d_bf16, int64_t M_total, int64_t N, int64_t K,
                                              void* stream);
 
+/*
+ * M-grouped masked block-scaled FP8 GEMM (MoE experts fed by a token dispatch):
+ * every group has a fixed buffer of M_max rows, of which only the first
+ * masked_m[g] hold tokens; the counts stay on the device, so no host
+ * synchronization is needed (deepgemm-rust README, "What's implemented",
+ * m_grouped_fp8_gemm_nt_masked: masked_m scheduler, DeepEP-style dispatch
+ * output, expected_m scheduling, zero CPU sync).
+ *
+ *   a_e4m3      [num_groups*M_max][K] E4M3: rows g*M_max .. g*M_max + M_max - 1
+ *               are group g's buffer (a [num_groups][M_max][K] tensor).
+ *   sfa         [K/128][num_groups*M_max] fp32 MN-major over all those rows, as
+ *               lnq_quantize_fp8_groups writes for M = num_groups*M_max.
+ *   b_e4m3      [num_groups*N][K] E4M3, sfb [num_groups*ceil(N/128)][K/128] fp32:
+ *               as in lnq_m_grouped_fp8_gemm_contiguous.
+ *   masked_m    [num_groups] int32 on the device: real rows of each group,
+ *               0 .. M_max.  A count outside that range is clamped and reported
+ *               by lnq_get_last_device_error as LNQ_ERR_INVALID_ARG.
+ *   expected_m  the caller's estimate of the rows per group (>= 0); a scheduling
+ *               hint only, results do not depend on it.
+ *   d_bf16      [num_groups*M_max][N] bf16: rows g*M_max + m for m < masked_m[g]
+ *               are written; the other rows are left untouched.
+ *   Requires: M_max % 128 == 0, N % 16 == 0, K % 128 == 0, sfb and masked_m
+ *   4-byte aligned, the other pointers 16-byte aligned.
+ */
+lnq_status lnq_m_grouped_fp8_gemm_masked(const void* a_e4m3, const float* sfa, const void* b_e4m3,
+                                         const float* sfb, const int32_t* masked_m,
+                                         int32_t num_groups, int64_t M_max, int64_t expected_m,
+                                         void* d_bf16, int64_t N, int64_t K, void* stream);
+
 /* Static text for a status code. */
 const char* lnq_status_string(lnq_status status);
 

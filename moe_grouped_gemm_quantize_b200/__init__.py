@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "lnq_fp8_block_gemm_nt_ws": [P, P, I64, P, P, P, I64, I64, I64, P, I64, P],
             "lnq_fp8_block_gemm_nt_static_ws": [P, P, I64, P, P, P, I64, I64, I64, P],
             "lnq_m_grouped_fp8_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
+            "lnq_m_grouped_fp8_gemm_masked": [P, P, P, P, P, I32, I64, I64, P, I64, I64, P],
             "lnq_get_last_device_error": [P],
             "lnq_selftest_wait_timeout": [I64, P],
         }
@@ -253,6 +254,34 @@ def lnq_m_grouped_fp8_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: tor
                                                    _ptr(m_indices), G, _ptr(d), M_total, N, K,
                                                    _stream(stream)),
            "lnq_m_grouped_fp8_gemm_contiguous")
+
+
+def lnq_m_grouped_fp8_gemm_masked(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                                  masked_m: torch.Tensor, d: torch.Tensor, expected_m: int = 0,
+                                  stream=None) -> None:
+    """a e4m3 [G, M_max, K] (or [G*M_max, K]), sfa fp32 [K/128, G*M_max], b e4m3 [G*N, K] (or
+    [G, N, K]), sfb fp32 [G*ceil(N/128), K/128], masked_m int32 [G] on the device, d bf16
+    [G, M_max, N] (or [G*M_max, N]): group g's first masked_m[g] rows of d are written."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.float32 or sfb.dtype != torch.float32 or \
+            d.dtype != torch.bfloat16 or masked_m.dtype != torch.int32:
+        raise TypeError("a, b float8_e4m3fn/uint8; sfa, sfb float32; masked_m int32; d bf16")
+    G = masked_m.numel()
+    if a.dim() == 3:
+        if a.shape[0] != G:
+            raise ValueError("a's first dimension must be the number of groups")
+        M_max, K = a.shape[1], a.shape[2]
+    else:
+        M_max, K = a.shape[0] // G, a.shape[1]
+    N = (b.shape[1] if b.dim() == 3 else b.shape[0] // G)
+    for t in (a, sfa, b, sfb, masked_m, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    if a.numel() != G * M_max * K or b.numel() != G * N * K or d.numel() != G * M_max * N or \
+            tuple(sfa.shape) != (K // 128, G * M_max) or tuple(sfb.shape) != (G * -(-N // 128), K // 128):
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_m_grouped_fp8_gemm_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(masked_m), G,
+                                               M_max, expected_m, _ptr(d), N, K, _stream(stream)),
+           "lnq_m_grouped_fp8_gemm_masked")
 
 
 def lnq_get_last_device_error(stream=None) -> int:

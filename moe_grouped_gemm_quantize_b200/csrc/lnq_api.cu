@@ -524,6 +524,54 @@ lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sf
     return launch_gemm<CfgGrouped128>(*dev, a_e4m3, M_total, b_e4m3, wrows, K, args, s);
 }
 
+lnq_status lnq_m_grouped_fp8_gemm_masked(const void* a_e4m3, const float* sfa, const void* b_e4m3,
+                                         const float* sfb, const int32_t* masked_m,
+                                         int32_t num_groups, int64_t M_max, int64_t expected_m,
+                                         void* d_bf16, int64_t N, int64_t K, void* stream) {
+    if (M_max <= 0 || N <= 0 || K <= 0 || num_groups <= 0 || expected_m < 0)
+        return LNQ_ERR_INVALID_ARG;
+    const int64_t M_total = static_cast<int64_t>(num_groups) * M_max;
+    if (M_max % 128 != 0 || K % 128 != 0 || N % 16 != 0 || N < 16 || M_total > kMaxRows ||
+        K > (int64_t{1} << 31) || static_cast<int64_t>(num_groups) * N > kMaxRows)
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!a_e4m3 || !sfa || !b_e4m3 || !sfb || !masked_m || !d_bf16) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned4(sfb) ||
+        !aligned16(d_bf16) || !aligned4(masked_m))
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+
+    // The grouped kernel with the group of a 128-row block given by its position and
+    // the block's real rows by masked_m, read on the device (no host synchronization).
+    // expected_m is accepted as the callers' scheduling hint; the blocks past a
+    // group's count are skipped by the CTA that owns them.
+    GemmArgs args{};
+    args.sfa = sfa;
+    args.sfb = sfb;
+    args.d = static_cast<uint16_t*>(d_bf16);
+    args.m_indices = nullptr;
+    args.masked_m = masked_m;
+    args.m_max = static_cast<int>(M_max);
+    args.M4 = M_total;
+    args.M = static_cast<int>(M_total);
+    args.N = static_cast<int>(N);
+    args.num_kb = static_cast<int>(K / 128);
+    args.nb = static_cast<int>((N + 127) / 128);
+    args.num_groups = num_groups;
+    args.tiles_p = static_cast<int>(M_total / 128);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t wrows = static_cast<int64_t>(num_groups) * N;
+    if (N >= 256) {
+        args.tiles_q = static_cast<int>((N + 255) / 256);
+        args.num_tiles = args.tiles_p * args.tiles_q;
+        return launch_gemm<CfgGrouped256>(*dev, a_e4m3, M_total, b_e4m3, wrows, K, args, s);
+    }
+    args.tiles_q = static_cast<int>((N + 127) / 128);
+    args.num_tiles = args.tiles_p * args.tiles_q;
+    return launch_gemm<CfgGrouped128>(*dev, a_e4m3, M_total, b_e4m3, wrows, K, args, s);
+}
+
 lnq_status lnq_get_last_device_error(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LNQ_ERR_CUDA;

@@ -66,6 +66,10 @@ struct GemmArgs {
     float* partials;  // [num_tiles][max_slots][128][BNQ]
     int* counters;    // [num_tiles], zero before and after every launch
     int max_slots;    // most CTAs sharing one tile
+    // Grouped, masked layout only (m_indices == nullptr): group g owns rows
+    // g*m_max .. g*m_max + m_max - 1, of which the first masked_m[g] are real.
+    const int32_t* masked_m;  // [num_groups], on the device
+    int m_max;                // rows per group, a multiple of 128
 };
 
 constexpr unsigned int kStatusBadGroup = 2u;
@@ -185,9 +189,10 @@ __device__ __forceinline__ int unit_owner(long long x, long long U, int units) {
 }
 
 struct TileCoord {
-    int p0;     // first row of this CTA's P operand (activation row, or weight row for SWAP)
-    int q0;     // first output column of the tile (weight row within the group, or token)
-    int group;  // grouped: group id of the tile, -1 skip; else 0
+    int p0;       // first row of this CTA's P operand (activation row, or weight row for SWAP)
+    int q0;       // first output column of the tile (weight row within the group, or token)
+    int group;    // grouped: group id of the tile, -1 skip; else 0
+    int row_end;  // output rows from row_end on are not stored (dense and grouped tiles)
 };
 
 // Tile t of this CTA (or of this CTA pair; `rank` is the CTA's rank in the pair).
@@ -198,6 +203,7 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32
         c.p0 = (t % a.tiles_p) * C::kP;
         c.q0 = (t / a.tiles_p) * C::BNQ;
         c.group = 0;
+        c.row_end = a.M;
     } else {
         // Bands of row tiles, column-major inside a band: a wave of tiles shares a
         // band of activation rows and a few weight column tiles.  Grouped: the
@@ -212,11 +218,27 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32
         const int r = t - band * band_tiles;
         c.p0 = (first + r % rows) * C::kTileM + static_cast<int>(rank) * C::kP;
         c.q0 = (r / rows) * C::BNQ;
+        c.row_end = a.M;
         if constexpr (C::GROUPED) {
-            c.group = __ldg(a.m_indices + c.p0);
-            if (c.group >= a.num_groups) {
-                atomicOr(a.status, kStatusBadGroup);
-                c.group = -1;
+            if (a.m_indices != nullptr) {
+                // contiguous: the block's group is that of its first row
+                c.group = __ldg(a.m_indices + c.p0);
+                if (c.group >= a.num_groups) {
+                    atomicOr(a.status, kStatusBadGroup);
+                    c.group = -1;
+                }
+            } else {
+                // masked: group g's first masked_m[g] rows are real; a block past
+                // them is skipped, a block that holds the last of them stops there
+                const int g = c.p0 / a.m_max;
+                int count = __ldg(a.masked_m + g);
+                if (count < 0 || count > a.m_max) {
+                    atomicOr(a.status, kStatusBadGroup);
+                    count = count < 0 ? 0 : a.m_max;
+                }
+                const int valid = g * a.m_max + count - c.p0;
+                c.group = valid > 0 ? g : -1;
+                c.row_end = c.p0 + (valid < C::kP ? valid : C::kP);
             }
         } else {
             c.group = 0;
@@ -796,7 +818,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             // ---- store the tile
             if constexpr (!C::SWAP) {
                 const int m = tc.p0 + row;
-                if (m < args.M) {
+                if (m < tc.row_end) {
                     uint16_t* drow = args.d + static_cast<long long>(m) * args.N;
 #pragma unroll
                     for (int c = 0; c < C::kCW / 8; ++c) {

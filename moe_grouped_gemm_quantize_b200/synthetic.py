@@ -127,6 +127,35 @@ class MoE:
         return 2.0 * self.total_rows * self.N * self.K
 
 
+@dataclass(frozen=True)
+class MoEMasked:
+    """Decode-time MoE after a token dispatch: every expert has a buffer of m_max rows,
+    of which the first count[g] hold tokens (multinomial over the experts, capped)."""
+    name: str = "moe_masked_32x128_n4096_k7168"
+    tokens: int = 2048
+    groups: int = 32
+    m_max: int = 128
+    N: int = 4096
+    K: int = 7168
+    a_std: float = 1.0
+    w_std: float = 0.02
+    counts_seed: int = 3
+    a_seed: int = 70
+    w_seed: int = 71
+
+    def counts(self) -> np.ndarray:
+        c = np.random.default_rng(self.counts_seed).multinomial(self.tokens, [1.0 / self.groups] * self.groups)
+        return np.minimum(c, self.m_max).astype(np.int32)
+
+    @property
+    def real_rows(self) -> int:
+        return int(self.counts().sum())
+
+    @property
+    def flops(self) -> float:
+        return 2.0 * self.real_rows * self.N * self.K
+
+
 TINY = Linear("tiny_128x256x512", 128, 256, 512)
 PREFILL = (
     Linear("prefill_qkv_2048x6144x4096", 2048, 6144, 4096, a_seed=10, w_seed=11),
@@ -137,6 +166,7 @@ PREFILL = (
 DECODE = tuple(Linear(f"decode_m{m}_12288x4096", m, 12288, 4096, a_seed=50 + m, w_seed=49)
                for m in (1, 8, 32, 64))
 MOE = MoE()
+MOE_MASKED = MoEMasked()
 SQUARE = Linear("square_8192", 8192, 8192, 8192, a_std=1.0, w_std=1.0, a_seed=60, w_seed=61,
                 outliers=True, a_outlier_seed=1, w_outlier_seed=2)
 
@@ -163,3 +193,10 @@ def make_moe_inputs(cfg: MoE = MOE, device="cpu"):
     a = a.masked_fill(pad.unsqueeze(1), 0.0)
     w = gaussian_bf16((cfg.groups * cfg.N, cfg.K), cfg.w_std, cfg.w_seed, device)
     return a, w, m_indices, sizes
+
+
+def make_moe_masked_inputs(cfg: MoEMasked = MOE_MASKED, device="cpu"):
+    """(A bf16 [G*m_max, K] with random rows past each count, W bf16 [G*N, K], counts)."""
+    a = gaussian_bf16((cfg.groups * cfg.m_max, cfg.K), cfg.a_std, cfg.a_seed, device)
+    w = gaussian_bf16((cfg.groups * cfg.N, cfg.K), cfg.w_std, cfg.w_seed, device)
+    return a, w, cfg.counts()

@@ -117,6 +117,22 @@ def test_grouped_argument_errors(L):
     assert call(a=A16 + 1) == MISALIGNED
 
 
+def test_masked_argument_errors(L):
+    f = L.lnq_m_grouped_fp8_gemm_masked
+
+    def call(M_max=256, N=256, K=512, G=4, mm=A16e + 0x1000, a=A16, expected=64):
+        return f(a, A16b, A16c, A16d, mm, G, M_max, expected, A16e, N, K, None)
+
+    assert call(G=0) == INVALID
+    assert call(expected=-1) == INVALID
+    assert call(M_max=200) == SHAPE            # M_max % 128
+    assert call(K=100) == SHAPE
+    assert call(N=20) == SHAPE
+    assert call(mm=None) == INVALID
+    assert call(mm=A16e + 0x1002) == MISALIGNED
+    assert call(a=A16 + 1) == MISALIGNED
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU failure path")
 def test_valid_arguments_without_gpu_fail_loudly(L):
     rc = L.lnq_fp8_block_gemm_nt(A16, A16b, 8, A16c, A16d, A16e, 8, 256, 512, None)
