@@ -189,7 +189,7 @@ class ClockSampler:
 class Linear:
     """One dense linear: bf16 activations resident on the device, weights pre-quantized."""
 
-    def __init__(self, cfg, dev, split: bool = False):
+    def __init__(self, cfg, dev, split: bool = False, fp8_out: bool = False):
         import moe_grouped_gemm_quantize_b200 as lnq
         from moe_grouped_gemm_quantize_b200 import synthetic
         self.cfg = cfg
@@ -212,6 +212,23 @@ class Linear:
         self.host_d = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
         # decode shapes: a workspace lets every SM share the weight stream (K split)
         self.work = lnq.gemm_workspace(M, N, K, dev) if split else None
+        # fused epilogue: the output quantized (E4M3 + 1x128 scales) for a next linear
+        self.fp8_out = fp8_out and M > 64 and N % 128 == 0 and N >= 256
+        if self.fp8_out:
+            self.qo = torch.empty((M, N), dtype=torch.float8_e4m3fn, device=dev)
+            self.so = torch.empty((N // 128, self.M4), dtype=torch.float32, device=dev)
+            self.gemm_bytes += -2 * M * N + M * N + 4 * (N // 128) * self.M4
+            self.d2h_bytes = M * N + 4 * (N // 128) * self.M4
+            self.host_qo = torch.empty((M, N), dtype=torch.uint8).pin_memory()
+            self.host_so = torch.empty((N // 128, self.M4), dtype=torch.float32).pin_memory()
+
+    def copy_out(self):
+        """The step's result to pinned host memory (asynchronous)."""
+        if self.fp8_out:
+            self.host_qo.copy_(self.qo.view(torch.uint8), non_blocking=True)
+            self.host_so.copy_(self.so, non_blocking=True)
+        else:
+            self.host_d.copy_(self.d, non_blocking=True)
 
     def calls(self, stream_ptr):
         """Pre-marshalled C-ABI calls (quantize, gemm)."""
@@ -225,6 +242,11 @@ class Linear:
                  P(self.sfa.data_ptr()), self.M4, s)
         gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), self.M4, P(self.wq.data_ptr()),
                  P(self.ws.data_ptr()), P(self.d.data_ptr()), c.M, c.N, c.K)
+        if self.fp8_out:
+            eargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), self.M4, P(self.wq.data_ptr()),
+                     P(self.ws.data_ptr()), P(0), P(0), P(self.qo.data_ptr()), P(self.so.data_ptr()),
+                     self.M4, c.M, c.N, c.K, s)
+            return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_fp8_block_gemm_nt_epilogue, eargs)
         if self.work is not None:
             return (L.lnq_quantize_fp8_groups, qargs), \
                 (L.lnq_fp8_block_gemm_nt_ws, gargs + (P(self.work.data_ptr()), self.work.numel(), s))
@@ -256,6 +278,9 @@ class Grouped:
         self.d2h_bytes = 2 * self.M * N
         self.host_x = self.x.cpu().pin_memory()
         self.host_d = torch.empty((self.M, N), dtype=torch.bfloat16).pin_memory()
+
+    def copy_out(self):
+        self.host_d.copy_(self.d, non_blocking=True)
 
     def calls(self, stream_ptr):
         import ctypes
@@ -301,6 +326,9 @@ class Masked:
         self.d2h_bytes = 2 * self.M * N
         self.host_x = self.x.cpu().pin_memory()
         self.host_d = torch.empty((self.M, N), dtype=torch.bfloat16).pin_memory()
+
+    def copy_out(self):
+        self.host_d.copy_(self.d, non_blocking=True)
 
     def calls(self, stream_ptr):
         import ctypes
@@ -369,7 +397,7 @@ def run_ours(args, world, rank, local):
 
     cfgs, kind = workload_units(args.workload)
     units = [Grouped(c, dev) if kind == "grouped" else Masked(c, dev) if kind == "masked"
-             else Linear(c, dev, split=args.split) for c in cfgs]
+             else Linear(c, dev, split=args.split, fp8_out=args.epilogue == "fp8") for c in cfgs]
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     calls = [u.calls(sp) for u in units]
@@ -439,7 +467,7 @@ def run_ours(args, world, rank, local):
         Ke = max(1, min(K, args.e2e_steps))
         for u in units:                       # warm the copy paths
             u.x.copy_(u.host_x, non_blocking=True)
-            u.host_d.copy_(u.d, non_blocking=True)
+            u.copy_out()
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -452,7 +480,7 @@ def run_ours(args, world, rank, local):
                 rc = qf(*qa) or gf(*ga)
                 if rc:
                     raise lnq.LnqError(rc, "e2e")
-                u.host_d.copy_(u.d, non_blocking=True)
+                u.copy_out()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(dist)
@@ -514,6 +542,8 @@ def run_ours(args, world, rank, local):
                    "weight_prefetch": not args.no_weight_prefetch,
                    "decode_k_split": args.split and any(getattr(u, "work", None) is not None
                                                          for u in units),
+                   "epilogue": "fp8 output (E4M3 + 1x128 scales)" if any(getattr(u, "fp8_out", False)
+                                                                         for u in units) else "bf16 output",
                    "parallelism": f"replicas x{world} (independent tokens per rank)",
                    "l2": "working set per step > 126 MB L2; no extra flush"},
         "roofline": roof,
@@ -679,6 +709,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--epilogue", choices=["bf16", "fp8"], default="bf16",
+                    help="dense GEMM output: bf16 D, or E4M3 codes + 1x128 scales for a next linear")
     ap.add_argument("--split", action="store_true",
                     help="decode GEMMs through the workspace K split (slower than whole weight tiles "
                          "per CTA at N = 12288 on B200)")

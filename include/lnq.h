@@ -121,6 +121,31 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
                                  int64_t N, int64_t K, void* stream);
 
 /*
+ * lnq_fp8_block_gemm_nt with a fused epilogue: an optional bias, and the output
+ * either in bf16 or already quantized for a next linear (deepgemm-rust README,
+ * "Key techniques": fused epilogues; Linnet plugin, _BlockProduct.execute adds
+ * the bias after the product).
+ *
+ *   bias_bf16  [N] bf16 or NULL (16-byte aligned): added to every row in FP32
+ *              before the output rounding.
+ *   d_bf16     [M][N] bf16 output, or NULL when q_e4m3 is given.
+ *   q_e4m3     [M][N] E4M3 output, or NULL: the result is rounded to bf16 (the
+ *              values d_bf16 would hold) and quantized per row in 1 x 128 groups
+ *              exactly as lnq_quantize_fp8_groups quantizes a bf16 input.
+ *   sfa_out    [N/128][M4_out] fp32 scales of q_e4m3 (MN-major; rows M ..
+ *              M4_out-1 get 0.0f), as lnq_quantize_fp8_groups writes them.
+ *   M4_out     >= ceil4(M), a multiple of 4.
+ *   Exactly one of d_bf16 and q_e4m3 is given.  The quantized output needs
+ *   M > 64, N >= 256 and N % 128 == 0 (LNQ_ERR_UNSUPPORTED_SHAPE otherwise);
+ *   q_e4m3 and sfa_out 16-byte aligned.  Other arguments as
+ *   lnq_fp8_block_gemm_nt.
+ */
+lnq_status lnq_fp8_block_gemm_nt_epilogue(const void* a_e4m3, const float* sfa, int64_t M4,
+                                          const void* b_e4m3, const float* sfb, const void* bias_bf16,
+                                          void* d_bf16, void* q_e4m3, float* sfa_out, int64_t M4_out,
+                                          int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
  * Bytes of workspace that lnq_fp8_block_gemm_nt_ws needs to split the K range of
  * a decode product (M <= 64) over `num_sms` CTAs, or 0 when the product does not
  * split (M > 64, K == 128, or at least one weight tile per SM already).  A pure

@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "lnq_quantize_fp8_blocks": [P, I64, I64, P, P, P],
             "lnq_fp8_block_gemm_nt": [P, P, I64, P, P, P, I64, I64, I64, P],
             "lnq_fp8_block_gemm_nt_ws": [P, P, I64, P, P, P, I64, I64, I64, P, I64, P],
+            "lnq_fp8_block_gemm_nt_epilogue": [P, P, I64, P, P, P, P, P, P, I64, I64, I64, I64, P],
             "lnq_fp8_block_gemm_nt_static_ws": [P, P, I64, P, P, P, I64, I64, I64, P],
             "lnq_m_grouped_fp8_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
             "lnq_m_grouped_fp8_gemm_masked": [P, P, P, P, P, I32, I64, I64, P, I64, I64, P],
@@ -169,6 +170,40 @@ def lnq_fp8_block_gemm_nt(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, s
         raise ValueError("inconsistent shapes")
     _check(lib().lnq_fp8_block_gemm_nt(_ptr(a), _ptr(sfa), sfa.shape[1], _ptr(b), _ptr(sfb), _ptr(d),
                                        M, N, K, _stream(stream)), "lnq_fp8_block_gemm_nt")
+
+
+def lnq_fp8_block_gemm_nt_epilogue(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                                   bias: torch.Tensor | None = None, d: torch.Tensor | None = None,
+                                   q: torch.Tensor | None = None, sfa_out: torch.Tensor | None = None,
+                                   stream=None) -> None:
+    """The GEMM with a fused epilogue: bias (bf16 [N] or None) added in FP32, and either d
+    (bf16 [M, N]) or q (E4M3 [M, N]) with sfa_out (fp32 [N/128, M4_out]) written."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.float32 or sfb.dtype != torch.float32:
+        raise TypeError("a, b float8_e4m3fn/uint8; sfa, sfb float32")
+    if (d is None) == (q is None):
+        raise ValueError("give exactly one of d and q")
+    if d is not None and d.dtype != torch.bfloat16:
+        raise TypeError("d bf16")
+    if q is not None and (not _is_fp8(q) or sfa_out is None or sfa_out.dtype != torch.float32):
+        raise TypeError("q float8_e4m3fn/uint8 with sfa_out float32")
+    if bias is not None and bias.dtype != torch.bfloat16:
+        raise TypeError("bias bf16")
+    M, K = a.shape
+    N = b.shape[0]
+    for t in (a, sfa, b, sfb, bias, d, q, sfa_out):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    out = d if d is not None else q
+    if b.shape[1] != K or tuple(out.shape) != (M, N) or sfa.shape[0] != K // 128 or \
+            tuple(sfb.shape) != (-(-N // 128), K // 128) or (bias is not None and bias.numel() != N) or \
+            (sfa_out is not None and sfa_out.shape[0] != N // 128):
+        raise ValueError("inconsistent shapes")
+    nul = ctypes.c_void_p(0)
+    _check(lib().lnq_fp8_block_gemm_nt_epilogue(
+        _ptr(a), _ptr(sfa), sfa.shape[1], _ptr(b), _ptr(sfb), _ptr(bias) if bias is not None else nul,
+        _ptr(d) if d is not None else nul, _ptr(q) if q is not None else nul,
+        _ptr(sfa_out) if sfa_out is not None else nul, sfa_out.shape[1] if sfa_out is not None else 0,
+        M, N, K, _stream(stream)), "lnq_fp8_block_gemm_nt_epilogue")
 
 
 def lnq_fp8_block_gemm_nt_workspace_bytes(M: int, N: int, K: int, num_sms: int) -> int:

@@ -356,18 +356,37 @@ SplitPlan plan_split(int64_t M, int64_t N, int64_t K, int64_t num_sms) {
     return plan;
 }
 
+// Output side of a dense product: bf16 D, or (fused) the E4M3 codes and 1 x 128
+// scales of the bf16-rounded result; an optional bf16 bias per column.
+struct Epilogue {
+    const void* bias = nullptr;
+    void* q_out = nullptr;
+    float* sfa_out = nullptr;
+    int64_t M4_out = 0;
+};
+
 lnq_status gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4, const void* b_e4m3,
                    const float* sfb, void* d_bf16, int64_t M, int64_t N, int64_t K,
-                   void* workspace, int64_t workspace_bytes, void* stream) {
+                   void* workspace, int64_t workspace_bytes, void* stream,
+                   const Epilogue& ep = Epilogue()) {
     if (M <= 0 || N <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
     if (K % 128 != 0 || N % 16 != 0 || N < 16 || M > kMaxRows || N > kMaxRows ||
         K > (int64_t{1} << 31))
         return LNQ_ERR_UNSUPPORTED_SHAPE;
     if (M4 < ((M + 3) / 4) * 4 || M4 % 4 != 0) return LNQ_ERR_UNSUPPORTED_SHAPE;
-    if (!a_e4m3 || !sfa || !b_e4m3 || !sfb || !d_bf16) return LNQ_ERR_INVALID_ARG;
+    const bool fp8_out = ep.q_out != nullptr;
+    if (!a_e4m3 || !sfa || !b_e4m3 || !sfb || (fp8_out ? (d_bf16 != nullptr) : (d_bf16 == nullptr)))
+        return LNQ_ERR_INVALID_ARG;
     if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned4(sfb) ||
-        !aligned16(d_bf16))
+        (d_bf16 && !aligned16(d_bf16)) || (ep.bias && !aligned16(ep.bias)))
         return LNQ_ERR_MISALIGNED;
+    if (fp8_out) {
+        // each epilogue thread must hold one whole 1 x 128 group: dense 128 x 256 tiles
+        if (M <= 64 || N % 128 != 0 || N < 256) return LNQ_ERR_UNSUPPORTED_SHAPE;
+        if (!ep.sfa_out) return LNQ_ERR_INVALID_ARG;
+        if (ep.M4_out < ((M + 3) / 4) * 4 || ep.M4_out % 4 != 0) return LNQ_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned16(ep.q_out) || !aligned16(ep.sfa_out)) return LNQ_ERR_MISALIGNED;
+    }
     DeviceInfo* dev = nullptr;
     lnq_status st = device_info(&dev);
     if (st != LNQ_OK) return st;
@@ -376,6 +395,10 @@ lnq_status gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4, const void*
     args.sfa = sfa;
     args.sfb = sfb;
     args.d = static_cast<uint16_t*>(d_bf16);
+    args.bias = static_cast<const uint16_t*>(ep.bias);
+    args.q_out = static_cast<uint8_t*>(ep.q_out);
+    args.sfa_out = ep.sfa_out;
+    args.M4_out = ep.M4_out;
     args.M4 = M4;
     args.M = static_cast<int>(M);
     args.N = static_cast<int>(N);
@@ -412,7 +435,8 @@ lnq_status gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4, const void*
         args.num_tiles = args.tiles_p * args.tiles_q;
         return launch_gemm<CfgSwap64>(*dev, a_e4m3, M, b_e4m3, N, K, args, s);
     }
-    const int pairs = g_dense_pairs.load(std::memory_order_relaxed);
+    int pairs = g_dense_pairs.load(std::memory_order_relaxed);
+    if (fp8_out && pairs == 2) pairs = 1;  // 256 x 128 pair tiles split a thread's 128-column group
     if (N >= 256 && M > 128 && pairs == 1) {
         // pairs of CTAs on 256 x 256 tiles
         args.tiles_p = static_cast<int>((M + 255) / 256);
@@ -448,6 +472,18 @@ lnq_status lnq_fp8_block_gemm_nt(const void* a_e4m3, const float* sfa, int64_t M
 
 int64_t lnq_fp8_block_gemm_nt_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t num_sms) {
     return plan_split(M, N, K, num_sms).need_bytes;
+}
+
+lnq_status lnq_fp8_block_gemm_nt_epilogue(const void* a_e4m3, const float* sfa, int64_t M4,
+                                          const void* b_e4m3, const float* sfb, const void* bias_bf16,
+                                          void* d_bf16, void* q_e4m3, float* sfa_out, int64_t M4_out,
+                                          int64_t M, int64_t N, int64_t K, void* stream) {
+    Epilogue ep;
+    ep.bias = bias_bf16;
+    ep.q_out = q_e4m3;
+    ep.sfa_out = sfa_out;
+    ep.M4_out = M4_out;
+    return gemm_nt(a_e4m3, sfa, M4, b_e4m3, sfb, d_bf16, M, N, K, nullptr, 0, stream, ep);
 }
 
 lnq_status lnq_fp8_block_gemm_nt_ws(const void* a_e4m3, const float* sfa, int64_t M4,

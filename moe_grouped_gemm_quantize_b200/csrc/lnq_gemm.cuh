@@ -40,6 +40,7 @@
 #include <cuda.h>
 
 #include "lnq_ptx.cuh"
+#include "lnq_quantize.cuh"
 
 namespace lnq {
 
@@ -70,6 +71,14 @@ struct GemmArgs {
     // g*m_max .. g*m_max + m_max - 1, of which the first masked_m[g] are real.
     const int32_t* masked_m;  // [num_groups], on the device
     int m_max;                // rows per group, a multiple of 128
+    // Fused epilogue (dense and decode tiles): an optional bf16 bias per output
+    // column added in FP32; and, instead of the bf16 D, the output quantized for a
+    // next linear (dense 128 x 256 tiles only): E4M3 codes [M][N] and FP32 scales
+    // [N/128][M4_out] of each 1 x 128 group of the bf16-rounded result.
+    const uint16_t* bias;  // [N] bf16 bits, or nullptr
+    uint8_t* q_out;        // [M][N] E4M3, or nullptr (bf16 D)
+    float* sfa_out;        // [N/128][M4_out]
+    long long M4_out;
 };
 
 constexpr unsigned int kStatusBadGroup = 2u;
@@ -311,10 +320,11 @@ __device__ __forceinline__ void store_decode_tile(const GemmArgs& args, const Ti
                                                   const float2 (&acc)[C::kCW / 2]) {
     const int n = tc.p0 + row;
     if (n >= args.N) return;
+    const float bias = args.bias != nullptr ? bf16_lo(static_cast<uint32_t>(args.bias[n])) : 0.f;
 #pragma unroll
     for (int j = 0; j < C::kCW; ++j) {
         const int m = tc.q0 + j;
-        const float v = (j & 1) ? acc[j >> 1].y : acc[j >> 1].x;
+        const float v = ((j & 1) ? acc[j >> 1].y : acc[j >> 1].x) + bias;
         if (m < args.M)
             args.d[static_cast<long long>(m) * args.N + n] =
                 static_cast<uint16_t>(pack_bf16x2(v, 0.f) & 0xFFFFu);
@@ -818,11 +828,56 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             // ---- store the tile
             if constexpr (!C::SWAP) {
                 const int m = tc.p0 + row;
-                if (m < tc.row_end) {
+                const int n0 = tc.q0 + wg * C::kCW;
+                if (args.bias != nullptr) {
+#pragma unroll
+                    for (int c = 0; c < C::kCW / 8; ++c) {
+                        if (n0 + c * 8 < args.N) {
+                            const uint4 b = *reinterpret_cast<const uint4*>(args.bias + n0 + c * 8);
+                            acc[c * 4 + 0] = __fadd2_rn(acc[c * 4 + 0], make_float2(bf16_lo(b.x), bf16_hi(b.x)));
+                            acc[c * 4 + 1] = __fadd2_rn(acc[c * 4 + 1], make_float2(bf16_lo(b.y), bf16_hi(b.y)));
+                            acc[c * 4 + 2] = __fadd2_rn(acc[c * 4 + 2], make_float2(bf16_lo(b.z), bf16_hi(b.z)));
+                            acc[c * 4 + 3] = __fadd2_rn(acc[c * 4 + 3], make_float2(bf16_lo(b.w), bf16_hi(b.w)));
+                        }
+                    }
+                }
+                if (args.q_out != nullptr) {
+                    if constexpr (C::kCW == 128) {
+                        // this thread's 128 columns are one 1 x 128 group of row m: round
+                        // to bf16 as the D store would, then quantize exactly as the
+                        // activation quantize kernel does
+                        if (n0 < args.N && m < tc.row_end) {
+                            uint32_t h[64];
+#pragma unroll
+                            for (int i = 0; i < 64; ++i) h[i] = pack_bf16x2(acc[i].x, acc[i].y);
+                            float amax = 0.f;
+#pragma unroll
+                            for (int i = 0; i < 64; ++i)
+                                amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(h[i])), fabsf(bf16_hi(h[i]))));
+                            const float sv = scale_of_amax(amax);
+                            const float rv = rcp_approx(sv);
+                            uint8_t* qrow = args.q_out + static_cast<long long>(m) * args.N + n0;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                float t0[8], t1[8];
+                                const uint4 r0 = make_uint4(h[8 * j + 0], h[8 * j + 1], h[8 * j + 2], h[8 * j + 3]);
+                                const uint4 r1 = make_uint4(h[8 * j + 4], h[8 * j + 5], h[8 * j + 6], h[8 * j + 7]);
+                                quotients8(r0, sv, rv, sv == 0.0f, !(sv >= 0x1p-125f), t0);
+                                quotients8(r1, sv, rv, sv == 0.0f, !(sv >= 0x1p-125f), t1);
+                                const uint2 p0 = pack8(t0), p1 = pack8(t1);
+                                *reinterpret_cast<uint4*>(qrow + 16 * j) = make_uint4(p0.x, p0.y, p1.x, p1.y);
+                            }
+                            args.sfa_out[static_cast<long long>(n0 >> 7) * args.M4_out + m] = sv;
+                        } else if (n0 < args.N && m >= args.M && m < args.M4_out) {
+                            // rows past M up to the padded scale count carry a zero scale
+                            args.sfa_out[static_cast<long long>(n0 >> 7) * args.M4_out + m] = 0.f;
+                        }
+                    }
+                } else if (m < tc.row_end) {
                     uint16_t* drow = args.d + static_cast<long long>(m) * args.N;
 #pragma unroll
                     for (int c = 0; c < C::kCW / 8; ++c) {
-                        const int n = tc.q0 + wg * C::kCW + c * 8;
+                        const int n = n0 + c * 8;
                         if (n < args.N) {
                             uint4 w;
                             w.x = pack_bf16x2(acc[c * 4 + 0].x, acc[c * 4 + 0].y);

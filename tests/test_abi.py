@@ -133,6 +133,23 @@ def test_masked_argument_errors(L):
     assert call(a=A16 + 1) == MISALIGNED
 
 
+def test_epilogue_argument_errors(L):
+    f = L.lnq_fp8_block_gemm_nt_epilogue
+
+    def call(M=256, N=256, K=512, bias=None, d=A16e, q=None, so=None, M4o=256):
+        return f(A16, A16b, ((M + 3) // 4) * 4, A16c, A16d, bias, d, q, so, M4o, M, N, K, None)
+
+    assert call(d=None) == INVALID                         # no output
+    assert call(q=A16e + 0x2000, so=A16e + 0x4000) == INVALID      # both outputs
+    assert call(d=None, q=A16e + 0x2000) == INVALID         # codes without scales
+    assert call(M=8, d=None, q=A16e + 0x2000, so=A16e + 0x4000, M4o=8) == SHAPE     # decode tiles
+    assert call(N=320, d=None, q=A16e + 0x2000, so=A16e + 0x4000) == SHAPE          # N % 128
+    assert call(N=128, d=None, q=A16e + 0x2000, so=A16e + 0x4000) == SHAPE          # N < 256
+    assert call(d=None, q=A16e + 0x2000, so=A16e + 0x4000, M4o=252) == SHAPE       # M4_out < ceil4(M)
+    assert call(bias=A16e + 0x2002) == MISALIGNED
+    assert call(d=None, q=A16e + 0x2001, so=A16e + 0x4000) == MISALIGNED
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU failure path")
 def test_valid_arguments_without_gpu_fail_loudly(L):
     rc = L.lnq_fp8_block_gemm_nt(A16, A16b, 8, A16c, A16d, A16e, 8, 256, 512, None)
