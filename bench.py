@@ -2,13 +2,15 @@
 """Benchmark of the block-scaled FP8 linear on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill|decode|moe|square|tiny]
+                    [--workload prefill|decode|moe|moe_psum|moe_masked|square|tiny]
 
 One step is one pass of the hot path over one batch of synthetic input: for each
 linear of the workload, the 1x128 activation quantize (lnq_quantize_fp8_groups)
 and the block-scaled FP8 GEMM (lnq_fp8_block_gemm_nt, or the M-grouped
-contiguous GEMM for `moe`).  Weights are model parameters: quantized to
-128x128 blocks once, before timing (lnq_quantize_fp8_blocks).
+contiguous GEMM for `moe` (per-row group ids) and `moe_psum` (prefix sums, groups
+aligned to 256 rows), or the masked one for `moe_masked`).  Weights are model
+parameters: quantized to 128x128 blocks once, before timing
+(lnq_quantize_fp8_blocks).
 
 Default workload (`prefill`): the dense-transformer prefill linears at M = 2048
 tokens, K = 4096 -- QKV N=6144, O N=4096, gate_up N=24576, down K=12288 -> N=4096.
@@ -254,25 +256,32 @@ class Linear:
 
 
 class Grouped:
-    """The M-grouped contiguous MoE GEMM: 16384 routed rows over 32 experts."""
+    """The M-grouped contiguous MoE GEMM: 16384 routed rows over 32 experts, described
+    by per-row group ids (128-row alignment) or, with `alignment` set, by the prefix
+    sums of the group sizes (group starts aligned to that many rows)."""
 
-    def __init__(self, cfg, dev):
+    def __init__(self, cfg, dev, alignment=None):
         import moe_grouped_gemm_quantize_b200 as lnq
         from moe_grouped_gemm_quantize_b200 import synthetic
         self.cfg = cfg
-        a, w, m_indices, sizes = synthetic.make_moe_inputs(cfg)
+        self.alignment = alignment
+        a, w, m_indices, sizes = synthetic.make_moe_inputs(cfg, alignment=alignment or 128)
         self.M = a.shape[0]
         self.x = a.to(dev)
         self.wq, self.ws = lnq.quantize_weights_grouped(w.to(dev), cfg.groups)
         del w
-        self.mi = torch.from_numpy(m_indices).to(dev)
+        if alignment is None:
+            self.mi = torch.from_numpy(m_indices).to(dev)
+        else:
+            self.mi = torch.from_numpy(synthetic.psum_layout(sizes, alignment)[0]).to(dev)
         K, N, G = cfg.K, cfg.N, cfg.groups
         self.q = torch.empty((self.M, K), dtype=torch.float8_e4m3fn, device=dev)
         self.sfa = torch.empty((K // 128, self.M), dtype=torch.float32, device=dev)
         self.d = torch.empty((self.M, N), dtype=torch.bfloat16, device=dev)
         self.flops = cfg.flops   # real rows only
         self.gemm_bytes = (self.M * K + 4 * (K // 128) * self.M + G * N * K
-                           + 4 * G * (-(-N // 128)) * (K // 128) + 2 * self.M * N + 4 * self.M)
+                           + 4 * G * (-(-N // 128)) * (K // 128) + 2 * self.M * N
+                           + 4 * (self.M if alignment is None else G))
         self.quant_bytes = 3 * self.M * K + 4 * (K // 128) * self.M
         self.h2d_bytes = 2 * self.M * K
         self.d2h_bytes = 2 * self.M * N
@@ -291,6 +300,11 @@ class Grouped:
         s = P(stream_ptr)
         qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K,
                  P(self.sfa.data_ptr()), self.M, s)
+        if self.alignment is not None:
+            gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), P(self.wq.data_ptr()),
+                     P(self.ws.data_ptr()), P(self.mi.data_ptr()), c.groups, self.alignment,
+                     P(self.d.data_ptr()), self.M, c.N, c.K, s)
+            return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_m_grouped_fp8_gemm_contiguous_psum, gargs)
         gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), P(self.wq.data_ptr()),
                  P(self.ws.data_ptr()), P(self.mi.data_ptr()), c.groups, P(self.d.data_ptr()),
                  self.M, c.N, c.K, s)
@@ -359,6 +373,8 @@ def workload_units(name: str):
         return [synthetic.MOE], "grouped"
     if name == "moe_masked":
         return [synthetic.MOE_MASKED], "masked"
+    if name == "moe_psum":
+        return [synthetic.MOE], "psum"
     raise ValueError(name)
 
 
@@ -368,6 +384,9 @@ WORKLOAD_DESC = {
     "moe": "M-grouped contiguous MoE: 16384 rows over 32 experts (multinomial seed 0), N=4096, K=7168",
     "square": "square 8192^3 with 5% outlier 1x128 groups (x100)",
     "tiny": "tiny 128x256x512",
+    "moe_psum": "M-grouped contiguous MoE, prefix-sum layout with 256-row group alignment "
+                "(256x256 tiles on CTA pairs): 16384 rows over 32 experts (multinomial seed 0), "
+                "N=4096, K=7168",
     "moe_masked": "M-grouped masked MoE: 32 expert buffers of 128 rows, 2048 routed tokens "
                   "(multinomial seed 3), N=4096, K=7168",
 }
@@ -391,12 +410,14 @@ def run_ours(args, world, rank, local):
     barrier(dist)
     lnq.lib()
     lnq.lib().lnq_set_dense_cta_pairs(args.cta_pairs)
+    lnq.lib().lnq_set_grouped_cta_pairs(args.grouped_cta_pairs)
     # the weights are model parameters quantized before timing: nothing in the step
     # writes them, so the GEMMs may stream them before the previous kernel completes
     lnq.lnq_set_weight_prefetch(not args.no_weight_prefetch)
 
     cfgs, kind = workload_units(args.workload)
-    units = [Grouped(c, dev) if kind == "grouped" else Masked(c, dev) if kind == "masked"
+    units = [Grouped(c, dev) if kind == "grouped" else Grouped(c, dev, alignment=256) if kind == "psum"
+             else Masked(c, dev) if kind == "masked"
              else Linear(c, dev, split=args.split, fp8_out=args.epilogue == "fp8") for c in cfgs]
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
@@ -539,6 +560,7 @@ def run_ours(args, world, rank, local):
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, bf16)",
         "config": {"workload": args.workload, "desc": WORKLOAD_DESC[args.workload],
                    "dense_cta_pairs": args.cta_pairs,
+                   "grouped_cta_pairs": args.grouped_cta_pairs,
                    "weight_prefetch": not args.no_weight_prefetch,
                    "decode_k_split": args.split and any(getattr(u, "work", None) is not None
                                                          for u in units),
@@ -584,7 +606,7 @@ def oracle_inputs(workload: str, max_rows: int):
             # group 0's real rows against group 0's weights
             wq, ws = oracle.quantize_fp8_blocks(synthetic.bf16_bits(w[:c.N]))
             items.append((synthetic.bf16_bits(a[:r]), wq, ws, 2.0 * c.N * c.K))
-        elif kind == "grouped":
+        elif kind in ("grouped", "psum"):
             a, w, m_indices, _ = synthetic.make_moe_inputs(c)
             r = min(max_rows, 128)
             # the first rows belong to group 0: its weights are the product's B
@@ -703,7 +725,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "decode", "moe", "moe_masked", "square", "tiny"],
+    ap.add_argument("--workload", choices=["prefill", "decode", "moe", "moe_psum", "moe_masked", "square", "tiny"],
                     default="prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -716,6 +738,8 @@ def main():
                          "per CTA at N = 12288 on B200)")
     ap.add_argument("--no-weight-prefetch", action="store_true",
                     help="GEMMs wait for the previous kernel before streaming weights")
+    ap.add_argument("--grouped-cta-pairs", type=int, default=0, choices=[0, 1],
+                    help="moe_psum: 256x256 tiles on CTA pairs (1) or 128-row tiles (0)")
     ap.add_argument("--cta-pairs", type=int, default=1, choices=[0, 1, 2],
                     help="dense GEMMs with M > 128: 0 one CTA per 128x256 tile, 1 CTA pairs on "
                          "256x256 tiles, 2 CTA pairs on 256x128 tiles")

@@ -239,6 +239,40 @@ lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sf
                                              void* stream);
 
 /*
+ * M-grouped contiguous block-scaled FP8 GEMM with the prefix-sum group layout
+ * (deepgemm-rust README: the device-level m_grouped contiguous entry point
+ * "(psum layout)", and "The mk_alignment knob (MoE tile width)": each group's
+ * tokens start at an aligned row of the A arena; on SM100 the alignment may be
+ * 256 so that tiles run at the MMA's full 256-row width).  The group boundaries
+ * stay on the device: no per-row ids and no host synchronization.
+ *
+ *   psum        [num_groups] int32 on the device: psum[g] = tokens of groups
+ *               0..g (non-decreasing).  Group g has count_g = psum[g] -
+ *               psum[g-1] tokens (psum[-1] = 0) at rows start_g .. start_g +
+ *               count_g - 1 of the arena, start_0 = 0 and start_{g+1} = start_g +
+ *               align_up(count_g, alignment).
+ *   alignment   128 or 256 (the mk_alignment of the layout).  Tiles are 128
+ *               rows; those holding pad rows only are skipped, so both
+ *               alignments compute the same rows.  With 256, N >= 256 and
+ *               lnq_set_grouped_cta_pairs(1) the tiles are 256 x 256 on CTA pairs.
+ *   a_e4m3      [M_total][K] E4M3 arena; sfa [K/128][M_total] fp32 MN-major.
+ *   b_e4m3      [num_groups*N][K] E4M3, sfb [num_groups*ceil(N/128)][K/128] fp32:
+ *               as in lnq_m_grouped_fp8_gemm_contiguous.
+ *   d_bf16      [M_total][N] bf16: the rows of each group's tokens are written;
+ *               pad rows and rows past the last group are left untouched.
+ *   Requires: alignment in {128, 256} (else LNQ_ERR_INVALID_ARG), M_total %
+ *   alignment == 0, N % 16 == 0, K % 128 == 0, sfb and psum 4-byte aligned, the
+ *   other pointers 16-byte aligned.  A decreasing psum (its negative counts are
+ *   taken as zero) or groups that overrun M_total (rows from M_total on are not
+ *   written) are reported by lnq_get_last_device_error as LNQ_ERR_INVALID_ARG.
+ */
+lnq_status lnq_m_grouped_fp8_gemm_contiguous_psum(const void* a_e4m3, const float* sfa,
+                                                  const void* b_e4m3, const float* sfb,
+                                                  const int32_t* psum, int32_t num_groups,
+                                                  int64_t alignment, void* d_bf16, int64_t M_total,
+                                                  int64_t N, int64_t K, void* stream);
+
+/*
  * M-grouped masked block-scaled FP8 GEMM (MoE experts fed by a token dispatch):
  * every group has a fixed buffer of M_max rows, of which only the first
  * masked_m[g] hold tokens; the counts stay on the device, so no host
@@ -300,6 +334,15 @@ lnq_status lnq_selftest_wait_timeout(int64_t timeout_ns, void* stream);
  * Returns the previous setting.
  */
 int32_t lnq_set_dense_cta_pairs(int32_t enable);
+
+/*
+ * Tuning knob (process-wide, default 0) for lnq_m_grouped_fp8_gemm_contiguous_psum
+ * with alignment 256 and N >= 256: 1 runs its 256 x 256 tiles on CTA pairs (each
+ * CTA loading half of the weight tile, as for dense tiles), any other value
+ * 128-row tiles on single CTAs, skipping tiles of pad rows only.  Results are the
+ * same up to FP32 summation order.  Returns the previous setting.
+ */
+int32_t lnq_set_grouped_cta_pairs(int32_t enable);
 
 /*
  * Weight prefetch (process-wide, default 0).  Every kernel of this library is

@@ -27,8 +27,10 @@ import torch
 __all__ = [
     "LnqError", "library_path", "lib",
     "lnq_quantize_fp8_groups", "lnq_quantize_fp8_blocks", "lnq_fp8_block_gemm_nt",
-    "lnq_m_grouped_fp8_gemm_contiguous", "lnq_get_last_device_error", "lnq_status_string",
-    "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "lnq_set_weight_prefetch",
+    "lnq_m_grouped_fp8_gemm_contiguous", "lnq_m_grouped_fp8_gemm_contiguous_psum",
+    "lnq_m_grouped_fp8_gemm_masked", "lnq_get_last_device_error", "lnq_status_string",
+    "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs",
+    "lnq_set_weight_prefetch",
     "quantize_activations", "quantize_weights",
     "quantize_weights_grouped", "linear",
     "m_grouped_linear", "ceil4",
@@ -77,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "lnq_fp8_block_gemm_nt_static_ws": [P, P, I64, P, P, P, I64, I64, I64, P],
             "lnq_m_grouped_fp8_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
             "lnq_m_grouped_fp8_gemm_masked": [P, P, P, P, P, I32, I64, I64, P, I64, I64, P],
+            "lnq_m_grouped_fp8_gemm_contiguous_psum": [P, P, P, P, P, I32, I64, P, I64, I64, I64, P],
             "lnq_get_last_device_error": [P],
             "lnq_selftest_wait_timeout": [I64, P],
         }
@@ -89,7 +92,7 @@ def lib() -> ctypes.CDLL:
         L.lnq_abi_version.restype = ctypes.c_int32
         L.lnq_fp8_block_gemm_nt_workspace_bytes.argtypes = [I64, I64, I64, I32]
         L.lnq_fp8_block_gemm_nt_workspace_bytes.restype = I64
-        for knob in ("lnq_set_dense_cta_pairs", "lnq_set_weight_prefetch"):
+        for knob in ("lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs", "lnq_set_weight_prefetch"):
             getattr(L, knob).argtypes = [ctypes.c_int32]
             getattr(L, knob).restype = ctypes.c_int32
         _lib = L
@@ -291,6 +294,29 @@ def lnq_m_grouped_fp8_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: tor
            "lnq_m_grouped_fp8_gemm_contiguous")
 
 
+def lnq_m_grouped_fp8_gemm_contiguous_psum(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,
+                                           sfb: torch.Tensor, psum: torch.Tensor, d: torch.Tensor,
+                                           alignment: int = 128, stream=None) -> None:
+    """a e4m3 [M_total, K], sfa [K/128, M_total], b e4m3 [G*N, K], sfb [G*ceil(N/128), K/128],
+    psum int32 [G] on the device (tokens of groups 0..g), d bf16 [M_total, N]; group g's tokens
+    start at the sum of the earlier groups' counts rounded up to `alignment` (128 or 256)."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.float32 or \
+            sfb.dtype != torch.float32 or d.dtype != torch.bfloat16 or psum.dtype != torch.int32:
+        raise TypeError("a, b e4m3; sfa, sfb float32; psum int32; d bf16")
+    for t in (a, sfa, b, sfb, psum, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    M_total, K = a.shape
+    G = psum.numel()
+    N = d.shape[1]
+    if G == 0 or b.shape[0] != G * N or b.shape[1] != K or tuple(sfa.shape) != (K // 128, M_total) or \
+            tuple(sfb.shape) != (G * -(-N // 128), K // 128) or d.shape[0] != M_total:
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_m_grouped_fp8_gemm_contiguous_psum(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(psum), G,
+                                                        int(alignment), _ptr(d), M_total, N, K, _stream(stream)),
+           "lnq_m_grouped_fp8_gemm_contiguous_psum")
+
+
 def lnq_m_grouped_fp8_gemm_masked(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
                                   masked_m: torch.Tensor, d: torch.Tensor, expected_m: int = 0,
                                   stream=None) -> None:
@@ -328,6 +354,12 @@ def lnq_set_dense_cta_pairs(mode: int) -> int:
     """Dense GEMM configuration for M > 128: 0 one CTA per 128x256 tile, 1 CTA pairs on
     256x256 tiles, 2 CTA pairs on 256x128 tiles.  Returns the previous setting."""
     return int(lib().lnq_set_dense_cta_pairs(int(mode)))
+
+
+def lnq_set_grouped_cta_pairs(mode: int) -> int:
+    """Prefix-sum grouped GEMM with 256-row alignment: 1 runs 256x256 tiles on CTA pairs,
+    0 (the default) 128-row tiles on single CTAs.  Returns the previous setting."""
+    return int(lib().lnq_set_grouped_cta_pairs(int(mode)))
 
 
 def lnq_set_weight_prefetch(enable: bool) -> bool:

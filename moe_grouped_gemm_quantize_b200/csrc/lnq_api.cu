@@ -42,6 +42,9 @@ struct DeviceInfo {
 std::mutex g_mutex;
 // Dense GEMMs with M > 128 run on CTA pairs when set (1: 256x256, 2: 256x128 tiles).
 std::atomic<int> g_dense_pairs{1};
+// Grouped GEMMs in the prefix-sum layout with 256-row alignment run 256 x 256 tiles on
+// CTA pairs when set (otherwise 128-row tiles, skipping those of pad rows only).
+std::atomic<int> g_grouped_pairs{0};
 // GEMMs may start streaming weights before the prior kernel completes.
 std::atomic<int> g_weight_prefetch{0};
 DeviceInfo g_devices[kMaxDevices];
@@ -186,6 +189,7 @@ using CfgPair128 = GemmCfg<128, 8, 2, false, false, true>;
 using CfgDense128 = GemmCfg<128, 6, 2, false, false>;
 using CfgGrouped256 = GemmCfg<256, 4, 2, false, true>;
 using CfgGrouped128 = GemmCfg<128, 6, 2, false, true>;
+using CfgGroupedPair256 = GemmCfg<256, 6, 2, false, true, true>;
 using CfgSwap32 = GemmCfg<32, 10, 1, true, false>;
 using CfgSwap64 = GemmCfg<64, 8, 1, true, false>;
 using CfgSwap32Split = GemmCfg<32, 10, 1, true, false, false, 1, true>;
@@ -212,6 +216,10 @@ extern "C" {
 int32_t lnq_abi_version(void) { return 10000; }
 
 int32_t lnq_set_weight_prefetch(int32_t enable) { return g_weight_prefetch.exchange(enable ? 1 : 0); }
+
+int32_t lnq_set_grouped_cta_pairs(int32_t enable) {
+    return g_grouped_pairs.exchange(enable == 1 ? 1 : 0);
+}
 
 int32_t lnq_set_dense_cta_pairs(int32_t enable) {
     const int previous = g_dense_pairs.exchange(enable >= 0 && enable <= 2 ? enable : 0);
@@ -550,6 +558,61 @@ lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sf
     args.tiles_p = static_cast<int>(M_total / 128);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t wrows = static_cast<int64_t>(num_groups) * N;
+    if (N >= 256) {
+        args.tiles_q = static_cast<int>((N + 255) / 256);
+        args.num_tiles = args.tiles_p * args.tiles_q;
+        return launch_gemm<CfgGrouped256>(*dev, a_e4m3, M_total, b_e4m3, wrows, K, args, s);
+    }
+    args.tiles_q = static_cast<int>((N + 127) / 128);
+    args.num_tiles = args.tiles_p * args.tiles_q;
+    return launch_gemm<CfgGrouped128>(*dev, a_e4m3, M_total, b_e4m3, wrows, K, args, s);
+}
+
+lnq_status lnq_m_grouped_fp8_gemm_contiguous_psum(const void* a_e4m3, const float* sfa,
+                                                  const void* b_e4m3, const float* sfb,
+                                                  const int32_t* psum, int32_t num_groups,
+                                                  int64_t alignment, void* d_bf16, int64_t M_total,
+                                                  int64_t N, int64_t K, void* stream) {
+    if (M_total <= 0 || N <= 0 || K <= 0 || num_groups <= 0) return LNQ_ERR_INVALID_ARG;
+    if (alignment != 128 && alignment != 256) return LNQ_ERR_INVALID_ARG;
+    if (M_total % alignment != 0 || K % 128 != 0 || N % 16 != 0 || N < 16 || M_total > kMaxRows ||
+        K > (int64_t{1} << 31) || static_cast<int64_t>(num_groups) * N > kMaxRows)
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!a_e4m3 || !sfa || !b_e4m3 || !sfb || !psum || !d_bf16) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned4(sfb) ||
+        !aligned16(d_bf16) || !aligned4(psum))
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+
+    // The grouped kernel with each tile's group looked up in psum on the device (no
+    // host synchronization, no per-row ids).  Groups aligned to 256 rows hold whole
+    // 256-row tiles, which may run on CTA pairs like the dense ones; by default the
+    // tiles are 128 rows and those holding pad rows only are skipped, so the rows
+    // computed are the same as with 128-row alignment.
+    GemmArgs args{};
+    args.sfa = sfa;
+    args.sfb = sfb;
+    args.d = static_cast<uint16_t*>(d_bf16);
+    args.m_indices = nullptr;
+    args.psum = psum;
+    args.align = static_cast<int>(alignment);
+    args.M4 = M_total;
+    args.M = static_cast<int>(M_total);
+    args.N = static_cast<int>(N);
+    args.num_kb = static_cast<int>(K / 128);
+    args.nb = static_cast<int>((N + 127) / 128);
+    args.num_groups = num_groups;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t wrows = static_cast<int64_t>(num_groups) * N;
+    if (alignment == 256 && N >= 256 && g_grouped_pairs.load(std::memory_order_relaxed) != 0) {
+        args.tiles_p = static_cast<int>(M_total / 256);
+        args.tiles_q = static_cast<int>((N + 255) / 256);
+        args.num_tiles = args.tiles_p * args.tiles_q;
+        return launch_gemm<CfgGroupedPair256>(*dev, a_e4m3, M_total, b_e4m3, wrows, K, args, s);
+    }
+    args.tiles_p = static_cast<int>(M_total / 128);
     if (N >= 256) {
         args.tiles_q = static_cast<int>((N + 255) / 256);
         args.num_tiles = args.tiles_p * args.tiles_q;

@@ -13,7 +13,10 @@
 //     operand"), BNQ weight rows in its N slot ("Q operand");
 //   * M-grouped contiguous (MoE): as single-CTA dense, each 128-row block of
 //     activations takes the weights of the group named by its first row's id
-//     (deepgemm-rust README, "Grouped (contiguous) MoE GEMM");
+//     (deepgemm-rust README, "Grouped (contiguous) MoE GEMM"), or of the group
+//     whose aligned rows hold it in the prefix-sum layout; with 256-row group
+//     alignment the grouped tiles run on CTA pairs as dense ones do
+//     (deepgemm-rust README, "The mk_alignment knob (MoE tile width)");
 //   * decode (M <= 64, "swap AB"): the weights fill the 128-row M slot and the
 //     few tokens the N slot, so the tensor core is not idle on padding rows.
 //
@@ -71,6 +74,11 @@ struct GemmArgs {
     // g*m_max .. g*m_max + m_max - 1, of which the first masked_m[g] are real.
     const int32_t* masked_m;  // [num_groups], on the device
     int m_max;                // rows per group, a multiple of 128
+    // Grouped, prefix-sum layout only (m_indices == nullptr, psum != nullptr): psum[g]
+    // counts the tokens of groups 0..g; group g's tokens start at the row
+    // sum_{j<g} align_up(count_j, align), align a multiple of the tile's rows.
+    const int32_t* psum;      // [num_groups], on the device
+    int align;
     // Fused epilogue (dense and decode tiles): an optional bf16 bias per output
     // column added in FP32; and, instead of the bf16 D, the output quantized for a
     // next linear (dense 128 x 256 tiles only): E4M3 codes [M][N] and FP32 scales
@@ -96,7 +104,7 @@ struct GemmCfg {
     static constexpr bool SPLITK = SPLITK_;
     static_assert(!SPLITK || SWAP, "the K split serves the decode configuration");
     static_assert(!(SWAP && GROUPED), "decode configuration is dense only");
-    static_assert(!(PAIR && (SWAP || GROUPED)), "CTA pairs serve the dense configuration");
+    static_assert(!(PAIR && SWAP), "CTA pairs serve the dense and grouped configurations");
     static_assert(BNQ % 16 == 0 && BNQ >= 16 && BNQ <= 256, "MMA N for M=128/256");
     static_assert(!SWAP || EPI_WG == 1, "decode epilogue: one thread per weight row");
     static_assert(!SWAP || BNQ % 32 == 0, "decode tiles read TMEM in 32-column chunks");
@@ -204,6 +212,54 @@ struct TileCoord {
     int row_end;  // output rows from row_end on are not stored (dense and grouped tiles)
 };
 
+// Prefix-sum layout: the group whose aligned rows hold arena row r, and the end of
+// its tokens (group -1 past the last group).  Runs on a whole warp: each lane takes
+// one group of a run of 32, the run's aligned counts are summed by a warp scan, and
+// the run whose aligned rows reach past r holds the group.  A count below zero (a
+// decreasing psum) is reported and taken as zero.  Returns the first row after the
+// runs scanned (after all groups when r lies past them).
+__device__ __forceinline__ long long psum_lookup(const GemmArgs& a, int r, int& group, int& row_end) {
+    const int lane = static_cast<int>(threadIdx.x & 31u);
+    const long long align = a.align;
+    long long base = 0;   // first row of the run's first group
+    int prev_psum = 0;    // psum of the group before the run
+    group = -1;
+    row_end = 0;
+    for (int g0 = 0; g0 < a.num_groups && base <= r; g0 += 32) {
+        const int g = g0 + lane;
+        const bool real = g < a.num_groups;
+        const int ps = real ? __ldg(a.psum + g) : 0;
+        int before = __shfl_up_sync(0xffffffffu, ps, 1);
+        if (lane == 0) before = prev_psum;
+        long long count = real ? static_cast<long long>(ps) - before : 0;
+        if (count < 0) {
+            atomicOr(a.status, kStatusBadGroup);
+            count = 0;
+        }
+        const long long padded = (count + align - 1) / align * align;
+        long long end = padded;  // inclusive scan of the aligned counts
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const long long v = __shfl_up_sync(0xffffffffu, end, d);
+            if (lane >= d) end += v;
+        }
+        end += base;
+        const long long start = end - padded;
+        const unsigned hit = __ballot_sync(0xffffffffu, count > 0 && start <= r && r < end);
+        if (hit != 0u) {
+            const int src = __ffs(hit) - 1;
+            group = g0 + src;
+            const long long tok_end = __shfl_sync(0xffffffffu, start + count, src);
+            row_end = static_cast<int>(tok_end < a.M ? tok_end : a.M);
+            if (tok_end > a.M) atomicOr(a.status, kStatusBadGroup);
+            break;
+        }
+        base = __shfl_sync(0xffffffffu, end, 31);
+        prev_psum = __shfl_sync(0xffffffffu, ps, 31);
+    }
+    return base;
+}
+
 // Tile t of this CTA (or of this CTA pair; `rank` is the CTA's rank in the pair).
 template <class C>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32_t rank) {
@@ -229,7 +285,17 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32
         c.q0 = (r / rows) * C::BNQ;
         c.row_end = a.M;
         if constexpr (C::GROUPED) {
-            if (a.m_indices != nullptr) {
+            if (a.psum != nullptr) {
+                // prefix-sum layout: the group is looked up at the pair's first row, so
+                // both CTAs of a pair take it (a group's aligned rows hold whole tiles)
+                int g, end;
+                psum_lookup(a, c.p0 - static_cast<int>(rank) * C::kP, g, end);
+                c.group = g;
+                c.row_end = end;
+                // a single-CTA tile of pad rows only (groups aligned to more rows than
+                // a tile) is skipped; a pair's tile always holds tokens of its group
+                if (!C::PAIR && end <= c.p0) c.group = -1;
+            } else if (a.m_indices != nullptr) {
                 // contiguous: the block's group is that of its first row
                 c.group = __ldg(a.m_indices + c.p0);
                 if (c.group >= a.num_groups) {
@@ -443,25 +509,25 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             // prior kernel, the activation halves after it.
             int prefetched = 0;
             if (args.prefetch_weights) {
-                if constexpr (!C::PAIR) {
+                // dense tiles only: a grouped tile's weights depend on group ids or
+                // counts that the prior kernel may still be writing
+                if constexpr (!C::PAIR && !C::GROUPED) {
                     Segment sg0;
                     if (segment<C>(args, unit, units, 0, sg0)) {
                         const TileCoord tc = tile_coord<C>(args, sg0.t, rank);
-                        if (tc.group >= 0 && !C::GROUPED) {
-                            prefetched = min(C::STAGES, sg0.kb_hi - sg0.kb_lo);
-                            if (elect_one()) {
-                                for (int s = 0; s < prefetched; ++s) {
-                                    mbar_arrive_expect_tx(full_bar(s), C::kPBytes + C::kQBytes);
-                                    if constexpr (C::SWAP)
-                                        tma_load_2d(sP + s * C::kPBytes, &map_p, full_bar(s),
-                                                    (sg0.kb_lo + s) * C::kBK, tc.p0);
-                                    else
-                                        tma_load_2d(sQ + s * C::kQBytes, &map_q, full_bar(s),
-                                                    (sg0.kb_lo + s) * C::kBK, tc.q0);
-                                }
+                        prefetched = min(C::STAGES, sg0.kb_hi - sg0.kb_lo);
+                        if (elect_one()) {
+                            for (int s = 0; s < prefetched; ++s) {
+                                mbar_arrive_expect_tx(full_bar(s), C::kPBytes + C::kQBytes);
+                                if constexpr (C::SWAP)
+                                    tma_load_2d(sP + s * C::kPBytes, &map_p, full_bar(s),
+                                                (sg0.kb_lo + s) * C::kBK, tc.p0);
+                                else
+                                    tma_load_2d(sQ + s * C::kQBytes, &map_q, full_bar(s),
+                                                (sg0.kb_lo + s) * C::kBK, tc.q0);
                             }
-                            __syncwarp();
                         }
+                        __syncwarp();
                     }
                 }
                 wait_prior_grids();
@@ -657,6 +723,14 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         uint32_t sphase = 0;
         bool ok = true;
         constexpr int kSaLanes = C::kSaPerTile / 4;  // lanes that copy 16 bytes of sa
+        if constexpr (C::GROUPED) {
+            // prefix-sum layout: groups whose aligned rows run past the arena are
+            // reported once per launch (tiles past M_total are never looked up)
+            if (args.psum != nullptr && blockIdx.x == 0) {
+                int g, e;
+                if (psum_lookup(args, 0x7fffffff, g, e) > args.M) atomicOr(args.status, kStatusBadGroup);
+            }
+        }
         Segment sg;
         for (int i = 0; ok && segment<C>(args, unit, units, i, sg); ++i) {
             const TileCoord tc = tile_coord<C>(args, sg.t, rank);

@@ -77,6 +77,18 @@ def contiguous_layout(sizes, block: int = BLOCK):
     return m_indices, starts, M_total
 
 
+def psum_layout(sizes, alignment: int = 256):
+    """Prefix-sum layout: (psum int32 [G], starts int64 [G], M_total).
+
+    psum[g] counts the tokens of groups 0..g; group g occupies rows starts[g] ..
+    starts[g]+sizes[g]-1, starts being the running sum of the sizes rounded up to
+    `alignment`, and M_total the sum of all rounded sizes.
+    """
+    m_indices, starts, M_total = contiguous_layout(sizes, alignment)
+    psum = np.cumsum(np.asarray(sizes, dtype=np.int64)).astype(np.int32)
+    return psum, starts, M_total
+
+
 def bf16_bits(x: torch.Tensor) -> np.ndarray:
     """The uint16 bit patterns of a CPU bf16 tensor (what the oracle reads)."""
     assert x.dtype == torch.bfloat16
@@ -184,10 +196,11 @@ def make_linear_inputs(cfg: Linear, device="cpu"):
     return a, w
 
 
-def make_moe_inputs(cfg: MoE = MOE, device="cpu"):
-    """(A bf16 [M_total, K] with zero pad rows, W bf16 [G*N, K], m_indices, sizes)."""
+def make_moe_inputs(cfg: MoE = MOE, device="cpu", alignment: int = BLOCK):
+    """(A bf16 [M_total, K] with zero pad rows, W bf16 [G*N, K], m_indices, sizes); each
+    group's rows start at a multiple of `alignment`."""
     sizes = cfg.group_sizes()
-    m_indices, _, M_total = contiguous_layout(sizes)
+    m_indices, _, M_total = contiguous_layout(sizes, alignment)
     a = gaussian_bf16((M_total, cfg.K), cfg.a_std, cfg.a_seed, device)
     pad = torch.from_numpy(m_indices < 0).to(device)
     a = a.masked_fill(pad.unsqueeze(1), 0.0)

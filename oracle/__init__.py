@@ -72,6 +72,8 @@ def _load():
         lib.oracle_m_grouped_gemm_points.restype = ctypes.c_int
         lib.oracle_m_grouped_gemm_points.argtypes = [
             P, P, P, P, P, ctypes.c_int32, I64, I64, I64, P, P, I64, P]
+        lib.oracle_m_grouped_gemm_psum.restype = ctypes.c_int
+        lib.oracle_m_grouped_gemm_psum.argtypes = [P, P, P, P, P, ctypes.c_int32, I64, I64, I64, I64, P]
         lib.oracle_m_grouped_gemm_masked.restype = ctypes.c_int
         lib.oracle_m_grouped_gemm_masked.argtypes = [P, P, I64, P, P, P, ctypes.c_int32, I64, I64, I64, P]
         lib.oracle_m_grouped_gemm_masked_points.restype = ctypes.c_int
@@ -251,3 +253,20 @@ def m_grouped_gemm_masked_points(qa, sfa, qb, sfb, masked_m, M_max: int, rows, c
                                                        _ptr(mm), G, M_max, N, K, _ptr(rows), _ptr(cols),
                                                        rows.size, _ptr(out)), "m_grouped_gemm_masked_points")
     return out
+
+
+def m_grouped_gemm_psum(qa, sfa, qb, sfb, psum, alignment: int) -> np.ndarray:
+    """FP64 D [M_total, N] of the prefix-sum grouped layout: group g's psum[g] - psum[g-1]
+    tokens start at the aligned row sum_{j<g} align_up(count_j, alignment); other rows NaN."""
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    sfa = _c(sfa, np.float32)
+    sfb = _c(sfb, np.float32)
+    ps = _c(np.asarray(psum, dtype=np.int32), np.int32)
+    G = ps.size
+    M_total, K = qa.shape
+    N = qb.shape[0] // G
+    D = np.full((M_total, N), np.nan, dtype=np.float64)
+    _check(_load().oracle_m_grouped_gemm_psum(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(ps), G,
+                                              alignment, M_total, N, K, _ptr(D)), "m_grouped_gemm_psum")
+    return D

@@ -38,6 +38,12 @@
  *     deepgemm-rust README, "What's implemented", m_grouped_fp8_gemm_nt_masked
  *     (masked_m scheduler, DeepEP-style dispatch output, zero CPU sync).  The
  *     weights and their scales are laid out as in the contiguous variant.
+ *   - M-grouped contiguous layout described by prefix sums: psum[g] is the
+ *     number of tokens of groups 0..g, and group g's tokens start at the row
+ *     sum_{j<g} align_up(count_j, alignment) of the A arena (alignment 128 or
+ *     256): deepgemm-rust README, "The mk_alignment knob (MoE tile width)"
+ *     (each group's tokens start at an aligned row) and the psum-layout
+ *     contiguous entry point of the device-level API.
  *   - E4M3 round-to-nearest-even with saturation at 448, scale = amax/448:
  *     the benchmark spec's numerics (the pages never print 448; the encoder
  *     below is written from the OCP FP8 E4M3 format definition: bias 7,
@@ -500,5 +506,68 @@ int oracle_m_grouped_gemm_masked_points(const uint8_t* qa, const float* sfa, int
         free(ad);
         free(bd);
     }
+    return 0;
+}
+
+/* M-grouped contiguous product with the prefix-sum layout: group g has
+ * count_g = psum[g] - psum[g-1] tokens (psum[-1] = 0) at rows start_g ..
+ * start_g + count_g - 1 of the arena, start_0 = 0, start_{g+1} = start_g +
+ * align_up(count_g, alignment).  Those rows of D get the product with group g's
+ * weights; every other row of D is left untouched.  qa is [M_total][K], sfa is
+ * [K/128][M_total].  Returns -1 if psum decreases or the groups overrun M_total. */
+int oracle_m_grouped_gemm_psum(const uint8_t* qa, const float* sfa, const uint8_t* qb,
+                               const float* sfb, const int32_t* psum, int32_t G,
+                               int64_t alignment, int64_t M_total, int64_t N, int64_t K, double* D)
+{
+    int64_t g, NB, start = 0, prev = 0;
+    int64_t* first = NULL;
+    int64_t* count = NULL;
+    if (G <= 0 || M_total <= 0 || N <= 0 || K <= 0 || K % ORACLE_GROUP != 0 || alignment <= 0)
+        return -1;
+    first = (int64_t*)malloc(sizeof(int64_t) * (size_t)G);
+    count = (int64_t*)malloc(sizeof(int64_t) * (size_t)G);
+    if (!first || !count) {
+        free(first);
+        free(count);
+        return -2;
+    }
+    for (g = 0; g < G; ++g) {
+        const int64_t c = (int64_t)psum[g] - prev;
+        if (c < 0) {
+            free(first);
+            free(count);
+            return -1;
+        }
+        first[g] = start;
+        count[g] = c;
+        start += (c + alignment - 1) / alignment * alignment;
+        prev = psum[g];
+    }
+    if (start > M_total) {
+        free(first);
+        free(count);
+        return -1;
+    }
+    NB = (N + ORACLE_GROUP - 1) / ORACLE_GROUP;
+    for (g = 0; g < G; ++g) {
+        int64_t i;
+#pragma omp parallel for schedule(dynamic, 1)
+        for (i = 0; i < count[g]; ++i) {
+            int64_t n, row = first[g] + i;
+            double* ad = (double*)malloc(sizeof(double) * (size_t)K);
+            double* bd = (double*)malloc(sizeof(double) * (size_t)K);
+            if (ad && bd) {
+                dequant_a_row(qa, sfa, M_total, K, row, ad);
+                for (n = 0; n < N; ++n) {
+                    dequant_b_row(qb, sfb, K, g * N + n, g * NB + n / ORACLE_GROUP, bd);
+                    D[row * N + n] = dot(ad, bd, K);
+                }
+            }
+            free(ad);
+            free(bd);
+        }
+    }
+    free(first);
+    free(count);
     return 0;
 }

@@ -133,6 +133,23 @@ def test_masked_argument_errors(L):
     assert call(a=A16 + 1) == MISALIGNED
 
 
+def test_psum_argument_errors(L):
+    f = L.lnq_m_grouped_fp8_gemm_contiguous_psum
+
+    def call(M_total=512, N=256, K=512, G=4, ps=A16e + 0x1000, align=256, a=A16):
+        return f(a, A16b, A16c, A16d, ps, G, align, A16e, M_total, N, K, None)
+
+    assert call(G=0) == INVALID
+    assert call(align=64) == INVALID
+    assert call(align=512) == INVALID
+    assert call(M_total=384) == SHAPE           # M_total % alignment
+    assert call(K=100) == SHAPE
+    assert call(N=20) == SHAPE
+    assert call(ps=None) == INVALID
+    assert call(ps=A16e + 0x1002) == MISALIGNED
+    assert call(a=A16 + 1) == MISALIGNED
+
+
 def test_epilogue_argument_errors(L):
     f = L.lnq_fp8_block_gemm_nt_epilogue
 
