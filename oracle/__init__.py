@@ -72,6 +72,8 @@ def _load():
         lib.oracle_m_grouped_gemm_points.restype = ctypes.c_int
         lib.oracle_m_grouped_gemm_points.argtypes = [
             P, P, P, P, P, ctypes.c_int32, I64, I64, I64, P, P, I64, P]
+        lib.oracle_silu_mul.restype = None
+        lib.oracle_silu_mul.argtypes = [P, P, I64, P]
         lib.oracle_m_grouped_gemm_psum.restype = ctypes.c_int
         lib.oracle_m_grouped_gemm_psum.argtypes = [P, P, P, P, P, ctypes.c_int32, I64, I64, I64, I64, P]
         lib.oracle_m_grouped_gemm_masked.restype = ctypes.c_int
@@ -270,3 +272,36 @@ def m_grouped_gemm_psum(qa, sfa, qb, sfb, psum, alignment: int) -> np.ndarray:
     _check(_load().oracle_m_grouped_gemm_psum(_ptr(qa), _ptr(sfa), _ptr(qb), _ptr(sfb), _ptr(ps), G,
                                               alignment, M_total, N, K, _ptr(D)), "m_grouped_gemm_psum")
     return D
+
+
+def silu_mul(g, u) -> np.ndarray:
+    """FP64 silu(g) * u elementwise, silu(x) = x / (1 + e^-x)."""
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    u = np.ascontiguousarray(u, dtype=np.float64)
+    if g.shape != u.shape:
+        raise ValueError("gate and up shapes differ")
+    h = np.empty_like(g)
+    _load().oracle_silu_mul(_ptr(g), _ptr(u), g.size, _ptr(h))
+    return h
+
+
+def gemm_nt_silu_mul(qa, sfa, qb, sfb) -> np.ndarray:
+    """FP64 h [M, I] of a gate_up linear: D = A.B^T with B [2I, K] (gate rows, then up
+    rows), h = silu(D[:, :I]) * D[:, I:]."""
+    D = gemm_nt(qa, sfa, qb, sfb)
+    I = D.shape[1] // 2
+    if D.shape[1] != 2 * I:
+        raise ValueError("the gate_up weight needs an even row count")
+    return silu_mul(D[:, :I], D[:, I:])
+
+
+def gemm_nt_silu_mul_points(qa, sfa, qb, sfb, rows, cols) -> np.ndarray:
+    """FP64 h at the points (rows[i], cols[i]), cols < I."""
+    I = qb.shape[0] // 2
+    rows = np.asarray(rows, dtype=np.int64)
+    cols = np.asarray(cols, dtype=np.int64)
+    if np.any(cols < 0) or np.any(cols >= I):
+        raise ValueError("columns must lie below I")
+    g = gemm_nt_points(qa, sfa, qb, sfb, rows, cols)
+    u = gemm_nt_points(qa, sfa, qb, sfb, rows, cols + I)
+    return silu_mul(g, u)

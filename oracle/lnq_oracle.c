@@ -44,6 +44,9 @@
  *     256): deepgemm-rust README, "The mk_alignment knob (MoE tile width)"
  *     (each group's tokens start at an aligned row) and the psum-layout
  *     contiguous entry point of the device-level API.
+ *   - SiLU.mul after a gate_up linear: deepgemm-rust README, "What's
+ *     implemented", moe_fp8_layer (grouped GEMM -> SiLU.mul -> grouped GEMM);
+ *     silu(x) = x / (1 + e^-x), the sigmoid-weighted linear unit.
  *   - E4M3 round-to-nearest-even with saturation at 448, scale = amax/448:
  *     the benchmark spec's numerics (the pages never print 448; the encoder
  *     below is written from the OCP FP8 E4M3 format definition: bias 7,
@@ -59,7 +62,10 @@
  *   - magnitudes above 448 saturate to +-448 (0x7E / 0xFE);
  *   - pad scale entries (rows M..M4-1) are written as 0.0f;
  *   - grouped rows whose group id is negative contribute nothing and their
- *     output row is left untouched.
+ *     output row is left untouched;
+ *   - SiLU.mul: the gate_up weight stacks the I gate rows over the I up rows,
+ *     and h[m][j] = silu(D[m][j]) * D[m][I + j] is taken of the product itself
+ *     (before any BF16 rounding of D).
  *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
  * x86-64 evaluates float arithmetic in SSE single precision
@@ -570,4 +576,14 @@ int oracle_m_grouped_gemm_psum(const uint8_t* qa, const float* sfa, const uint8_
     free(first);
     free(count);
     return 0;
+}
+
+/* SiLU.mul of n gate/up pairs: h[i] = silu(g[i]) * u[i], silu(x) = x / (1 + e^-x)
+ * in FP64.  For x below about -709, e^-x overflows to infinity and x / inf gives
+ * -0.0, which is silu's limit there. */
+void oracle_silu_mul(const double* g, const double* u, int64_t n, double* h)
+{
+    int64_t i;
+    for (i = 0; i < n; ++i)
+        h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
 }
