@@ -191,7 +191,7 @@ class ClockSampler:
 class Linear:
     """One dense linear: bf16 activations resident on the device, weights pre-quantized."""
 
-    def __init__(self, cfg, dev, split: bool = False, fp8_out: bool = False):
+    def __init__(self, cfg, dev, split: bool = False, fp8_out: bool = False, silu: bool = False):
         import moe_grouped_gemm_quantize_b200 as lnq
         from moe_grouped_gemm_quantize_b200 import synthetic
         self.cfg = cfg
@@ -223,6 +223,13 @@ class Linear:
             self.d2h_bytes = M * N + 4 * (N // 128) * self.M4
             self.host_qo = torch.empty((M, N), dtype=torch.uint8).pin_memory()
             self.host_so = torch.empty((N // 128, self.M4), dtype=torch.float32).pin_memory()
+        # fused epilogue of a gate_up linear: h = silu(gate) * up, N/2 bf16 columns
+        self.silu = silu and not self.fp8_out and "gate_up" in cfg.name and N % 256 == 0
+        if self.silu:
+            self.d = torch.empty((M, N // 2), dtype=torch.bfloat16, device=dev)
+            self.gemm_bytes -= M * N
+            self.d2h_bytes = M * N
+            self.host_d = torch.empty((M, N // 2), dtype=torch.bfloat16).pin_memory()
 
     def copy_out(self):
         """The step's result to pinned host memory (asynchronous)."""
@@ -249,6 +256,10 @@ class Linear:
                      P(self.ws.data_ptr()), P(0), P(0), P(self.qo.data_ptr()), P(self.so.data_ptr()),
                      self.M4, c.M, c.N, c.K, s)
             return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_fp8_block_gemm_nt_epilogue, eargs)
+        if self.silu:
+            sargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), self.M4, P(self.wq.data_ptr()),
+                     P(self.ws.data_ptr()), P(self.d.data_ptr()), c.M, c.N // 2, c.K, s)
+            return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_fp8_block_gemm_nt_silu_mul, sargs)
         if self.work is not None:
             return (L.lnq_quantize_fp8_groups, qargs), \
                 (L.lnq_fp8_block_gemm_nt_ws, gargs + (P(self.work.data_ptr()), self.work.numel(), s))
@@ -418,7 +429,8 @@ def run_ours(args, world, rank, local):
     cfgs, kind = workload_units(args.workload)
     units = [Grouped(c, dev) if kind == "grouped" else Grouped(c, dev, alignment=256) if kind == "psum"
              else Masked(c, dev) if kind == "masked"
-             else Linear(c, dev, split=args.split, fp8_out=args.epilogue == "fp8") for c in cfgs]
+             else Linear(c, dev, split=args.split, fp8_out=args.epilogue == "fp8",
+                         silu=args.epilogue == "silu") for c in cfgs]
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     calls = [u.calls(sp) for u in units]
@@ -731,8 +743,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
-    ap.add_argument("--epilogue", choices=["bf16", "fp8"], default="bf16",
-                    help="dense GEMM output: bf16 D, or E4M3 codes + 1x128 scales for a next linear")
+    ap.add_argument("--epilogue", choices=["bf16", "fp8", "silu"], default="bf16",
+                    help="dense GEMM output: bf16 D, E4M3 codes + 1x128 scales for a next linear, or "
+                         "(silu) h = silu(gate) * up of the gate_up linear in bf16")
     ap.add_argument("--split", action="store_true",
                     help="decode GEMMs through the workspace K split (slower than whole weight tiles "
                          "per CTA at N = 12288 on B200)")

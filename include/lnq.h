@@ -146,6 +146,24 @@ lnq_status lnq_fp8_block_gemm_nt_epilogue(const void* a_e4m3, const float* sfa, 
                                           int64_t M, int64_t N, int64_t K, void* stream);
 
 /*
+ * Gate_up linear with SiLU.mul fused into its epilogue (deepgemm-rust README,
+ * "What's implemented", moe_fp8_layer: grouped GEMM -> SiLU.mul -> grouped GEMM):
+ *     h[m][j] = bf16( silu(D[m][j]) * D[m][I + j] ),  silu(x) = x / (1 + e^-x),
+ * D = A . B^T promoted in FP32 as in lnq_fp8_block_gemm_nt; gate and up values
+ * are the FP32 products (D is never rounded to bf16).
+ *
+ *   b_e4m3   [2I][K] E4M3: the I gate rows, then the I up rows.
+ *   sfb      [2I/128][K/128] fp32, as lnq_quantize_fp8_blocks writes for 2I rows.
+ *   h_bf16   [M][I] bf16 row-major, fully overwritten.
+ *   Requires: M >= 1, I % 128 == 0, K % 128 == 0, M4 >= ceil4(M), M4 % 4 == 0,
+ *   sfb 4-byte aligned, the other pointers 16-byte aligned.  M > 128 runs
+ *   256-row tiles on CTA pairs (unless lnq_set_dense_cta_pairs(0)).
+ */
+lnq_status lnq_fp8_block_gemm_nt_silu_mul(const void* a_e4m3, const float* sfa, int64_t M4,
+                                          const void* b_e4m3, const float* sfb, void* h_bf16,
+                                          int64_t M, int64_t I, int64_t K, void* stream);
+
+/*
  * Bytes of workspace that lnq_fp8_block_gemm_nt_ws needs to split the K range of
  * a decode product (M <= 64) over `num_sms` CTAs, or 0 when the product does not
  * split (M > 64, K == 128, or at least one weight tile per SM already).  A pure

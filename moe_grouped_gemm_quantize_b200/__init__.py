@@ -28,6 +28,7 @@ __all__ = [
     "LnqError", "library_path", "lib",
     "lnq_quantize_fp8_groups", "lnq_quantize_fp8_blocks", "lnq_fp8_block_gemm_nt",
     "lnq_m_grouped_fp8_gemm_contiguous", "lnq_m_grouped_fp8_gemm_contiguous_psum",
+    "lnq_fp8_block_gemm_nt_silu_mul",
     "lnq_m_grouped_fp8_gemm_masked", "lnq_get_last_device_error", "lnq_status_string",
     "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs",
     "lnq_set_weight_prefetch",
@@ -80,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "lnq_m_grouped_fp8_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
             "lnq_m_grouped_fp8_gemm_masked": [P, P, P, P, P, I32, I64, I64, P, I64, I64, P],
             "lnq_m_grouped_fp8_gemm_contiguous_psum": [P, P, P, P, P, I32, I64, P, I64, I64, I64, P],
+            "lnq_fp8_block_gemm_nt_silu_mul": [P, P, I64, P, P, P, I64, I64, I64, P],
             "lnq_get_last_device_error": [P],
             "lnq_selftest_wait_timeout": [I64, P],
         }
@@ -292,6 +294,26 @@ def lnq_m_grouped_fp8_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: tor
                                                    _ptr(m_indices), G, _ptr(d), M_total, N, K,
                                                    _stream(stream)),
            "lnq_m_grouped_fp8_gemm_contiguous")
+
+
+def lnq_fp8_block_gemm_nt_silu_mul(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                                   h: torch.Tensor, stream=None) -> None:
+    """Gate_up linear with SiLU.mul: a e4m3 [M, K], sfa [K/128, M4], b e4m3 [2I, K] (gate rows
+    then up rows), sfb [2I/128, K/128], h bf16 [M, I] = silu(D[:, :I]) * D[:, I:]."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.float32 or sfb.dtype != torch.float32 or \
+            h.dtype != torch.bfloat16:
+        raise TypeError("a, b e4m3; sfa, sfb float32; h bf16")
+    for t in (a, sfa, b, sfb, h):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    M, K = a.shape
+    I = h.shape[1]
+    if b.shape[0] != 2 * I or b.shape[1] != K or h.shape[0] != M or sfa.shape[0] != K // 128 or \
+            tuple(sfb.shape) != (-(-2 * I // 128), K // 128):
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_fp8_block_gemm_nt_silu_mul(_ptr(a), _ptr(sfa), sfa.shape[1], _ptr(b), _ptr(sfb), _ptr(h),
+                                                M, I, K, _stream(stream)),
+           "lnq_fp8_block_gemm_nt_silu_mul")
 
 
 def lnq_m_grouped_fp8_gemm_contiguous_psum(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,

@@ -116,7 +116,8 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
     } else {
         st = encode_e4m3_map(&map_p, act, act_rows, K, C::kP);
         if (st == LNQ_OK)
-            st = encode_e4m3_map(&map_q, wgt, wgt_rows, K, C::PAIR ? C::kSliceQRows : C::kQRowsPerCta);
+            st = encode_e4m3_map(&map_q, wgt, wgt_rows, K,
+                                 C::SILU ? C::kQBoxRows : (C::PAIR ? C::kSliceQRows : C::kQRowsPerCta));
     }
     if (st != LNQ_OK) return st;
     static bool attr_set[kMaxDevices] = {};
@@ -190,6 +191,8 @@ using CfgDense128 = GemmCfg<128, 6, 2, false, false>;
 using CfgGrouped256 = GemmCfg<256, 4, 2, false, true>;
 using CfgGrouped128 = GemmCfg<128, 6, 2, false, true>;
 using CfgGroupedPair256 = GemmCfg<256, 6, 2, false, true, true>;
+using CfgSilu = GemmCfg<256, 4, 2, false, false, false, 1, false, true>;
+using CfgSiluPair = GemmCfg<256, 6, 2, false, false, true, 1, false, true>;
 using CfgSwap32 = GemmCfg<32, 10, 1, true, false>;
 using CfgSwap64 = GemmCfg<64, 8, 1, true, false>;
 using CfgSwap32Split = GemmCfg<32, 10, 1, true, false, false, 1, true>;
@@ -566,6 +569,44 @@ lnq_status lnq_m_grouped_fp8_gemm_contiguous(const void* a_e4m3, const float* sf
     args.tiles_q = static_cast<int>((N + 127) / 128);
     args.num_tiles = args.tiles_p * args.tiles_q;
     return launch_gemm<CfgGrouped128>(*dev, a_e4m3, M_total, b_e4m3, wrows, K, args, s);
+}
+
+lnq_status lnq_fp8_block_gemm_nt_silu_mul(const void* a_e4m3, const float* sfa, int64_t M4,
+                                          const void* b_e4m3, const float* sfb, void* h_bf16,
+                                          int64_t M, int64_t I, int64_t K, void* stream) {
+    if (M <= 0 || I <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
+    if (K % 128 != 0 || I % 128 != 0 || M > kMaxRows || 2 * I > kMaxRows || K > (int64_t{1} << 31))
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (M4 < ((M + 3) / 4) * 4 || M4 % 4 != 0) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!a_e4m3 || !sfa || !b_e4m3 || !sfb || !h_bf16) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(a_e4m3) || !aligned16(sfa) || !aligned16(b_e4m3) || !aligned4(sfb) || !aligned16(h_bf16))
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+
+    // Dense tiles of 128 outputs: the MMA's 256 columns are the outputs' 128 gate
+    // rows and their 128 up rows (I further on in the weight).
+    GemmArgs args{};
+    args.sfa = sfa;
+    args.sfb = sfb;
+    args.d = static_cast<uint16_t*>(h_bf16);
+    args.M4 = M4;
+    args.M = static_cast<int>(M);
+    args.N = static_cast<int>(I);
+    args.num_kb = static_cast<int>(K / 128);
+    args.nb = static_cast<int>(2 * I / 128);
+    args.num_groups = 1;
+    args.tiles_q = static_cast<int>(I / 128);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M > 128 && g_dense_pairs.load(std::memory_order_relaxed) != 0) {
+        args.tiles_p = static_cast<int>((M + 255) / 256);
+        args.num_tiles = args.tiles_p * args.tiles_q;
+        return launch_gemm<CfgSiluPair>(*dev, a_e4m3, M, b_e4m3, 2 * I, K, args, s);
+    }
+    args.tiles_p = static_cast<int>((M + 127) / 128);
+    args.num_tiles = args.tiles_p * args.tiles_q;
+    return launch_gemm<CfgSilu>(*dev, a_e4m3, M, b_e4m3, 2 * I, K, args, s);
 }
 
 lnq_status lnq_m_grouped_fp8_gemm_contiguous_psum(const void* a_e4m3, const float* sfa,

@@ -18,7 +18,12 @@
 //     alignment the grouped tiles run on CTA pairs as dense ones do
 //     (deepgemm-rust README, "The mk_alignment knob (MoE tile width)");
 //   * decode (M <= 64, "swap AB"): the weights fill the 128-row M slot and the
-//     few tokens the N slot, so the tensor core is not idle on padding rows.
+//     few tokens the N slot, so the tensor core is not idle on padding rows;
+//   * gate_up with SiLU.mul (SILU, dense, single CTA or pair): the weight holds I
+//     gate rows over I up rows; a tile's 256 MMA columns are 128 gate columns and
+//     the 128 up columns of the same outputs, and the epilogue stores
+//     h = silu(gate) * up (deepgemm-rust README, "What's implemented",
+//     moe_fp8_layer: grouped GEMM -> SiLU.mul -> grouped GEMM).
 //
 // Roles (warps of one CTA):
 //   warp 0      TMA producer: P and Q tiles of one 128-wide K block per stage
@@ -92,7 +97,7 @@ struct GemmArgs {
 constexpr unsigned int kStatusBadGroup = 2u;
 
 template <int BNQ_, int STAGES_, int EPI_WG_, bool SWAP_, bool GROUPED_, bool PAIR_ = false,
-          int SLICES_ = 1, bool SPLITK_ = false>
+          int SLICES_ = 1, bool SPLITK_ = false, bool SILU_ = false>
 struct GemmCfg {
     static constexpr int BNQ = BNQ_;   // MMA N (the whole pair's N for PAIR)
     static constexpr int STAGES = STAGES_;
@@ -103,6 +108,10 @@ struct GemmCfg {
     // decode only: (tile, K block) units shared in contiguous runs by all CTAs
     static constexpr bool SPLITK = SPLITK_;
     static_assert(!SPLITK || SWAP, "the K split serves the decode configuration");
+    // gate_up with SiLU.mul: a tile covers 128 outputs, i.e. 128 gate and 128 up columns
+    static constexpr bool SILU = SILU_;
+    static_assert(!SILU || (!SWAP && !GROUPED && !SPLITK && BNQ == 256 && EPI_WG_ == 2 && SLICES_ == 1),
+                  "SiLU.mul tiles are dense 128 x 256 (or 256 x 256 on pairs) with two epilogue warpgroups");
     static_assert(!(SWAP && GROUPED), "decode configuration is dense only");
     static_assert(!(PAIR && SWAP), "CTA pairs serve the dense and grouped configurations");
     static_assert(BNQ % 16 == 0 && BNQ >= 16 && BNQ <= 256, "MMA N for M=128/256");
@@ -116,6 +125,11 @@ struct GemmCfg {
     static constexpr int kPBytes = kP * kBK;
     static constexpr int kQRowsPerCta = PAIR ? BNQ / 2 : BNQ;
     static constexpr int kQBytes = kQRowsPerCta * kBK;
+    // rows of one weight TMA box: a single-CTA SiLU.mul tile loads its gate and up
+    // halves as two boxes
+    static constexpr int kQBoxRows = (PAIR || SILU) ? 128 : kQRowsPerCta;
+    // output columns per tile
+    static constexpr int kTileN = SILU ? 128 : BNQ;
     // Scale ring.  Each slot holds the scales of kScaleBatch consecutive K blocks of
     // a tile, so the epilogue waits on (and releases) a slot once per batch.  Scale
     // copies travel the load/store path and take several microseconds to land under
@@ -131,6 +145,14 @@ struct GemmCfg {
     // TMEM columns per load in the promotion (each load issued one chunk ahead)
     static constexpr int kLdCols = 32;
     static_assert(kCW % kLdCols == 0, "promotion chunks tile the thread's columns");
+    // TMEM column of the thread's promotion chunk c, from its first column: SiLU.mul
+    // threads take kCW/2 gate columns and the kCW/2 up columns 128 further on
+    __host__ __device__ static constexpr int chunk_col(int c) {
+        return SILU ? (c < kCW / kLdCols / 2 ? c * kLdCols : 128 + (c - kCW / kLdCols / 2) * kLdCols)
+                    : c * kLdCols;
+    }
+    // first TMEM column of epilogue warpgroup wg's chunks
+    __host__ __device__ static constexpr int wg_col(int wg) { return SILU ? wg * (kCW / 2) : wg * kCW; }
     static constexpr int kEpiThreads = 128 * EPI_WG;
     static constexpr int kThreads = 128 + kEpiThreads;
     // TMEM accumulators of BNQ columns each, as many as the 512 columns hold (at
@@ -212,20 +234,28 @@ struct TileCoord {
     int row_end;  // output rows from row_end on are not stored (dense and grouped tiles)
 };
 
-// Prefix-sum layout: the group whose aligned rows hold arena row r, and the end of
-// its tokens (group -1 past the last group).  Runs on a whole warp: each lane takes
-// one group of a run of 32, the run's aligned counts are summed by a warp scan, and
-// the run whose aligned rows reach past r holds the group.  A count below zero (a
-// decreasing psum) is reported and taken as zero.  Returns the first row after the
-// runs scanned (after all groups when r lies past them).
-__device__ __forceinline__ long long psum_lookup(const GemmArgs& a, int r, int& group, int& row_end) {
+// Prefix-sum layout: the tiles of TILE_M rows that hold tokens, numbered group by
+// group (group g has ceil(count_g / TILE_M) of them, from its first aligned row on).
+// Tile v's group, first arena row and end of its group's tokens; group -1 past the
+// last tile.  Numbering only the tiles with tokens keeps the pad rows of a coarse
+// alignment out of the schedule: every CTA gets its share of real tiles.  Runs on a
+// whole warp: each lane takes one group of a run of 32, the run's aligned row counts
+// and tile counts are summed by warp scans, and the run whose tiles reach past v
+// holds the group.  A count below zero (a decreasing psum) is reported and taken as
+// zero.  Returns the first row after the runs scanned (after all groups when v lies
+// past the last tile).
+template <int TILE_M>
+__device__ __forceinline__ long long psum_tile(const GemmArgs& a, int v, int& group, long long& p0,
+                                               int& row_end) {
     const int lane = static_cast<int>(threadIdx.x & 31u);
     const long long align = a.align;
     long long base = 0;   // first row of the run's first group
+    int base_tiles = 0;   // tiles of the groups before the run
     int prev_psum = 0;    // psum of the group before the run
     group = -1;
+    p0 = 0;
     row_end = 0;
-    for (int g0 = 0; g0 < a.num_groups && base <= r; g0 += 32) {
+    for (int g0 = 0; g0 < a.num_groups && base_tiles <= v; g0 += 32) {
         const int g = g0 + lane;
         const bool real = g < a.num_groups;
         const int ps = real ? __ldg(a.psum + g) : 0;
@@ -237,24 +267,34 @@ __device__ __forceinline__ long long psum_lookup(const GemmArgs& a, int r, int& 
             count = 0;
         }
         const long long padded = (count + align - 1) / align * align;
-        long long end = padded;  // inclusive scan of the aligned counts
+        const int tiles = static_cast<int>((count + TILE_M - 1) / TILE_M);
+        long long end = padded;  // inclusive scans of the aligned rows and of the tiles
+        int tend = tiles;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            const long long v = __shfl_up_sync(0xffffffffu, end, d);
-            if (lane >= d) end += v;
+            const long long x = __shfl_up_sync(0xffffffffu, end, d);
+            const int y = __shfl_up_sync(0xffffffffu, tend, d);
+            if (lane >= d) {
+                end += x;
+                tend += y;
+            }
         }
         end += base;
+        tend += base_tiles;
         const long long start = end - padded;
-        const unsigned hit = __ballot_sync(0xffffffffu, count > 0 && start <= r && r < end);
+        const int tstart = tend - tiles;
+        const unsigned hit = __ballot_sync(0xffffffffu, tiles > 0 && tstart <= v && v < tend);
         if (hit != 0u) {
             const int src = __ffs(hit) - 1;
             group = g0 + src;
+            p0 = __shfl_sync(0xffffffffu, start + static_cast<long long>(v - tstart) * TILE_M, src);
             const long long tok_end = __shfl_sync(0xffffffffu, start + count, src);
             row_end = static_cast<int>(tok_end < a.M ? tok_end : a.M);
             if (tok_end > a.M) atomicOr(a.status, kStatusBadGroup);
             break;
         }
         base = __shfl_sync(0xffffffffu, end, 31);
+        base_tiles = __shfl_sync(0xffffffffu, tend, 31);
         prev_psum = __shfl_sync(0xffffffffu, ps, 31);
     }
     return base;
@@ -282,19 +322,19 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32
         const int rows = min(a.tiles_p - first, kBand);
         const int r = t - band * band_tiles;
         c.p0 = (first + r % rows) * C::kTileM + static_cast<int>(rank) * C::kP;
-        c.q0 = (r / rows) * C::BNQ;
+        c.q0 = (r / rows) * C::kTileN;
         c.row_end = a.M;
         if constexpr (C::GROUPED) {
             if (a.psum != nullptr) {
-                // prefix-sum layout: the group is looked up at the pair's first row, so
-                // both CTAs of a pair take it (a group's aligned rows hold whole tiles)
+                // prefix-sum layout: the raster's row tile is the index among the tiles
+                // that hold tokens (the same for both CTAs of a pair); a tile that would
+                // start past the arena (groups that overrun it) is skipped
                 int g, end;
-                psum_lookup(a, c.p0 - static_cast<int>(rank) * C::kP, g, end);
-                c.group = g;
+                long long base_row;
+                psum_tile<C::kTileM>(a, c.p0 / C::kTileM, g, base_row, end);
+                c.group = base_row < a.M ? g : -1;
+                c.p0 = static_cast<int>(base_row < a.M ? base_row : 0) + static_cast<int>(rank) * C::kP;
                 c.row_end = end;
-                // a single-CTA tile of pad rows only (groups aligned to more rows than
-                // a tile) is skipped; a pair's tile always holds tokens of its group
-                if (!C::PAIR && end <= c.p0) c.group = -1;
             } else if (a.m_indices != nullptr) {
                 // contiguous: the block's group is that of its first row
                 c.group = __ldg(a.m_indices + c.p0);
@@ -348,29 +388,39 @@ template <class C, class Release>
 __device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint32_t taddr,
                                                 const float* slot, int row, int wg,
                                                 Release&& release) {
-    float2 s2;
-    if constexpr (!C::SWAP) {
-        const float s = slot[row] * slot[C::kSbOffset + (wg * C::kCW) / 128];
-        s2 = make_float2(s, s);
-    } else {
-        const float sb = slot[C::kSbOffset];
-        s2 = make_float2(sb, sb);
-    }
     // chunks of kLdCols columns, each load issued one chunk ahead of the FMAs
     constexpr int X = C::kLdCols;
     constexpr int NC = C::kCW / X;
+    float2 s2, s2_up;
+    if constexpr (C::SILU) {
+        // gate columns take the gate block's weight scale, up columns the up block's
+        const float sa = slot[row];
+        const float sg = sa * slot[C::kSbOffset];
+        const float su = sa * slot[C::kSbOffset + 1];
+        s2 = make_float2(sg, sg);
+        s2_up = make_float2(su, su);
+    } else if constexpr (!C::SWAP) {
+        const float s = slot[row] * slot[C::kSbOffset + (wg * C::kCW) / 128];
+        s2 = make_float2(s, s);
+        s2_up = s2;
+    } else {
+        const float sb = slot[C::kSbOffset];
+        s2 = make_float2(sb, sb);
+        s2_up = s2;
+    }
     uint32_t ra[X], rb[X];
-    tmem_ld_async(taddr, ra);
+    tmem_ld_async(taddr + C::chunk_col(0), ra);
     tmem_wait_ld(ra);
     if (NC == 1) release();
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
         if (c + 1 < NC) {
-            if (c & 1) tmem_ld_async(taddr + (c + 1) * X, ra);
-            else tmem_ld_async(taddr + (c + 1) * X, rb);
+            if (c & 1) tmem_ld_async(taddr + C::chunk_col(c + 1), ra);
+            else tmem_ld_async(taddr + C::chunk_col(c + 1), rb);
         }
-        if (c & 1) promote_chunk<C, X>(acc, rb, c * X, slot, s2);
-        else promote_chunk<C, X>(acc, ra, c * X, slot, s2);
+        const float2 sc = (C::SILU && c >= NC / 2) ? s2_up : s2;
+        if (c & 1) promote_chunk<C, X>(acc, rb, c * X, slot, sc);
+        else promote_chunk<C, X>(acc, ra, c * X, slot, sc);
         if (c + 1 < NC) {
             if (c & 1) tmem_wait_ld(ra);
             else tmem_wait_ld(rb);
@@ -519,12 +569,16 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         if (elect_one()) {
                             for (int s = 0; s < prefetched; ++s) {
                                 mbar_arrive_expect_tx(full_bar(s), C::kPBytes + C::kQBytes);
-                                if constexpr (C::SWAP)
+                                if constexpr (C::SWAP) {
                                     tma_load_2d(sP + s * C::kPBytes, &map_p, full_bar(s),
                                                 (sg0.kb_lo + s) * C::kBK, tc.p0);
-                                else
+                                } else {
                                     tma_load_2d(sQ + s * C::kQBytes, &map_q, full_bar(s),
                                                 (sg0.kb_lo + s) * C::kBK, tc.q0);
+                                    if constexpr (C::SILU)  // the up rows of the same outputs
+                                        tma_load_2d(sQ + s * C::kQBytes + C::kQBoxRows * C::kBK, &map_q,
+                                                    full_bar(s), (sg0.kb_lo + s) * C::kBK, tc.q0 + args.N);
+                                }
                             }
                         }
                         __syncwarp();
@@ -540,6 +594,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 if constexpr (C::SWAP) {
                     p_row = tc.p0;
                     q_row = tc.q0;
+                } else if constexpr (C::SILU) {
+                    // gate rows q0.. (and, on a pair's second CTA, the up rows I + q0..)
+                    p_row = tc.p0;
+                    q_row = tc.q0 + static_cast<int>(rank) * args.N;
                 } else {
                     p_row = tc.p0;
                     q_row = tc.group * args.N + tc.q0 + static_cast<int>(rank) * C::kSliceQRows;
@@ -580,6 +638,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                                 mbar_arrive_expect_tx(full_bar(stage), C::kPBytes + C::kQBytes);
                                 tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK, p_row);
                                 tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK, q_row);
+                                if constexpr (C::SILU && !C::PAIR)  // the up rows of the same outputs
+                                    tma_load_2d(sQ + stage * C::kQBytes + C::kQBoxRows * C::kBK, &map_q,
+                                                full_bar(stage), kb * C::kBK, q_row + args.N);
                             }
                         }
                         __syncwarp();
@@ -725,10 +786,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         constexpr int kSaLanes = C::kSaPerTile / 4;  // lanes that copy 16 bytes of sa
         if constexpr (C::GROUPED) {
             // prefix-sum layout: groups whose aligned rows run past the arena are
-            // reported once per launch (tiles past M_total are never looked up)
+            // reported once per launch (tiles that would start past it are skipped)
             if (args.psum != nullptr && blockIdx.x == 0) {
                 int g, e;
-                if (psum_lookup(args, 0x7fffffff, g, e) > args.M) atomicOr(args.status, kStatusBadGroup);
+                long long r0;
+                if (psum_tile<C::kTileM>(args, 0x7fffffff, g, r0, e) > args.M) atomicOr(args.status, kStatusBadGroup);
             }
         }
         Segment sg;
@@ -739,7 +801,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             long long a_row = (C::SWAP ? tc.q0 : tc.p0) + lane * 4;
             if (a_row > args.M4 - 4) a_row = args.M4 - 4;
             const int nb_first = C::SWAP ? tc.p0 / 128 : tc.q0 / 128;
-            const int nb_lane = min(nb_first + lane, args.nb - 1);
+            // SiLU.mul: lane 0 the gate block's scales, lane 1 the up block's (I/128 further)
+            const int nb_lane = min(C::SILU ? nb_first + lane * (args.N / 128) : nb_first + lane, args.nb - 1);
             const long long sb_row = static_cast<long long>(C::SWAP ? 0 : tc.group) * args.nb + nb_lane;
             const float* sa_src = args.sfa + a_row;
             const float* sb_src = args.sfb + sb_row * args.num_kb;
@@ -796,7 +859,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 }
                 tc_fence_after();
                 const float* slot = scale_slots + sstage * C::kScaleSlotFloats + j * C::kScaleKbFloats;
-                const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(abuf * C::BNQ + wg * C::kCW);
+                const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(abuf * C::BNQ + C::wg_col(wg));
                 // the accumulator slice and the scale slot are only read, and each arrival
                 // follows the completion of those reads: no release fence is needed (one
                 // would also wait for this warp's outstanding output stores).  The slice is
@@ -900,7 +963,26 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 }
             }
             // ---- store the tile
-            if constexpr (!C::SWAP) {
+            if constexpr (C::SILU) {
+                // h[m][q0 + wg*64 + i] = silu(gate_i) * up_i: acc[0 .. kCW/4) hold the gate
+                // columns in pairs, acc[kCW/4 ..) the up columns of the same outputs
+                const int m = tc.p0 + row;
+                const int n0 = tc.q0 + wg * (C::kCW / 2);
+                if (m < tc.row_end && n0 < args.N) {
+                    uint16_t* hrow = args.d + static_cast<long long>(m) * args.N + n0;
+#pragma unroll
+                    for (int c = 0; c < C::kCW / 16; ++c) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 g = acc[c * 4 + i];
+                            const float2 u = acc[C::kCW / 4 + c * 4 + i];
+                            w[i] = pack_bf16x2(g.x / (1.0f + expf(-g.x)) * u.x, g.y / (1.0f + expf(-g.y)) * u.y);
+                        }
+                        *reinterpret_cast<uint4*>(hrow + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            } else if constexpr (!C::SWAP) {
                 const int m = tc.p0 + row;
                 const int n0 = tc.q0 + wg * C::kCW;
                 if (args.bias != nullptr) {

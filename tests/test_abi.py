@@ -150,6 +150,21 @@ def test_psum_argument_errors(L):
     assert call(a=A16 + 1) == MISALIGNED
 
 
+def test_silu_mul_argument_errors(L):
+    f = L.lnq_fp8_block_gemm_nt_silu_mul
+
+    def call(M=256, I=256, K=512, M4=256, h=A16e, a=A16):
+        return f(a, A16b, M4, A16c, A16d, h, M, I, K, None)
+
+    assert call(M=0) == INVALID
+    assert call(h=None) == INVALID
+    assert call(I=200) == SHAPE                 # I % 128
+    assert call(K=100) == SHAPE
+    assert call(M4=252) == SHAPE                # M4 < ceil4(M)
+    assert call(h=A16e + 8) == MISALIGNED
+    assert call(a=A16 + 1) == MISALIGNED
+
+
 def test_epilogue_argument_errors(L):
     f = L.lnq_fp8_block_gemm_nt_epilogue
 
