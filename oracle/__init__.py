@@ -72,6 +72,10 @@ def _load():
         lib.oracle_m_grouped_gemm_points.restype = ctypes.c_int
         lib.oracle_m_grouped_gemm_points.argtypes = [
             P, P, P, P, P, ctypes.c_int32, I64, I64, I64, P, P, I64, P]
+        lib.oracle_quantize_ue8m0_groups.restype = ctypes.c_int
+        lib.oracle_quantize_ue8m0_groups.argtypes = [P, I64, I64, I64, P, I64, P]
+        lib.oracle_quantize_ue8m0_blocks.restype = ctypes.c_int
+        lib.oracle_quantize_ue8m0_blocks.argtypes = [P, I64, I64, P, P]
         lib.oracle_silu_mul.restype = None
         lib.oracle_silu_mul.argtypes = [P, P, I64, P]
         lib.oracle_m_grouped_gemm_psum.restype = ctypes.c_int
@@ -305,3 +309,35 @@ def gemm_nt_silu_mul_points(qa, sfa, qb, sfb, rows, cols) -> np.ndarray:
     g = gemm_nt_points(qa, sfa, qb, sfb, rows, cols)
     u = gemm_nt_points(qa, sfa, qb, sfb, rows, cols + I)
     return silu_mul(g, u)
+
+
+def quantize_ue8m0_groups(x_bf16_bits: np.ndarray):
+    """UE8M0 recipe, 1x128 activation groups of a bf16 matrix given as uint16 bits [M, K].
+
+    Returns (q uint8 [M, K], sfe uint8 [K/128, M]): each group's scale is 2^(sfe - 127),
+    the smallest power of two p with 448 p >= amax.
+    """
+    x = _c(x_bf16_bits, np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), dtype=np.uint8)
+    sfe = np.empty((K // GROUP, M), dtype=np.uint8)
+    _check(_load().oracle_quantize_ue8m0_groups(_ptr(x), M, K, K, _ptr(q), K, _ptr(sfe)),
+           "quantize_ue8m0_groups")
+    return q, sfe
+
+
+def quantize_ue8m0_blocks(w_bf16_bits: np.ndarray):
+    """UE8M0 recipe, 128x128 weight blocks: (q uint8 [N, K], sfe uint8 [ceil(N/128), K/128])."""
+    w = _c(w_bf16_bits, np.uint16)
+    N, K = w.shape
+    q = np.empty((N, K), dtype=np.uint8)
+    sfe = np.empty((-(-N // GROUP), K // GROUP), dtype=np.uint8)
+    _check(_load().oracle_quantize_ue8m0_blocks(_ptr(w), N, K, _ptr(q), _ptr(sfe)),
+           "quantize_ue8m0_blocks")
+    return q, sfe
+
+
+def ue8m0_value(sfe) -> np.ndarray:
+    """The scale 2^(b - 127) of UE8M0 bytes, as float32 (exact for b in 0..254)."""
+    b = np.asarray(sfe, dtype=np.int32)
+    return np.ldexp(np.float32(1.0), b - 127).astype(np.float32)

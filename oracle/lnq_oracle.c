@@ -47,6 +47,12 @@
  *   - SiLU.mul after a gate_up linear: deepgemm-rust README, "What's
  *     implemented", moe_fp8_layer (grouped GEMM -> SiLU.mul -> grouped GEMM);
  *     silu(x) = x / (1 + e^-x), the sigmoid-weighted linear unit.
+ *   - The UE8M0 recipe: the same groups and blocks with power-of-two scales
+ *     stored as 8-bit exponents (value 2^(e - 127)), consumed by the
+ *     tensor core's block-scaled MMA: deepgemm-rust README, "Blackwell-native
+ *     FP4/FP8 (SM100a, tcgen05)" (UE8M0 power-of-two scales, block-scaled
+ *     MMA) and "What's implemented" (gran-128 recipe on either side; FP32
+ *     scales transformed into packed UE8M0).
  *   - E4M3 round-to-nearest-even with saturation at 448, scale = amax/448:
  *     the benchmark spec's numerics (the pages never print 448; the encoder
  *     below is written from the OCP FP8 E4M3 format definition: bias 7,
@@ -63,6 +69,9 @@
  *   - pad scale entries (rows M..M4-1) are written as 0.0f;
  *   - grouped rows whose group id is negative contribute nothing and their
  *     output row is left untouched;
+ *   - UE8M0 scale of a group or block: the smallest power of two p with
+ *     448 * p >= amax (so no code saturates), exponent clamped to [-127, 127];
+ *     an all-zero group gets p = 1 (byte 127); codes are the E4M3 RNE of x / p;
  *   - SiLU.mul: the gate_up weight stacks the I gate rows over the I up rows,
  *     and h[m][j] = silu(D[m][j]) * D[m][I + j] is taken of the product itself
  *     (before any BF16 rounding of D).
@@ -586,4 +595,93 @@ void oracle_silu_mul(const double* g, const double* u, int64_t n, double* h)
     int64_t i;
     for (i = 0; i < n; ++i)
         h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
+}
+
+/* UE8M0 recipe: the exponent e of the smallest power of two with 448 * 2^e >= amax,
+ * clamped to [-127, 127]; 0 for amax == 0.  Every comparison is exact in double. */
+static int ue8m0_exponent(float amax)
+{
+    int e;
+    if (!(amax > 0.0f))
+        return 0;
+    (void)frexp((double)amax, &e);     /* amax < 2^e, so 448 * 2^(e - 8) > amax */
+    e -= 10;
+    while (ldexp(448.0, e) < (double)amax)
+        ++e;
+    if (e < -127)
+        e = -127;
+    if (e > 127)
+        e = 127;
+    return e;
+}
+
+/* E4M3 code of x / 2^e (the division by a power of two is exact). */
+static uint8_t quantize_pow2(float x, int e)
+{
+    return oracle_e4m3_encode((float)ldexp((double)x, -e));
+}
+
+/* UE8M0 activation quantization, 1 x 128 groups.
+ *   x    bf16 [M][ld_x];  q  E4M3 [M][ld_q];
+ *   sfe  uint8 [K/128][M], sfe[g*M + m] = e + 127 of row m's group g. */
+int oracle_quantize_ue8m0_groups(const uint16_t* x, int64_t M, int64_t K, int64_t ld_x,
+                                 uint8_t* q, int64_t ld_q, uint8_t* sfe)
+{
+    int64_t G, m;
+    if (M <= 0 || K <= 0 || K % ORACLE_GROUP != 0 || ld_x < K || ld_q < K)
+        return -1;
+    G = K / ORACLE_GROUP;
+#pragma omp parallel for schedule(static)
+    for (m = 0; m < M; ++m) {
+        int64_t g, k;
+        for (g = 0; g < G; ++g) {
+            float amax = 0.0f;
+            int e;
+            for (k = 0; k < ORACLE_GROUP; ++k) {
+                float v = fabsf(bf16_bits_to_float(x[m * ld_x + g * ORACLE_GROUP + k]));
+                if (v > amax)
+                    amax = v;
+            }
+            e = ue8m0_exponent(amax);
+            sfe[g * M + m] = (uint8_t)(e + 127);
+            for (k = 0; k < ORACLE_GROUP; ++k) {
+                int64_t col = g * ORACLE_GROUP + k;
+                q[m * ld_q + col] = quantize_pow2(bf16_bits_to_float(x[m * ld_x + col]), e);
+            }
+        }
+    }
+    return 0;
+}
+
+/* UE8M0 weight quantization, 128 x 128 blocks (a ragged last row block takes its
+ * amax over the rows that exist).  sfe uint8 [ceil(N/128)][K/128]. */
+int oracle_quantize_ue8m0_blocks(const uint16_t* w, int64_t N, int64_t K, uint8_t* q, uint8_t* sfe)
+{
+    int64_t NB, KB, blk;
+    if (N <= 0 || K <= 0 || K % ORACLE_GROUP != 0)
+        return -1;
+    NB = (N + ORACLE_GROUP - 1) / ORACLE_GROUP;
+    KB = K / ORACLE_GROUP;
+#pragma omp parallel for schedule(static)
+    for (blk = 0; blk < NB * KB; ++blk) {
+        int64_t nb = blk / KB, kb = blk % KB;
+        int64_t n0 = nb * ORACLE_GROUP, n1 = n0 + ORACLE_GROUP;
+        int64_t n, k;
+        float amax = 0.0f;
+        int e;
+        if (n1 > N)
+            n1 = N;
+        for (n = n0; n < n1; ++n)
+            for (k = kb * ORACLE_GROUP; k < (kb + 1) * ORACLE_GROUP; ++k) {
+                float v = fabsf(bf16_bits_to_float(w[n * K + k]));
+                if (v > amax)
+                    amax = v;
+            }
+        e = ue8m0_exponent(amax);
+        sfe[nb * KB + kb] = (uint8_t)(e + 127);
+        for (n = n0; n < n1; ++n)
+            for (k = kb * ORACLE_GROUP; k < (kb + 1) * ORACLE_GROUP; ++k)
+                q[n * K + k] = quantize_pow2(bf16_bits_to_float(w[n * K + k]), e);
+    }
+    return 0;
 }
