@@ -191,13 +191,19 @@ class ClockSampler:
 class Linear:
     """One dense linear: bf16 activations resident on the device, weights pre-quantized."""
 
-    def __init__(self, cfg, dev, split: bool = False, fp8_out: bool = False, silu: bool = False):
+    def __init__(self, cfg, dev, split: bool = False, fp8_out: bool = False, silu: bool = False,
+                 recipe: str = "fp32"):
         import moe_grouped_gemm_quantize_b200 as lnq
         from moe_grouped_gemm_quantize_b200 import synthetic
         self.cfg = cfg
         a, w = synthetic.make_linear_inputs(cfg)
         self.x = a.to(dev)
-        self.wq, self.ws = lnq.quantize_weights(w.to(dev))
+        # UE8M0 recipe: power-of-two scales applied by the tensor core (no promotion)
+        self.ue8m0 = recipe == "ue8m0"
+        if self.ue8m0:
+            self.wq, self.ws = lnq.quantize_weights_ue8m0(w.to(dev))
+        else:
+            self.wq, self.ws = lnq.quantize_weights(w.to(dev))
         del w
         M, N, K = cfg.M, cfg.N, cfg.K
         self.M4 = lnq.ceil4(M)
@@ -213,7 +219,13 @@ class Linear:
         self.host_x = self.x.cpu().pin_memory()
         self.host_d = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
         # decode shapes: a workspace lets every SM share the weight stream (K split)
-        self.work = lnq.gemm_workspace(M, N, K, dev) if split else None
+        self.work = lnq.gemm_workspace(M, N, K, dev) if split and not self.ue8m0 else None
+        if self.ue8m0:
+            Mp, Np = -(-M // 128) * 128, -(-N // 128) * 128
+            self.sfa = lnq.ue8m0_atoms(M, K, dev)
+            self.gemm_bytes = M * K + 4 * (K // 128) * Mp + N * K + 4 * (K // 128) * Np + 2 * M * N
+            self.quant_bytes = 2 * M * K + M * K + 4 * (K // 128) * Mp
+            fp8_out = silu = False
         # fused epilogue: the output quantized (E4M3 + 1x128 scales) for a next linear
         self.fp8_out = fp8_out and M > 64 and N % 128 == 0 and N >= 256
         if self.fp8_out:
@@ -247,6 +259,12 @@ class Linear:
         P = ctypes.c_void_p
         c = self.cfg
         s = P(stream_ptr)
+        if self.ue8m0:
+            qargs = (P(self.x.data_ptr()), c.M, c.K, self.x.stride(0), P(self.q.data_ptr()), c.K,
+                     P(self.sfa.data_ptr()), s)
+            margs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), P(self.wq.data_ptr()), P(self.ws.data_ptr()),
+                     P(self.d.data_ptr()), c.M, c.N, c.K, s)
+            return (L.lnq_quantize_ue8m0_groups, qargs), (L.lnq_mx_block_gemm_nt, margs)
         qargs = (P(self.x.data_ptr()), c.M, c.K, self.x.stride(0), P(self.q.data_ptr()), c.K,
                  P(self.sfa.data_ptr()), self.M4, s)
         gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), self.M4, P(self.wq.data_ptr()),
@@ -430,7 +448,7 @@ def run_ours(args, world, rank, local):
     units = [Grouped(c, dev) if kind == "grouped" else Grouped(c, dev, alignment=256) if kind == "psum"
              else Masked(c, dev) if kind == "masked"
              else Linear(c, dev, split=args.split, fp8_out=args.epilogue == "fp8",
-                         silu=args.epilogue == "silu") for c in cfgs]
+                         silu=args.epilogue == "silu", recipe=args.recipe) for c in cfgs]
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
     calls = [u.calls(sp) for u in units]
@@ -548,9 +566,11 @@ def run_ours(args, world, rank, local):
                 "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4)}
         peak_note = (f"dense FP8 = {FP8_OVER_BF16:g} x bf16 cuBLAS burst {peaks['bf16_tflops']} "
                      f"TFLOP/s ({peak_src})")
-    traffic = recorded_traffic("k_fp8_block_gemm", args.workload)
+    ue8m0 = any(getattr(u, "ue8m0", False) for u in units)
+    kernel_name = "k_mx_block_gemm" if ue8m0 else "k_fp8_block_gemm"
+    traffic = recorded_traffic(kernel_name, args.workload)
     roof["traffic"] = traffic
-    roof["kernel"] = "k_fp8_block_gemm"
+    roof["kernel"] = kernel_name
     roof["peak_source"] = peak_note
     roof["algorithmic_per_launch"] = ({"bytes": [int(u.gemm_bytes) for u in units]}
                                       if is_hbm_bound(args.workload)
@@ -568,7 +588,8 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out",
+        "dtype": ("e4m3 x e4m3 with UE8M0 block scales -> f32 accumulate, bf16 out" if ue8m0
+                  else "e4m3 x e4m3 -> f32 accumulate, bf16 out"),
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, bf16)",
         "config": {"workload": args.workload, "desc": WORKLOAD_DESC[args.workload],
                    "dense_cta_pairs": args.cta_pairs,
@@ -576,8 +597,11 @@ def run_ours(args, world, rank, local):
                    "weight_prefetch": not args.no_weight_prefetch,
                    "decode_k_split": args.split and any(getattr(u, "work", None) is not None
                                                          for u in units),
-                   "epilogue": "fp8 output (E4M3 + 1x128 scales)" if any(getattr(u, "fp8_out", False)
-                                                                         for u in units) else "bf16 output",
+                   "epilogue": ("fp8 output (E4M3 + 1x128 scales)" if any(getattr(u, "fp8_out", False) for u in units)
+                                else "gate_up with SiLU.mul (bf16 h)" if any(getattr(u, "silu", False) for u in units)
+                                else "bf16 output"),
+                   "recipe": ("UE8M0 power-of-two scales in the tensor core" if ue8m0
+                              else "FP32 scales, per-128-K-block promotion"),
                    "parallelism": f"replicas x{world} (independent tokens per rank)",
                    "l2": "working set per step > 126 MB L2; no extra flush"},
         "roofline": roof,
@@ -751,6 +775,9 @@ def main():
                          "per CTA at N = 12288 on B200)")
     ap.add_argument("--no-weight-prefetch", action="store_true",
                     help="GEMMs wait for the previous kernel before streaming weights")
+    ap.add_argument("--recipe", choices=["fp32", "ue8m0"], default="fp32",
+                    help="dense workloads: FP32 scales with promotion (the default), or UE8M0 power-of-two "
+                         "scales applied by the block-scaled MMA")
     ap.add_argument("--grouped-cta-pairs", type=int, default=0, choices=[0, 1],
                     help="moe_psum: 256x256 tiles on CTA pairs (1) or 128-row tiles (0)")
     ap.add_argument("--cta-pairs", type=int, default=1, choices=[0, 1, 2],

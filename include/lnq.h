@@ -319,6 +319,43 @@ lnq_status lnq_m_grouped_fp8_gemm_masked(const void* a_e4m3, const float* sfa, c
                                          int32_t num_groups, int64_t M_max, int64_t expected_m,
                                          void* d_bf16, int64_t N, int64_t K, void* stream);
 
+/*
+ * UE8M0 recipe (deepgemm-rust README, "Blackwell-native FP4/FP8 (SM100a,
+ * tcgen05)": UE8M0 power-of-two scales copied into tensor memory and consumed
+ * by the block-scaled MMA; "What's implemented": gran-128 on either side).
+ * The same 1 x 128 activation groups and 128 x 128 weight blocks as the
+ * FP32-scale recipe; each scale is the smallest power of two p with
+ * 448 p >= amax (no code saturates; an all-zero group takes p = 1), stored as
+ * the byte e + 127 of p = 2^e, e clamped to [-127, 127].  Codes are the E4M3
+ * round-to-nearest-even of x / p.
+ *
+ * Scale atoms: for each K block kb and 128-row block rb, 128 uint32 words; row
+ * r = r0 + 32 r1 of the block (r0 < 32, r1 < 4) owns word 4 r0 + r1, whose low
+ * byte is the row's exponent byte (the other bytes 0).  Each atom is 512
+ * contiguous bytes, the layout the tensor core's scale copy reads.
+ *
+ * lnq_quantize_ue8m0_groups: x bf16 [M][ld_x] -> q E4M3 [M][ld_q] and
+ *   sfa_atoms uint32 [K/128][ceil(M/128)][128] (rows M .. of the last block get
+ *   p = 1).  Requires K % 128 == 0, ld_x % 8 == 0, ld_q % 16 == 0, pointers
+ *   16-byte aligned.
+ * lnq_quantize_ue8m0_blocks: w bf16 [N][K] -> q E4M3 [N][K] and sfb_atoms uint32
+ *   [K/128][ceil(N/128)][128], every row of a block carrying the block's byte.
+ *   Requires K % 128 == 0, pointers 16-byte aligned.
+ * lnq_mx_block_gemm_nt: D[m][n] = bf16( sum_k a[m][k] 2^ea[m][k/128] *
+ *   b[n][k] 2^eb[n/128][k/128] ), the scales applied by the tensor core
+ *   (tcgen05.mma kind::mxf8f6f4.block_scale) and the sum accumulated in FP32
+ *   over the whole K range.  a_e4m3 [M][K], b_e4m3 [N][K] (K-major), d_bf16
+ *   [M][N] fully overwritten.  Requires N % 16 == 0, K % 128 == 0, pointers
+ *   16-byte aligned.
+ */
+lnq_status lnq_quantize_ue8m0_groups(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, void* q_e4m3,
+                                     int64_t ld_q, void* sfa_atoms, void* stream);
+lnq_status lnq_quantize_ue8m0_blocks(const void* w_bf16, int64_t N, int64_t K, void* q_e4m3, void* sfb_atoms,
+                                     void* stream);
+lnq_status lnq_mx_block_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                const void* sfb_atoms, void* d_bf16, int64_t M, int64_t N, int64_t K,
+                                void* stream);
+
 /* Static text for a status code. */
 const char* lnq_status_string(lnq_status status);
 

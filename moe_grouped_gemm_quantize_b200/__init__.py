@@ -28,7 +28,8 @@ __all__ = [
     "LnqError", "library_path", "lib",
     "lnq_quantize_fp8_groups", "lnq_quantize_fp8_blocks", "lnq_fp8_block_gemm_nt",
     "lnq_m_grouped_fp8_gemm_contiguous", "lnq_m_grouped_fp8_gemm_contiguous_psum",
-    "lnq_fp8_block_gemm_nt_silu_mul",
+    "lnq_fp8_block_gemm_nt_silu_mul", "lnq_mx_block_gemm_nt", "quantize_activations_ue8m0",
+    "quantize_weights_ue8m0", "ue8m0_atoms",
     "lnq_m_grouped_fp8_gemm_masked", "lnq_get_last_device_error", "lnq_status_string",
     "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs",
     "lnq_set_weight_prefetch",
@@ -82,6 +83,9 @@ def lib() -> ctypes.CDLL:
             "lnq_m_grouped_fp8_gemm_masked": [P, P, P, P, P, I32, I64, I64, P, I64, I64, P],
             "lnq_m_grouped_fp8_gemm_contiguous_psum": [P, P, P, P, P, I32, I64, P, I64, I64, I64, P],
             "lnq_fp8_block_gemm_nt_silu_mul": [P, P, I64, P, P, P, I64, I64, I64, P],
+            "lnq_quantize_ue8m0_groups": [P, I64, I64, I64, P, I64, P, P],
+            "lnq_quantize_ue8m0_blocks": [P, I64, I64, P, P, P],
+            "lnq_mx_block_gemm_nt": [P, P, P, P, P, I64, I64, I64, P],
             "lnq_get_last_device_error": [P],
             "lnq_selftest_wait_timeout": [I64, P],
         }
@@ -314,6 +318,53 @@ def lnq_fp8_block_gemm_nt_silu_mul(a: torch.Tensor, sfa: torch.Tensor, b: torch.
     _check(lib().lnq_fp8_block_gemm_nt_silu_mul(_ptr(a), _ptr(sfa), sfa.shape[1], _ptr(b), _ptr(sfb), _ptr(h),
                                                 M, I, K, _stream(stream)),
            "lnq_fp8_block_gemm_nt_silu_mul")
+
+
+def ue8m0_atoms(rows: int, K: int, device) -> torch.Tensor:
+    """Scale-atom storage of the UE8M0 recipe: uint32-valued int32 [K/128, ceil(rows/128)*128]."""
+    return torch.empty((K // 128, -(-rows // 128) * 128), dtype=torch.int32, device=device)
+
+
+def quantize_activations_ue8m0(x: torch.Tensor, stream=None):
+    """UE8M0 recipe, 1x128 groups: (q e4m3 [M, K], scale atoms int32 [K/128, ceil(M/128)*128])."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise TypeError("x must be a row-major bf16 matrix")
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    sf = ue8m0_atoms(M, K, x.device)
+    _check(lib().lnq_quantize_ue8m0_groups(_ptr(x), M, K, x.stride(0), _ptr(q), K, _ptr(sf), _stream(stream)),
+           "lnq_quantize_ue8m0_groups")
+    return q, sf
+
+
+def quantize_weights_ue8m0(w: torch.Tensor, stream=None):
+    """UE8M0 recipe, 128x128 blocks: (q e4m3 [N, K], scale atoms int32 [K/128, ceil(N/128)*128])."""
+    if w.dtype != torch.bfloat16 or w.dim() != 2 or not w.is_contiguous():
+        raise TypeError("w must be a contiguous bf16 matrix")
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
+    sf = ue8m0_atoms(N, K, w.device)
+    _check(lib().lnq_quantize_ue8m0_blocks(_ptr(w), N, K, _ptr(q), _ptr(sf), _stream(stream)),
+           "lnq_quantize_ue8m0_blocks")
+    return q, sf
+
+
+def lnq_mx_block_gemm_nt(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                         d: torch.Tensor, stream=None) -> None:
+    """UE8M0 recipe GEMM: a e4m3 [M, K], b e4m3 [N, K], their scale atoms, d bf16 [M, N]."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.int32 or sfb.dtype != torch.int32 or \
+            d.dtype != torch.bfloat16:
+        raise TypeError("a, b e4m3; sfa, sfb int32 scale atoms; d bf16")
+    for t in (a, sfa, b, sfb, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K or tuple(d.shape) != (M, N) or tuple(sfa.shape) != (K // 128, -(-M // 128) * 128) or \
+            tuple(sfb.shape) != (K // 128, -(-N // 128) * 128):
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_mx_block_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream(stream)),
+           "lnq_mx_block_gemm_nt")
 
 
 def lnq_m_grouped_fp8_gemm_contiguous_psum(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,

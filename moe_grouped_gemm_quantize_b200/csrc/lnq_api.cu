@@ -14,6 +14,7 @@
 
 #include "lnq.h"
 #include "lnq_gemm.cuh"
+#include "lnq_mx.cuh"
 #include "lnq_ptx.cuh"
 #include "lnq_quantize.cuh"
 
@@ -327,6 +328,112 @@ lnq_status lnq_quantize_fp8_blocks(const void* w_bf16, int64_t N, int64_t K, voi
     dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>(K / 128));
     k_quantize_blocks<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint16_t*>(w_bf16), N, K, static_cast<uint8_t*>(q_e4m3), sfb);
+    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- UE8M0 recipe
+
+lnq_status lnq_quantize_ue8m0_groups(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, void* q_e4m3,
+                                     int64_t ld_q, void* sfa_atoms, void* stream) {
+    if (M <= 0 || K <= 0 || ld_x < K || ld_q < K) return LNQ_ERR_INVALID_ARG;
+    if (K % 128 != 0 || M > kMaxRows || K > (int64_t{1} << 31)) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!x_bf16 || !q_e4m3 || !sfa_atoms) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(q_e4m3) || !aligned16(sfa_atoms) || ld_x % 8 != 0 || ld_q % 16 != 0)
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    const int64_t Mpad = (M + 127) / 128 * 128;
+    const int64_t units = Mpad * (K / 128);
+    const int64_t want = (units + 15) / 16;  // 8 warps of two groups per CTA
+    const int grid = static_cast<int>(want < 4 * dev->sm_count ? want : 4 * dev->sm_count);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_quantize_ue8m0_groups, static_cast<const uint16_t*>(x_bf16), static_cast<int>(M),
+                           static_cast<int>(K), static_cast<long long>(ld_x), static_cast<uint8_t*>(q_e4m3),
+                           static_cast<long long>(ld_q), static_cast<uint32_t*>(sfa_atoms),
+                           static_cast<int>(Mpad)) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+lnq_status lnq_quantize_ue8m0_blocks(const void* w_bf16, int64_t N, int64_t K, void* q_e4m3, void* sfb_atoms,
+                                     void* stream) {
+    if (N <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N > kMaxRows || K > (int64_t{1} << 31) || ((N + 127) / 128) * (K / 128) > INT32_MAX)
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!w_bf16 || !q_e4m3 || !sfb_atoms) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(w_bf16) || !aligned16(q_e4m3) || !aligned16(sfb_atoms)) return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    const int nblocks = static_cast<int>((N + 127) / 128);
+    k_quantize_ue8m0_blocks<<<static_cast<unsigned>(nblocks * (K / 128)), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(w_bf16), static_cast<int>(N), static_cast<int>(K), static_cast<uint8_t*>(q_e4m3),
+        static_cast<uint32_t*>(sfb_atoms), nblocks);
+    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+lnq_status lnq_mx_block_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                const void* sfb_atoms, void* d_bf16, int64_t M, int64_t N, int64_t K,
+                                void* stream) {
+    using C = MxCfg<4>;
+    if (M <= 0 || N <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N % 16 != 0 || M > kMaxRows || N > kMaxRows || K > (int64_t{1} << 31))
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!a_e4m3 || !sfa_atoms || !b_e4m3 || !sfb_atoms || !d_bf16) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(a_e4m3) || !aligned16(sfa_atoms) || !aligned16(b_e4m3) || !aligned16(sfb_atoms) ||
+        !aligned16(d_bf16))
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    CUtensorMap map_a, map_b;
+    st = encode_e4m3_map(&map_a, a_e4m3, M, K, 128);
+    if (st == LNQ_OK) st = encode_e4m3_map(&map_b, b_e4m3, N, K, 256);
+    if (st != LNQ_OK) return st;
+    static bool attr_set[kMaxDevices] = {};
+    int devno = 0;
+    cudaGetDevice(&devno);
+    if (!attr_set[devno]) {
+        if (cudaFuncSetAttribute(k_mx_block_gemm<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+            cudaSuccess)
+            return LNQ_ERR_CUDA;
+        attr_set[devno] = true;
+    }
+    MxArgs args{};
+    args.sfa = static_cast<const uint32_t*>(sfa_atoms);
+    args.sfb = static_cast<const uint32_t*>(sfb_atoms);
+    args.d = static_cast<uint16_t*>(d_bf16);
+    args.status = dev->status;
+    args.timeout_ns = kDefaultTimeoutNs;
+    args.M = static_cast<int>(M);
+    args.N = static_cast<int>(N);
+    args.num_kb = static_cast<int>(K / 128);
+    args.mblocks = static_cast<int>((M + 127) / 128);
+    args.nblocks = static_cast<int>((N + 127) / 128);
+    args.tiles_p = args.mblocks;
+    args.tiles_q = static_cast<int>((N + 255) / 256);
+    args.num_tiles = args.tiles_p * args.tiles_q;
+    const int grid = args.num_tiles < dev->sm_count ? args.num_tiles : dev->sm_count;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4>, map_a, map_b, args) != cudaSuccess) return LNQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
 }
 

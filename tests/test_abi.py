@@ -165,6 +165,24 @@ def test_silu_mul_argument_errors(L):
     assert call(a=A16 + 1) == MISALIGNED
 
 
+def test_ue8m0_argument_errors(L):
+    q = L.lnq_quantize_ue8m0_groups
+    assert q(A16, 0, 128, 128, A16b, 128, A16c, None) == INVALID
+    assert q(A16, 4, 256, 128, A16b, 256, A16c, None) == INVALID      # ld_x < K
+    assert q(A16, 4, 200, 256, A16b, 256, A16c, None) == SHAPE        # K % 128
+    assert q(A16, 4, 128, 132, A16b, 128, A16c, None) == MISALIGNED   # ld_x % 8
+    assert q(A16, 4, 128, 128, A16b, 128, A16c + 4, None) == MISALIGNED
+    b = L.lnq_quantize_ue8m0_blocks
+    assert b(A16, 0, 128, A16b, A16c, None) == INVALID
+    assert b(A16, 4, 100, A16b, A16c, None) == SHAPE
+    assert b(A16, 4, 128, A16b, None, None) == INVALID
+    g = L.lnq_mx_block_gemm_nt
+    assert g(A16, A16b, A16c, A16d, A16e, 0, 256, 128, None) == INVALID
+    assert g(A16, A16b, A16c, A16d, A16e, 8, 20, 128, None) == SHAPE   # N % 16
+    assert g(A16, A16b, A16c, A16d, A16e, 8, 256, 100, None) == SHAPE  # K % 128
+    assert g(A16, A16b + 4, A16c, A16d, A16e, 8, 256, 128, None) == MISALIGNED
+
+
 def test_epilogue_argument_errors(L):
     f = L.lnq_fp8_block_gemm_nt_epilogue
 
