@@ -48,6 +48,7 @@ FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 KERNEL_SOURCES = ["moe_grouped_gemm_quantize_b200/csrc/lnq_gemm.cuh",
                   "moe_grouped_gemm_quantize_b200/csrc/lnq_ptx.cuh",
                   "moe_grouped_gemm_quantize_b200/csrc/lnq_quantize.cuh",
+                  "moe_grouped_gemm_quantize_b200/csrc/lnq_mx.cuh",
                   "moe_grouped_gemm_quantize_b200/csrc/lnq_api.cu"]
 
 
