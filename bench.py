@@ -290,15 +290,20 @@ class Grouped:
     by per-row group ids (128-row alignment) or, with `alignment` set, by the prefix
     sums of the group sizes (group starts aligned to that many rows)."""
 
-    def __init__(self, cfg, dev, alignment=None):
+    def __init__(self, cfg, dev, alignment=None, recipe: str = "fp32"):
         import moe_grouped_gemm_quantize_b200 as lnq
         from moe_grouped_gemm_quantize_b200 import synthetic
         self.cfg = cfg
         self.alignment = alignment
+        # UE8M0 recipe (group-id layout only): power-of-two scales applied by the tensor core
+        self.ue8m0 = recipe == "ue8m0" and alignment is None
         a, w, m_indices, sizes = synthetic.make_moe_inputs(cfg, alignment=alignment or 128)
         self.M = a.shape[0]
         self.x = a.to(dev)
-        self.wq, self.ws = lnq.quantize_weights_grouped(w.to(dev), cfg.groups)
+        if self.ue8m0:
+            self.wq, self.ws = lnq.quantize_weights_ue8m0(w.to(dev))
+        else:
+            self.wq, self.ws = lnq.quantize_weights_grouped(w.to(dev), cfg.groups)
         del w
         if alignment is None:
             self.mi = torch.from_numpy(m_indices).to(dev)
@@ -313,6 +318,9 @@ class Grouped:
                            + 4 * G * (-(-N // 128)) * (K // 128) + 2 * self.M * N
                            + 4 * (self.M if alignment is None else G))
         self.quant_bytes = 3 * self.M * K + 4 * (K // 128) * self.M
+        if self.ue8m0:
+            self.sfa = lnq.ue8m0_atoms(self.M, K, dev)
+            self.gemm_bytes += 4 * (K // 128) * G * N - 4 * G * (-(-N // 128)) * (K // 128)
         self.h2d_bytes = 2 * self.M * K
         self.d2h_bytes = 2 * self.M * N
         self.host_x = self.x.cpu().pin_memory()
@@ -328,6 +336,11 @@ class Grouped:
         P = ctypes.c_void_p
         c = self.cfg
         s = P(stream_ptr)
+        if self.ue8m0:
+            qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K, P(self.sfa.data_ptr()), s)
+            gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), P(self.wq.data_ptr()), P(self.ws.data_ptr()),
+                     P(self.mi.data_ptr()), c.groups, P(self.d.data_ptr()), self.M, c.N, c.K, s)
+            return (L.lnq_quantize_ue8m0_groups, qargs), (L.lnq_m_grouped_mx_gemm_contiguous, gargs)
         qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K,
                  P(self.sfa.data_ptr()), self.M, s)
         if self.alignment is not None:
@@ -446,7 +459,7 @@ def run_ours(args, world, rank, local):
     lnq.lnq_set_weight_prefetch(not args.no_weight_prefetch)
 
     cfgs, kind = workload_units(args.workload)
-    units = [Grouped(c, dev) if kind == "grouped" else Grouped(c, dev, alignment=256) if kind == "psum"
+    units = [Grouped(c, dev, recipe=args.recipe) if kind == "grouped" else Grouped(c, dev, alignment=256) if kind == "psum"
              else Masked(c, dev) if kind == "masked"
              else Linear(c, dev, split=args.split, fp8_out=args.epilogue == "fp8",
                          silu=args.epilogue == "silu", recipe=args.recipe) for c in cfgs]
@@ -777,8 +790,8 @@ def main():
     ap.add_argument("--no-weight-prefetch", action="store_true",
                     help="GEMMs wait for the previous kernel before streaming weights")
     ap.add_argument("--recipe", choices=["fp32", "ue8m0"], default="fp32",
-                    help="dense workloads: FP32 scales with promotion (the default), or UE8M0 power-of-two "
-                         "scales applied by the block-scaled MMA")
+                    help="dense and moe workloads: FP32 scales with promotion (the default), or UE8M0 "
+                         "power-of-two scales applied by the block-scaled MMA")
     ap.add_argument("--grouped-cta-pairs", type=int, default=0, choices=[0, 1],
                     help="moe_psum: 256x256 tiles on CTA pairs (1) or 128-row tiles (0)")
     ap.add_argument("--cta-pairs", type=int, default=1, choices=[0, 1, 2],

@@ -356,6 +356,25 @@ lnq_status lnq_mx_block_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const
                                 const void* sfb_atoms, void* d_bf16, int64_t M, int64_t N, int64_t K,
                                 void* stream);
 
+/*
+ * lnq_mx_block_gemm_nt for the M-grouped contiguous MoE layout (deepgemm-rust
+ * README, "Grouped (contiguous) MoE GEMM"): each 128-row block of the A arena
+ * takes the weights of the group named by its first row's id, as in
+ * lnq_m_grouped_fp8_gemm_contiguous.
+ *   a_e4m3 [M_total][K], sfa_atoms from lnq_quantize_ue8m0_groups over M_total rows;
+ *   b_e4m3 [num_groups*N][K], sfb_atoms from lnq_quantize_ue8m0_blocks over all
+ *   num_groups*N rows (N % 128 == 0, so no weight block spans two groups);
+ *   m_indices int32 [M_total]: a block whose first id is negative is skipped (its
+ *   rows of D untouched); pad rows inside a block are computed with the block's
+ *   group and their rows of D are unspecified; an id >= num_groups skips the
+ *   block and is reported by lnq_get_last_device_error as LNQ_ERR_INVALID_ARG.
+ *   Requires M_total % 128 == 0, N % 128 == 0, K % 128 == 0, m_indices 4-byte
+ *   aligned, the other pointers 16-byte aligned.
+ */
+lnq_status lnq_m_grouped_mx_gemm_contiguous(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                            const void* sfb_atoms, const int32_t* m_indices, int32_t num_groups,
+                                            void* d_bf16, int64_t M_total, int64_t N, int64_t K, void* stream);
+
 /* Static text for a status code. */
 const char* lnq_status_string(lnq_status status);
 

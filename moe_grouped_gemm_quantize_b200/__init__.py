@@ -28,7 +28,7 @@ __all__ = [
     "LnqError", "library_path", "lib",
     "lnq_quantize_fp8_groups", "lnq_quantize_fp8_blocks", "lnq_fp8_block_gemm_nt",
     "lnq_m_grouped_fp8_gemm_contiguous", "lnq_m_grouped_fp8_gemm_contiguous_psum",
-    "lnq_fp8_block_gemm_nt_silu_mul", "lnq_mx_block_gemm_nt", "quantize_activations_ue8m0",
+    "lnq_fp8_block_gemm_nt_silu_mul", "lnq_mx_block_gemm_nt", "lnq_m_grouped_mx_gemm_contiguous", "quantize_activations_ue8m0",
     "quantize_weights_ue8m0", "ue8m0_atoms",
     "lnq_m_grouped_fp8_gemm_masked", "lnq_get_last_device_error", "lnq_status_string",
     "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs",
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "lnq_quantize_ue8m0_groups": [P, I64, I64, I64, P, I64, P, P],
             "lnq_quantize_ue8m0_blocks": [P, I64, I64, P, P, P],
             "lnq_mx_block_gemm_nt": [P, P, P, P, P, I64, I64, I64, P],
+            "lnq_m_grouped_mx_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
             "lnq_get_last_device_error": [P],
             "lnq_selftest_wait_timeout": [I64, P],
         }
@@ -365,6 +366,29 @@ def lnq_mx_block_gemm_nt(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sf
         raise ValueError("inconsistent shapes")
     _check(lib().lnq_mx_block_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream(stream)),
            "lnq_mx_block_gemm_nt")
+
+
+def lnq_m_grouped_mx_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                                     m_indices: torch.Tensor, num_groups: int, d: torch.Tensor,
+                                     stream=None) -> None:
+    """UE8M0 recipe, M-grouped contiguous: a e4m3 [M_total, K] and its scale atoms, b e4m3 [G*N, K]
+    and its scale atoms, m_indices int32 [M_total], d bf16 [M_total, N]."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.int32 or sfb.dtype != torch.int32 or \
+            d.dtype != torch.bfloat16 or m_indices.dtype != torch.int32:
+        raise TypeError("a, b e4m3; sfa, sfb int32 scale atoms; m_indices int32; d bf16")
+    for t in (a, sfa, b, sfb, m_indices, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    M_total, K = a.shape
+    G = int(num_groups)
+    N = d.shape[1]
+    if b.shape[0] != G * N or b.shape[1] != K or d.shape[0] != M_total or m_indices.shape[0] != M_total or \
+            tuple(sfa.shape) != (K // 128, -(-M_total // 128) * 128) or \
+            tuple(sfb.shape) != (K // 128, -(-G * N // 128) * 128):
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_m_grouped_mx_gemm_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(m_indices), G,
+                                                  _ptr(d), M_total, N, K, _stream(stream)),
+           "lnq_m_grouped_mx_gemm_contiguous")
 
 
 def lnq_m_grouped_fp8_gemm_contiguous_psum(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,

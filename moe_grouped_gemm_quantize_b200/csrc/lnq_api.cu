@@ -716,6 +716,66 @@ lnq_status lnq_fp8_block_gemm_nt_silu_mul(const void* a_e4m3, const float* sfa, 
     return launch_gemm<CfgSilu>(*dev, a_e4m3, M, b_e4m3, 2 * I, K, args, s);
 }
 
+lnq_status lnq_m_grouped_mx_gemm_contiguous(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                            const void* sfb_atoms, const int32_t* m_indices, int32_t num_groups,
+                                            void* d_bf16, int64_t M_total, int64_t N, int64_t K, void* stream) {
+    using C = MxCfg<4>;
+    if (M_total <= 0 || N <= 0 || K <= 0 || num_groups <= 0) return LNQ_ERR_INVALID_ARG;
+    if (M_total % 128 != 0 || N % 128 != 0 || K % 128 != 0 || M_total > kMaxRows || K > (int64_t{1} << 31) ||
+        static_cast<int64_t>(num_groups) * N > kMaxRows)
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!a_e4m3 || !sfa_atoms || !b_e4m3 || !sfb_atoms || !m_indices || !d_bf16) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(a_e4m3) || !aligned16(sfa_atoms) || !aligned16(b_e4m3) || !aligned16(sfb_atoms) ||
+        !aligned16(d_bf16) || !aligned4(m_indices))
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    const int64_t wrows = static_cast<int64_t>(num_groups) * N;
+    CUtensorMap map_a, map_b;
+    st = encode_e4m3_map(&map_a, a_e4m3, M_total, K, 128);
+    if (st == LNQ_OK) st = encode_e4m3_map(&map_b, b_e4m3, wrows, K, 256);
+    if (st != LNQ_OK) return st;
+    static bool attr_set[kMaxDevices] = {};
+    int devno = 0;
+    cudaGetDevice(&devno);
+    if (!attr_set[devno]) {
+        if (cudaFuncSetAttribute(k_mx_block_gemm<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes) != cudaSuccess)
+            return LNQ_ERR_CUDA;
+        attr_set[devno] = true;
+    }
+    MxArgs args{};
+    args.sfa = static_cast<const uint32_t*>(sfa_atoms);
+    args.sfb = static_cast<const uint32_t*>(sfb_atoms);
+    args.d = static_cast<uint16_t*>(d_bf16);
+    args.status = dev->status;
+    args.timeout_ns = kDefaultTimeoutNs;
+    args.M = static_cast<int>(M_total);
+    args.N = static_cast<int>(N);
+    args.num_kb = static_cast<int>(K / 128);
+    args.mblocks = static_cast<int>(M_total / 128);
+    args.nblocks = static_cast<int>(wrows / 128);
+    args.tiles_p = args.mblocks;
+    args.tiles_q = static_cast<int>((N + 255) / 256);
+    args.num_tiles = args.tiles_p * args.tiles_q;
+    args.m_indices = m_indices;
+    args.num_groups = num_groups;
+    const int grid = args.num_tiles < dev->sm_count ? args.num_tiles : dev->sm_count;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4, true>, map_a, map_b, args) != cudaSuccess) return LNQ_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
 lnq_status lnq_m_grouped_fp8_gemm_contiguous_psum(const void* a_e4m3, const float* sfa,
                                                   const void* b_e4m3, const float* sfb,
                                                   const int32_t* psum, int32_t num_groups,

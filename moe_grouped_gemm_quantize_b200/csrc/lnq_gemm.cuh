@@ -94,8 +94,6 @@ struct GemmArgs {
     long long M4_out;
 };
 
-constexpr unsigned int kStatusBadGroup = 2u;
-
 template <int BNQ_, int STAGES_, int EPI_WG_, bool SWAP_, bool GROUPED_, bool PAIR_ = false,
           int SLICES_ = 1, bool SPLITK_ = false, bool SILU_ = false>
 struct GemmCfg {

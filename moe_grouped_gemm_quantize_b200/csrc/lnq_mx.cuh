@@ -196,13 +196,18 @@ __global__ void __launch_bounds__(256) k_quantize_ue8m0_blocks(const uint16_t* _
 
 struct MxArgs {
     const uint32_t* sfa;   // activation scale atoms [K/128][ceil(M/128)][128]
-    const uint32_t* sfb;   // weight scale atoms [K/128][ceil(N/128)][128]
+    const uint32_t* sfb;   // weight scale atoms [K/128][ceil(rows of B / 128)][128]
     uint16_t* d;           // [M][N] bf16 bits
     unsigned int* status;  // device status word
     unsigned long long timeout_ns;
     int M, N, num_kb;
-    int mblocks, nblocks;  // ceil(M/128), ceil(N/128)
+    int mblocks, nblocks;  // ceil(M/128), ceil(rows of B / 128)
     int tiles_p, tiles_q, num_tiles;
+    // M-grouped contiguous layout (GROUPED): each 128-row block of A takes the weights
+    // of the group named by its first row's id (rows g*N .. g*N + N - 1 of B, N % 128
+    // == 0); a block led by a negative id is skipped.
+    const int32_t* m_indices;
+    int num_groups;
 };
 
 // One persistent CTA per SM, tiles of 128 rows x 256 columns, 384 threads:
@@ -213,6 +218,8 @@ struct MxArgs {
 //               four block-scaled MMAs of K = 32 into the tile's accumulator;
 //   warps 4-11  epilogue: after the tile's last K block, read the 128 x 256 FP32
 //               accumulator, release it, round to bf16 and store.
+// With GROUPED, a 128-row block of A takes its group's weights (the M-grouped
+// contiguous MoE layout, deepgemm-rust README, "Grouped (contiguous) MoE GEMM").
 // Tensor memory: the accumulator in columns 0-255; stage s's A scales in columns
 // 256 + 16 s .. + 3 and its B scales in 256 + 16 s + 4 .. + 11.  The scales are
 // applied by the tensor core, so no promotion FMAs run and the accumulator is read
@@ -237,7 +244,7 @@ struct MxCfg {
     static_assert(kSfCol0 + 16 * STAGES <= kTmemCols, "scale columns");
 };
 
-template <int STAGES>
+template <int STAGES, bool GROUPED = false>
 __global__ void __launch_bounds__(384, 1)
     k_mx_block_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const MxArgs args) {
@@ -287,9 +294,11 @@ __global__ void __launch_bounds__(384, 1)
     wctx.status = args.status;
     wctx.timeout_ns = args.timeout_ns;
 
-    // banded raster, column-major inside bands of 16 row tiles
-    auto tile_rc = [&](int t, int& p0, int& q0) {
-        constexpr int kBand = 16;
+    // banded raster, column-major inside bands of row tiles (16 dense, 8 grouped: the
+    // blocks of a group walk its weight columns together).  Returns the tile's group
+    // (0 dense; -1 for a grouped block to skip) and its first row of B.
+    auto tile_rc = [&](int t, int& p0, int& q0, int& b_row) {
+        constexpr int kBand = GROUPED ? 8 : 16;
         const int band_tiles = kBand * args.tiles_q;
         const int band = t / band_tiles;
         const int first = band * kBand;
@@ -297,6 +306,16 @@ __global__ void __launch_bounds__(384, 1)
         const int r = t - band * band_tiles;
         p0 = (first + r % rows) * 128;
         q0 = (r / rows) * 256;
+        int g = 0;
+        if constexpr (GROUPED) {
+            g = __ldg(args.m_indices + p0);
+            if (g >= args.num_groups) {
+                atomicOr(args.status, kStatusBadGroup);
+                g = -1;
+            }
+        }
+        b_row = (g < 0 ? 0 : g) * args.N + q0;
+        return g;
     };
 
     if (warp < 4) {
@@ -312,10 +331,10 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t phase = 0, filled = 0, fill_parity = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
-                int p0, q0;
-                tile_rc(t, p0, q0);
+                int p0, q0, b_row;
+                if (tile_rc(t, p0, q0, b_row) < 0) continue;
                 const int mb = p0 / 128;
-                const int nb0 = q0 / 128;
+                const int nb0 = b_row / 128;
                 const int nb1 = min(nb0 + 1, args.nblocks - 1);
                 for (int kb = 0; kb < args.num_kb; ++kb) {
                     if (!mbar_wait_warp(empty_bar(stage), phase ^ 1u, wctx)) {
@@ -327,7 +346,7 @@ __global__ void __launch_bounds__(384, 1)
                         const uint32_t sf = sSf + stage * C::kSfBytes;
                         mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes + C::kSfBytes);
                         tma_load_2d(sA + stage * C::kABytes, &map_a, fb, kb * C::kBK, p0);
-                        tma_load_2d(sB + stage * C::kBBytes, &map_b, fb, kb * C::kBK, q0);
+                        tma_load_2d(sB + stage * C::kBBytes, &map_b, fb, kb * C::kBK, b_row);
                         const long long kbase = static_cast<long long>(kb);
                         bulk_load(sf, args.sfa + (kbase * args.mblocks + mb) * 128, 512u, fb);
                         bulk_load(sf + 512u, args.sfb + (kbase * args.nblocks + nb0) * 128, 512u, fb);
@@ -359,6 +378,8 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t phase = 0, aphase = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
+                int p0, q0, b_row;
+                if (tile_rc(t, p0, q0, b_row) < 0) continue;
                 // the epilogue has read the previous tile's accumulator
                 if (!mbar_wait_warp(tempty_bar, aphase ^ 1u, wctx)) break;
                 tc_fence_after();
@@ -409,8 +430,8 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
         uint32_t aphase = 0;
         for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
-            int p0, q0;
-            tile_rc(t, p0, q0);
+            int p0, q0, b_row;
+            if (tile_rc(t, p0, q0, b_row) < 0) continue;
             if (!mbar_wait_warp(tfull_bar, aphase, wctx)) break;
             tc_fence_after();
             uint32_t ra[64], rb[64];

@@ -11,8 +11,10 @@
 
 namespace lnq {
 
-// Device status word bits (read by lnq_get_last_device_error).
+// Device status word bits (read by lnq_get_last_device_error): a wait that timed
+// out; a group id, count or prefix sum out of range.
 constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusBadGroup = 2u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

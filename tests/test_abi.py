@@ -181,6 +181,12 @@ def test_ue8m0_argument_errors(L):
     assert g(A16, A16b, A16c, A16d, A16e, 8, 20, 128, None) == SHAPE   # N % 16
     assert g(A16, A16b, A16c, A16d, A16e, 8, 256, 100, None) == SHAPE  # K % 128
     assert g(A16, A16b + 4, A16c, A16d, A16e, 8, 256, 128, None) == MISALIGNED
+    h = L.lnq_m_grouped_mx_gemm_contiguous
+    assert h(A16, A16b, A16c, A16d, A16e + 0x100, 0, A16e, 256, 256, 128, None) == INVALID
+    assert h(A16, A16b, A16c, A16d, A16e + 0x100, 2, A16e, 200, 256, 128, None) == SHAPE    # M_total % 128
+    assert h(A16, A16b, A16c, A16d, A16e + 0x100, 2, A16e, 256, 192, 128, None) == SHAPE    # N % 128
+    assert h(A16, A16b, A16c, A16d, None, 2, A16e, 256, 256, 128, None) == INVALID
+    assert h(A16, A16b, A16c, A16d, A16e + 0x102, 2, A16e, 256, 256, 128, None) == MISALIGNED
 
 
 def test_epilogue_argument_errors(L):

@@ -10,6 +10,10 @@ by the block-scaled MMA) and "What's implemented" (gran-128 on either side).
 * The GEMM (tcgen05.mma kind::mxf8f6f4.block_scale) is compared with the oracle's FP64
   product of the same codes and power-of-two scales, within the GEMM tolerance, element by
   element on ragged shapes and at sampled points on a prefill linear.
+* The M-grouped contiguous form (each 128-row block takes the group of its first row) is
+  compared with the oracle's grouped product on rows with a group id, element by element on
+  small layouts and at sampled points on the 32-expert MoE workload; blocks led by -1 stay
+  untouched.
 """
 import numpy as np
 import pytest
@@ -110,3 +114,47 @@ def test_repeated_runs_are_identical():
     d1, d2 = run_gemm(a, w), run_gemm(a, w)
     torch.cuda.synchronize()
     assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+
+
+def run_grouped(a, w, m_indices, G):
+    aq, sa = lnq.quantize_activations_ue8m0(a.to(DEV))
+    wq, sw = lnq.quantize_weights_ue8m0(w.to(DEV))
+    N = w.shape[0] // G
+    d = torch.full((a.shape[0], N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lnq.lnq_m_grouped_mx_gemm_contiguous(aq, sa, wq, sw, torch.from_numpy(m_indices).to(DEV), G, d)
+    return d
+
+
+@pytest.mark.parametrize("sizes,N,K", [([130, 0, 256, 7, 300], 256, 256), ([1], 384, 512),
+                                       ([128, 128, 5], 128, 1024), ([200, 90, 129], 512, 256)])
+def test_grouped_elementwise(sizes, N, K):
+    G = len(sizes)
+    m_indices, _, M_total = synthetic.contiguous_layout(sizes)
+    a = synthetic.gaussian_bf16((M_total, K), 1.0, seed=G + N)
+    w = synthetic.gaussian_bf16((G * N, K), 0.02, seed=K + N)
+    d = run_grouped(a, w, m_indices, G)
+    assert lnq.lnq_get_last_device_error() == 0
+    qa, ea = oracle.quantize_ue8m0_groups(synthetic.bf16_bits(a))
+    qb, eb = oracle.quantize_ue8m0_blocks(synthetic.bf16_bits(w))
+    ref = oracle.m_grouped_gemm_contiguous(qa, oracle.ue8m0_value(ea), qb, oracle.ue8m0_value(eb), m_indices, G)
+    got = to_f64(d)
+    real = m_indices >= 0
+    assert_gemm_close(got[real], ref[real], f"ue8m0 grouped {sizes} {N}x{K}")
+    led_by_pad = np.repeat(m_indices[::128] < 0, 128)
+    assert np.all(np.isnan(got[led_by_pad]))
+
+
+def test_grouped_moe_workload_sampled():
+    cfg = synthetic.MOE
+    a, w, m_indices, sizes = synthetic.make_moe_inputs(cfg)
+    d = run_grouped(a, w, m_indices, cfg.groups)
+    assert lnq.lnq_get_last_device_error() == 0
+    qa, ea = oracle.quantize_ue8m0_groups(synthetic.bf16_bits(a))
+    qb, eb = oracle.quantize_ue8m0_blocks(synthetic.bf16_bits(w))
+    rng = np.random.default_rng(23)
+    real = np.flatnonzero(m_indices >= 0)
+    rows = rng.choice(real, 20000)
+    cols = rng.integers(0, cfg.N, 20000)
+    ref = oracle.m_grouped_gemm_points(qa, oracle.ue8m0_value(ea), qb, oracle.ue8m0_value(eb), m_indices,
+                                       cfg.groups, rows, cols)
+    assert_gemm_close(to_f64(d)[rows, cols], ref, "ue8m0 MoE workload")
