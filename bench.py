@@ -45,11 +45,13 @@ if ROOT not in sys.path:
 METRIC = "block-scaled FP8 GEMM TFLOP/s (and GB/s for decode) + % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0   # nominal dense ratio (4.5 / 2.25 PFLOP/s)
-KERNEL_SOURCES = ["moe_grouped_gemm_quantize_b200/csrc/lnq_gemm.cuh",
-                  "moe_grouped_gemm_quantize_b200/csrc/lnq_ptx.cuh",
-                  "moe_grouped_gemm_quantize_b200/csrc/lnq_quantize.cuh",
-                  "moe_grouped_gemm_quantize_b200/csrc/lnq_mx.cuh",
-                  "moe_grouped_gemm_quantize_b200/csrc/lnq_api.cu"]
+_CSRC = "moe_grouped_gemm_quantize_b200/csrc/"
+# the files each GEMM kernel is built and launched from: a recorded ncu traffic figure
+# stands only while these are unchanged
+KERNEL_SOURCES = {
+    "k_fp8_block_gemm": [_CSRC + f for f in ("lnq_gemm.cuh", "lnq_ptx.cuh", "lnq_quantize.cuh", "lnq_api.cu")],
+    "k_mx_block_gemm": [_CSRC + f for f in ("lnq_mx.cuh", "lnq_ptx.cuh", "lnq_quantize.cuh", "lnq_api.cu")],
+}
 
 
 # --------------------------------------------------------------------------- setup
@@ -102,9 +104,9 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str = "k_fp8_block_gemm") -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -118,7 +120,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(path) as f:
         rec = json.load(f)
     e = rec.get(workload, {}).get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 
