@@ -99,12 +99,15 @@ __device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64
 
 // ------------------------------------------------------------------ quantize
 
-// Activations: every half warp quantizes one 1 x 128 group (row m, group g) per
-// step, 8 inputs per lane.  Rows M .. Mpad-1 only get the scale word of p = 1.
+// Activations: every half warp quantizes four consecutive 1 x 128 groups per step
+// (8 inputs per lane and group; the four 16-byte loads of a lane are issued before
+// any reduction, so they are in flight together).  Rows M .. Mpad-1 only get the
+// scale word of p = 1.
 __global__ void __launch_bounds__(256) k_quantize_ue8m0_groups(const uint16_t* __restrict__ x, int M, int K,
                                                                long long ld_x, uint8_t* __restrict__ q,
                                                                long long ld_q, uint32_t* __restrict__ sf,
                                                                int Mpad) {
+    constexpr int kPerHalf = 4;
     wait_prior_grids();
     launch_dependents();
     const int G = K / 128;
@@ -114,34 +117,43 @@ __global__ void __launch_bounds__(256) k_quantize_ue8m0_groups(const uint16_t* _
     const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
     const long long warp = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int rblocks = Mpad / 128;
-    for (long long base = warp * 2; base < units; base += warps * 2) {
-        const long long u = base + half;
-        const bool valid = u < units;
-        const int m = valid ? static_cast<int>(u / G) : 0;
-        const int g = valid ? static_cast<int>(u % G) : 0;
-        const bool real = valid && m < M;
-        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-        if (real) raw = ld_nc_v4(x + m * ld_x + g * 128 + l16 * 8);
-        float amax = absmax8(raw);
+    for (long long base = warp * 2 * kPerHalf; base < units; base += warps * 2 * kPerHalf) {
+        uint4 raw[kPerHalf];
+        int m[kPerHalf], g[kPerHalf];
+        bool valid[kPerHalf], real[kPerHalf];
 #pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const int e = ue8m0_exponent(amax);
-        if (real) {
-            const float r = pow2_neg(e);
-            float t[8];
-            t[0] = bf16_lo(raw.x) * r;
-            t[1] = bf16_hi(raw.x) * r;
-            t[2] = bf16_lo(raw.y) * r;
-            t[3] = bf16_hi(raw.y) * r;
-            t[4] = bf16_lo(raw.z) * r;
-            t[5] = bf16_hi(raw.z) * r;
-            t[6] = bf16_lo(raw.w) * r;
-            t[7] = bf16_hi(raw.w) * r;
-            *reinterpret_cast<uint2*>(q + m * ld_q + g * 128 + l16 * 8) = pack8(t);
+        for (int j = 0; j < kPerHalf; ++j) {
+            const long long u = base + half * kPerHalf + j;
+            valid[j] = u < units;
+            m[j] = valid[j] ? static_cast<int>(u / G) : 0;
+            g[j] = valid[j] ? static_cast<int>(u % G) : 0;
+            real[j] = valid[j] && m[j] < M;
+            raw[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (real[j]) raw[j] = ld_nc_v4(x + m[j] * ld_x + g[j] * 128 + l16 * 8);
         }
-        if (valid && l16 == 0)
-            sf[(static_cast<long long>(g) * rblocks + m / 128) * 128 + atom_word(m & 127)] =
-                static_cast<uint32_t>(e + 127);
+#pragma unroll
+        for (int j = 0; j < kPerHalf; ++j) {
+            float amax = absmax8(raw[j]);
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const int e = ue8m0_exponent(amax);
+            if (real[j]) {
+                const float r = pow2_neg(e);
+                float t[8];
+                t[0] = bf16_lo(raw[j].x) * r;
+                t[1] = bf16_hi(raw[j].x) * r;
+                t[2] = bf16_lo(raw[j].y) * r;
+                t[3] = bf16_hi(raw[j].y) * r;
+                t[4] = bf16_lo(raw[j].z) * r;
+                t[5] = bf16_hi(raw[j].z) * r;
+                t[6] = bf16_lo(raw[j].w) * r;
+                t[7] = bf16_hi(raw[j].w) * r;
+                *reinterpret_cast<uint2*>(q + m[j] * ld_q + g[j] * 128 + l16 * 8) = pack8(t);
+            }
+            if (valid[j] && l16 == 0)
+                sf[(static_cast<long long>(g[j]) * rblocks + m[j] / 128) * 128 + atom_word(m[j] & 127)] =
+                    static_cast<uint32_t>(e + 127);
+        }
     }
 }
 
