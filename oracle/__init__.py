@@ -23,24 +23,34 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "lnq_oracle.c")
 _LIB = os.path.join(_HERE, "liblnq_oracle.so")
+# The mutation tests point this at a compiled copy of the oracle with one planted
+# mistake, to show that the pins catch it; unset, the oracle is built from _SRC.
+_LIB_OVERRIDE = os.environ.get("LNQ_ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
 GROUP = 128
 
 
-def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (OpenMP, no FMA contraction, no fast-math)."""
-    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
-        return _LIB
-    tmp = _LIB + f".tmp{os.getpid()}"
+def compile_source(src: str, out: str) -> str:
+    """Compile an oracle source file with gcc (OpenMP, no FMA contraction, no fast-math)."""
+    tmp = out + f".tmp{os.getpid()}"
     cmd = [
         "gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-        "-fPIC", "-shared", "-Wall", "-o", tmp, _SRC, "-lm",
+        "-fPIC", "-shared", "-Wall", "-o", tmp, src, "-lm",
     ]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, _LIB)
-    return _LIB
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Build the oracle library next to its source (when out of date)."""
+    if _LIB_OVERRIDE:
+        return _LIB_OVERRIDE
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    return compile_source(_SRC, _LIB)
 
 
 def _load():
@@ -48,8 +58,7 @@ def _load():
     with _lock:
         if _lib is not None:
             return _lib
-        build()
-        lib = ctypes.CDLL(_LIB)
+        lib = ctypes.CDLL(build())
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         lib.oracle_num_threads.restype = ctypes.c_int
