@@ -7,7 +7,9 @@ The planted mistakes are the slips a reader of the pages could make: gate and up
 the sign of the SiLU exponent, a scale one power of two too large at exact multiples of 448,
 the wrong scale of an all-zero group, a block amax over one row, an off-by-one group count,
 the next group's weights, the plain (non-aligned) row order of the prefix-sum layout, a
-dropped weight scale, and a wrong rounding of E4M3 ties.
+dropped weight scale, a wrong rounding of E4M3 ties, a wrong scale divisor, row-major
+instead of MN-major activation scales, a transposed activation-scale index in the product,
+and a masked count taken as inclusive.
 """
 import os
 import subprocess
@@ -58,6 +60,22 @@ MUTATIONS = {
         "    f = nearbyint((scaled - 1.0) * 8.0); /* 3-bit mantissa, ties to even */",
         "    f = floor((scaled - 1.0) * 8.0 + 0.5);",
         "tests/test_oracle_e4m3.py"),
+    "quantize_scale_divisor": (
+        "            s = amax / 448.0f;\n            sfa[g * M4 + m] = s;",
+        "            s = amax / 447.0f;\n            sfa[g * M4 + m] = s;",
+        "tests/test_oracle_quantize.py"),
+    "quantize_scales_row_major": (
+        "            sfa[g * M4 + m] = s;",
+        "            sfa[m * G + g] = s;",
+        "tests/test_oracle_quantize.py"),
+    "gemm_activation_scale_index": (
+        "(double)sfa[(k / ORACLE_GROUP) * M4 + m];",
+        "(double)sfa[(k / ORACLE_GROUP) + m * (K / ORACLE_GROUP)];",
+        "tests/test_oracle_gemm.py"),
+    "masked_count_inclusive": (
+        "            if (m >= masked_m[gr] || !ad || !bd)",
+        "            if (m > masked_m[gr] || !ad || !bd)",
+        "tests/test_oracle_masked.py"),
     "gemm_weight_scale_dropped": (
         "        out[k] = oracle_e4m3_value(qb[row * K + k]) * (double)sfb[sb_row * KB + k / ORACLE_GROUP];",
         "        out[k] = oracle_e4m3_value(qb[row * K + k]);",
