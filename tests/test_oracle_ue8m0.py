@@ -6,13 +6,16 @@ reading: a group's (or block's) scale is the smallest power of two p with 448 p 
 stored as e + 127; codes are the E4M3 RNE of x / p.  Pinned against:
 
 * the defining inequalities 448 p >= amax > 448 p / 2, evaluated in exact rationals, over
-  random and boundary amax values, and hand-worked examples;
+  random and boundary amax values, and hand-worked examples (one of them the four-group
+  row of tests/golden/ue8m0_worked_example.json);
 * torch's independent float32 -> float8_e4m3fn conversion of x / p;
 * properties: no code saturates, every non-zero group has a code of magnitude >= 224,
   dequantized values lie within half an E4M3 step of the input;
 * blocks: the amax over a 128 x 128 block (ragged edges included), and the activation
   rule applied to a single-row block.
 """
+import json
+import os
 from fractions import Fraction
 
 import numpy as np
@@ -140,3 +143,19 @@ def test_gemm_with_ue8m0_scales_is_the_plain_product():
     qb2, sb2 = oracle.quantize_fp8_blocks(synthetic.bf16_bits(w))
     D2 = oracle.gemm_nt(qa2, sa2, qb2, sb2)
     assert np.linalg.norm(D - D2) / np.linalg.norm(D2) < 0.1
+
+
+def test_golden_worked_example():
+    path = os.path.join(os.path.dirname(__file__), "golden", "ue8m0_worked_example.json")
+    ex = json.load(open(path))
+    row = np.zeros(ex["K"], dtype=np.float32)
+    for k, v in ex["inputs"].items():
+        row[int(k)] = v
+    bits = bf16_bits_of(row)[None, :]
+    assert np.array_equal(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()[0], row)
+    q, sfe = oracle.quantize_ue8m0_groups(bits)
+    assert list(sfe[:, 0]) == ex["scale_bytes"]
+    expected = np.zeros(ex["K"], dtype=np.uint8)
+    for k, c in ex["codes"].items():
+        expected[int(k)] = c
+    assert np.array_equal(q[0], expected)
