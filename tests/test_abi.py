@@ -52,6 +52,18 @@ def test_library_exports_every_declared_symbol(L):
     assert L.lnq_abi_version() == 10000
 
 
+def test_library_exports_nothing_undeclared(L):
+    # every lnq_* symbol the library exports is part of the declared ABI
+    import shutil
+    import subprocess
+    if shutil.which("nm") is None:
+        pytest.skip("nm not available")
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.split() and line.split()[-1].startswith("lnq_")}
+    assert exported == set(declared_functions())
+
+
 def test_status_strings(L):
     for code in range(7):
         assert lnq.lnq_status_string(code)
