@@ -219,8 +219,12 @@ lnq_status lnq_fp8_block_gemm_nt_ws(const void* a_e4m3, const float* sfa, int64_
  * The array is shared by every call on the device: calls that overlap in time (on
  * different streams, or from several threads without ordering) race on it and
  * must not be issued.  After a call the array keeps that call's partial tiles
- * (its counters are zero again); after LNQ_ERR_TIMEOUT the counters may not be
- * zero and later results of this entry point are undefined.
+ * (its counters are zero again).  A call that gave up on a wait may leave tile
+ * counters non-zero; lnq_get_last_device_error, when it reports LNQ_ERR_TIMEOUT,
+ * zeroes the counter region of the array on the current device (a memset of its
+ * first 4 KiB; nothing is allocated), so later calls are correct again.
+ * Argument errors are returned before any CUDA call, as for lnq_fp8_block_gemm_nt;
+ * a device numbered 64 or above returns LNQ_ERR_INVALID_ARG.
  */
 lnq_status lnq_fp8_block_gemm_nt_static_ws(const void* a_e4m3, const float* sfa, int64_t M4,
                                            const void* b_e4m3, const float* sfb, void* d_bf16,
@@ -384,6 +388,9 @@ const char* lnq_status_string(lnq_status status);
  * since the last call gave up on a bounded wait (the kernel then skipped its
  * remaining work and released its tensor memory; its outputs are
  * unspecified), LNQ_ERR_CUDA if the synchronization failed, else LNQ_OK.
+ * On a timeout it also zeroes the tile counters of the scratch array that
+ * lnq_fp8_block_gemm_nt_static_ws uses on this device (on `stream`, then
+ * synchronizes it again).
  */
 lnq_status lnq_get_last_device_error(void* stream);
 

@@ -36,6 +36,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 struct DeviceInfo {
     bool ready = false;
     bool supported = false;
+    int ordinal = 0;                 // device number, < kMaxDevices
     int sm_count = 0;
     unsigned int* status = nullptr;  // device address of g_status
 };
@@ -52,6 +53,19 @@ DeviceInfo g_devices[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Raises a kernel's dynamic shared-memory limit once per device.  The per-device flags
+// are atomic: first calls racing from several host threads may each set the attribute,
+// which is harmless.
+template <class Kernel>
+lnq_status smem_attr_once(std::atomic<bool> (&done)[kMaxDevices], int ordinal, Kernel* kernel, int bytes) {
+    if (!done[ordinal].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+            return LNQ_ERR_CUDA;
+        done[ordinal].store(true, std::memory_order_release);
+    }
+    return LNQ_OK;
+}
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // Current device's capabilities; resolves the driver's tensor-map encoder once.
@@ -68,6 +82,7 @@ lnq_status device_info(DeviceInfo** out) {
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return LNQ_ERR_CUDA;
         d.supported = (major == 10 && minor == 0);
+        d.ordinal = dev;
         d.sm_count = sms;
         if (d.supported) {
             void* p = nullptr;
@@ -121,22 +136,16 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
                                  C::SILU ? C::kQBoxRows : (C::PAIR ? C::kSliceQRows : C::kQRowsPerCta));
     }
     if (st != LNQ_OK) return st;
-    static bool attr_set[kMaxDevices] = {};
-    int devno = 0;
-    cudaGetDevice(&devno);
-    if (!attr_set[devno]) {
-        if (cudaFuncSetAttribute(k_fp8_block_gemm<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes) != cudaSuccess)
-            return LNQ_ERR_CUDA;
-        attr_set[devno] = true;
-    }
+    static std::atomic<bool> attr_set[kMaxDevices];
+    st = smem_attr_once(attr_set, dev.ordinal, k_fp8_block_gemm<C>, C::kSmemBytes);
+    if (st != LNQ_OK) return st;
     args.status = dev.status;
     args.timeout_ns = kDefaultTimeoutNs;
     args.prefetch_weights = g_weight_prefetch.load(std::memory_order_relaxed);
     if constexpr (C::PAIR) {
         // clusters of two CTAs sharing one MMA; as many pairs as can be resident
         constexpr int kCluster = 2;
-        static int max_clusters[kMaxDevices] = {};
+        static std::atomic<int> max_clusters[kMaxDevices];
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -150,14 +159,14 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
         cfg.stream = stream;
         cfg.attrs = attr;
         cfg.numAttrs = 2;
-        if (max_clusters[devno] == 0) {
-            int n = 0;
+        int resident = max_clusters[dev.ordinal].load(std::memory_order_relaxed);
+        if (resident == 0) {
             cfg.gridDim = dim3(2 * (dev.sm_count / 2), 1, 1);
-            if (cudaOccupancyMaxActiveClusters(&n, k_fp8_block_gemm<C>, &cfg) != cudaSuccess || n <= 0)
+            if (cudaOccupancyMaxActiveClusters(&resident, k_fp8_block_gemm<C>, &cfg) != cudaSuccess || resident <= 0)
                 return LNQ_ERR_CUDA;
-            max_clusters[devno] = n;
+            max_clusters[dev.ordinal].store(resident, std::memory_order_relaxed);
         }
-        const int clusters = args.num_tiles < max_clusters[devno] ? args.num_tiles : max_clusters[devno];
+        const int clusters = args.num_tiles < resident ? args.num_tiles : resident;
         if (clusters <= 0) return LNQ_OK;
         cfg.gridDim = dim3(kCluster * clusters, 1, 1);
         if (cudaLaunchKernelEx(&cfg, k_fp8_block_gemm<C>, map_p, map_q, args) != cudaSuccess)
@@ -200,6 +209,8 @@ using CfgSwap32Split = GemmCfg<32, 10, 1, true, false, false, 1, true>;
 using CfgSwap64Split = GemmCfg<64, 8, 1, true, false, false, 1, true>;
 
 constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
+// Split workspace: one int32 counter per weight tile in a fixed region at its start.
+constexpr int64_t kSplitCounterBytes = 4096;
 
 }  // namespace
 }  // namespace lnq
@@ -211,9 +222,39 @@ using namespace lnq;
 // counters zero), so that entry point allocates nothing.  Calls on several streams
 // would share it: they must not overlap.
 static constexpr int64_t kStaticSplitBytes = int64_t{10} << 20;
+static constexpr int kStaticSplitDevices = 64;
 static __device__ __align__(256) unsigned char g_static_split_scratch[kStaticSplitBytes];
-static void* g_static_split_addr[64] = {};
+static void* g_static_split_addr[kStaticSplitDevices] = {};
 static std::mutex g_static_split_mutex;
+
+// Device address of the scratch array on device `devno` (the current device), looked
+// up once per device; nullptr if the lookup fails.
+static void* static_split_scratch(int devno) {
+    std::lock_guard<std::mutex> lock(g_static_split_mutex);
+    if (g_static_split_addr[devno] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_split_scratch) != cudaSuccess) return nullptr;
+        g_static_split_addr[devno] = p;
+    }
+    return g_static_split_addr[devno];
+}
+
+// After a kernel gave up on a wait, a split may have left tile counters of the scratch
+// array non-zero; later calls would then finish tiles early.  Zero the counter region
+// (the first kSplitCounterBytes) of this device's array if it has been used.  Called
+// with the stream already synchronized.
+static lnq_status reset_static_split_counters(int devno, cudaStream_t stream) {
+    void* p = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_static_split_mutex);
+        if (devno >= 0 && devno < kStaticSplitDevices) p = g_static_split_addr[devno];
+    }
+    if (p == nullptr) return LNQ_OK;  // never used on this device: still all zero
+    if (cudaMemsetAsync(p, 0, static_cast<size_t>(kSplitCounterBytes), stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    return LNQ_OK;
+}
 
 extern "C" {
 
@@ -291,15 +332,9 @@ lnq_status lnq_quantize_fp8_groups(const void* x_bf16, int64_t M, int64_t K, int
     const long long tiles = ((M4 + kQuantRows - 1) / kQuantRows) * static_cast<long long>(qa.col_tiles);
     if (tiles > 0x7FFFFFFFLL) return LNQ_ERR_UNSUPPORTED_SHAPE;
     qa.num_tiles = static_cast<int>(tiles);
-    static bool attr_set[kMaxDevices] = {};
-    int devno = 0;
-    cudaGetDevice(&devno);
-    if (!attr_set[devno]) {
-        if (cudaFuncSetAttribute(k_quantize_groups, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kQuantSmemBytes) != cudaSuccess)
-            return LNQ_ERR_CUDA;
-        attr_set[devno] = true;
-    }
+    static std::atomic<bool> attr_set[kMaxDevices];
+    st = smem_attr_once(attr_set, dev->ordinal, k_quantize_groups, kQuantSmemBytes);
+    if (st != LNQ_OK) return st;
     const long long max_ctas = 3LL * dev->sm_count;
     const int grid = static_cast<int>(tiles < max_ctas ? tiles : max_ctas);
     cudaLaunchConfig_t cfg = {};
@@ -399,15 +434,9 @@ lnq_status lnq_mx_block_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const
     st = encode_e4m3_map(&map_a, a_e4m3, M, K, 128);
     if (st == LNQ_OK) st = encode_e4m3_map(&map_b, b_e4m3, N, K, 256);
     if (st != LNQ_OK) return st;
-    static bool attr_set[kMaxDevices] = {};
-    int devno = 0;
-    cudaGetDevice(&devno);
-    if (!attr_set[devno]) {
-        if (cudaFuncSetAttribute(k_mx_block_gemm<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-            cudaSuccess)
-            return LNQ_ERR_CUDA;
-        attr_set[devno] = true;
-    }
+    static std::atomic<bool> attr_set[kMaxDevices];
+    st = smem_attr_once(attr_set, dev->ordinal, k_mx_block_gemm<4>, C::kSmemBytes);
+    if (st != LNQ_OK) return st;
     MxArgs args{};
     args.sfa = static_cast<const uint32_t*>(sfa_atoms);
     args.sfb = static_cast<const uint32_t*>(sfb_atoms);
@@ -445,7 +474,6 @@ namespace {
 // at the same place for every shape, so one workspace (zeroed once) serves any
 // sequence of products: each call rezeroes the counters it used, and no call writes
 // partial tiles over another shape's counters.
-constexpr int64_t kSplitCounterBytes = 4096;
 struct SplitPlan {
     int64_t need_bytes = 0;
     int64_t partials_offset = kSplitCounterBytes;
@@ -483,10 +511,10 @@ struct Epilogue {
     int64_t M4_out = 0;
 };
 
-lnq_status gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4, const void* b_e4m3,
-                   const float* sfb, void* d_bf16, int64_t M, int64_t N, int64_t K,
-                   void* workspace, int64_t workspace_bytes, void* stream,
-                   const Epilogue& ep = Epilogue()) {
+// The argument checks of a dense product, made on the host before any CUDA call.
+lnq_status check_gemm_args(const void* a_e4m3, const float* sfa, int64_t M4, const void* b_e4m3,
+                           const float* sfb, const void* d_bf16, int64_t M, int64_t N, int64_t K,
+                           const Epilogue& ep) {
     if (M <= 0 || N <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
     if (K % 128 != 0 || N % 16 != 0 || N < 16 || M > kMaxRows || N > kMaxRows ||
         K > (int64_t{1} << 31))
@@ -505,8 +533,18 @@ lnq_status gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4, const void*
         if (ep.M4_out < ((M + 3) / 4) * 4 || ep.M4_out % 4 != 0) return LNQ_ERR_UNSUPPORTED_SHAPE;
         if (!aligned16(ep.q_out) || !aligned16(ep.sfa_out)) return LNQ_ERR_MISALIGNED;
     }
+    return LNQ_OK;
+}
+
+lnq_status gemm_nt(const void* a_e4m3, const float* sfa, int64_t M4, const void* b_e4m3,
+                   const float* sfb, void* d_bf16, int64_t M, int64_t N, int64_t K,
+                   void* workspace, int64_t workspace_bytes, void* stream,
+                   const Epilogue& ep = Epilogue()) {
+    lnq_status st = check_gemm_args(a_e4m3, sfa, M4, b_e4m3, sfb, d_bf16, M, N, K, ep);
+    if (st != LNQ_OK) return st;
+    const bool fp8_out = ep.q_out != nullptr;
     DeviceInfo* dev = nullptr;
-    lnq_status st = device_info(&dev);
+    st = device_info(&dev);
     if (st != LNQ_OK) return st;
 
     GemmArgs args{};
@@ -615,24 +653,20 @@ lnq_status lnq_fp8_block_gemm_nt_ws(const void* a_e4m3, const float* sfa, int64_
 lnq_status lnq_fp8_block_gemm_nt_static_ws(const void* a_e4m3, const float* sfa, int64_t M4,
                                            const void* b_e4m3, const float* sfb, void* d_bf16,
                                            int64_t M, int64_t N, int64_t K, void* stream) {
-    DeviceInfo* dev = nullptr;
-    lnq_status st = device_info(&dev);
+    // argument errors come back before any CUDA call, as for every other entry point
+    lnq_status st = check_gemm_args(a_e4m3, sfa, M4, b_e4m3, sfb, d_bf16, M, N, K, Epilogue());
     if (st != LNQ_OK) return st;
-    int devno = 0;
-    if (cudaGetDevice(&devno) != cudaSuccess) return LNQ_ERR_CUDA;
+    DeviceInfo* dev = nullptr;
+    st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    const int devno = dev->ordinal;
+    if (devno < 0 || devno >= kStaticSplitDevices) return LNQ_ERR_INVALID_ARG;
     const int64_t need = plan_split(M, N, K, dev->sm_count).need_bytes;
     if (need > kStaticSplitBytes) return LNQ_ERR_UNSUPPORTED_SHAPE;
     void* ws = nullptr;
     if (need > 0) {
-        std::lock_guard<std::mutex> lock(g_static_split_mutex);
-        if (g_static_split_addr[devno] == nullptr) {
-            // the device address of the file-scope scratch array, once per device
-            void* p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_static_split_scratch) != cudaSuccess || p == nullptr)
-                return LNQ_ERR_CUDA;
-            g_static_split_addr[devno] = p;
-        }
-        ws = g_static_split_addr[devno];
+        ws = static_split_scratch(devno);
+        if (ws == nullptr) return LNQ_ERR_CUDA;
     }
     return gemm_nt(a_e4m3, sfa, M4, b_e4m3, sfb, d_bf16, M, N, K, ws, kStaticSplitBytes, stream);
 }
@@ -736,15 +770,9 @@ lnq_status lnq_m_grouped_mx_gemm_contiguous(const void* a_e4m3, const void* sfa_
     st = encode_e4m3_map(&map_a, a_e4m3, M_total, K, 128);
     if (st == LNQ_OK) st = encode_e4m3_map(&map_b, b_e4m3, wrows, K, 256);
     if (st != LNQ_OK) return st;
-    static bool attr_set[kMaxDevices] = {};
-    int devno = 0;
-    cudaGetDevice(&devno);
-    if (!attr_set[devno]) {
-        if (cudaFuncSetAttribute(k_mx_block_gemm<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes) != cudaSuccess)
-            return LNQ_ERR_CUDA;
-        attr_set[devno] = true;
-    }
+    static std::atomic<bool> attr_set[kMaxDevices];
+    st = smem_attr_once(attr_set, dev->ordinal, k_mx_block_gemm<4, true>, C::kSmemBytes);
+    if (st != LNQ_OK) return st;
     MxArgs args{};
     args.sfa = static_cast<const uint32_t*>(sfa_atoms);
     args.sfb = static_cast<const uint32_t*>(sfb_atoms);
@@ -891,7 +919,11 @@ lnq_status lnq_get_last_device_error(void* stream) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return LNQ_ERR_CUDA;
     }
-    if (v & kStatusTimeout) return LNQ_ERR_TIMEOUT;
+    if (v & kStatusTimeout) {
+        st = reset_static_split_counters(dev->ordinal, static_cast<cudaStream_t>(stream));
+        if (st != LNQ_OK) return st;
+        return LNQ_ERR_TIMEOUT;
+    }
     if (v & kStatusBadGroup) return LNQ_ERR_INVALID_ARG;
     return LNQ_OK;
 }

@@ -114,6 +114,29 @@ def test_gemm_argument_errors(L):
     assert call(sfa=A16b + 4) == MISALIGNED
 
 
+@pytest.mark.parametrize("entry", ["lnq_fp8_block_gemm_nt_static_ws", "lnq_fp8_block_gemm_nt_ws"])
+def test_split_entry_points_reject_arguments_before_any_cuda_call(L, entry):
+    # the allocation-free and the workspace entry points validate exactly as
+    # lnq_fp8_block_gemm_nt does, before touching a device (here there is none)
+    f = getattr(L, entry)
+    args = dict(a=A16, sfa=A16b, M4=8, b=A16c, sfb=A16d, d=A16e, M=8, N=256, K=512)
+
+    def call(**kw):
+        v = dict(args, **kw)
+        tail = (None,) if entry.endswith("static_ws") else (None, 0, None)
+        return f(v["a"], v["sfa"], v["M4"], v["b"], v["sfb"], v["d"], v["M"], v["N"], v["K"], *tail)
+
+    assert call(M=0) == INVALID
+    assert call(M=-3) == INVALID
+    assert call(K=500) == SHAPE
+    assert call(N=8) == SHAPE
+    assert call(M4=4) == SHAPE
+    assert call(a=None) == INVALID
+    assert call(d=None) == INVALID
+    assert call(d=A16e + 8) == MISALIGNED
+    assert call(sfa=A16b + 4) == MISALIGNED
+
+
 def test_grouped_argument_errors(L):
     f = L.lnq_m_grouped_fp8_gemm_contiguous
 

@@ -65,3 +65,26 @@ def test_a_split_larger_than_the_array_is_rejected():
     with pytest.raises(lnq.LnqError):
         lnq.lnq_fp8_block_gemm_nt_static_ws(aq, sa, wq, ws, d)
     assert lnq.lnq_get_last_device_error() == 0
+
+
+def test_a_reported_timeout_leaves_the_array_usable():
+    # lnq_get_last_device_error, on reporting a timeout, zeroes the tile counters of
+    # the array (a split that gave up on a wait could have left some non-zero); the
+    # timeout here comes from the self-test wait, so none is left, and the calls after
+    # it must still give the workspace entry point's bytes
+    M, N, K = 32, 12288, 4096
+    aq, sa, wq, ws = operands(M, N, K, seed=11)
+    work = lnq.gemm_workspace(M, N, K, DEV)
+    d_ref = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
+    lnq.lnq_fp8_block_gemm_nt_ws(aq, sa, wq, ws, d_ref, work)
+    d = torch.empty_like(d_ref)
+    lnq.lnq_fp8_block_gemm_nt_static_ws(aq, sa, wq, ws, d)
+    lnq.lnq_selftest_wait_timeout(5_000_000)
+    assert lnq.lnq_get_last_device_error() == 6
+    assert lnq.lnq_get_last_device_error() == 0
+    for _ in range(2):
+        d.fill_(float("nan"))
+        lnq.lnq_fp8_block_gemm_nt_static_ws(aq, sa, wq, ws, d)
+        torch.cuda.synchronize()
+        assert lnq.lnq_get_last_device_error() == 0
+        assert torch.equal(d.view(torch.int16), d_ref.view(torch.int16))
