@@ -2,7 +2,7 @@
 """Benchmark of the block-scaled FP8 linear on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill|decode|moe|moe_psum|moe_masked|square|tiny]
+                    [--workload all|prefill|decode|moe|moe_psum|moe_masked|square|tiny]
 
 One step is one pass of the hot path over one batch of synthetic input: for each
 linear of the workload, the 1x128 activation quantize (lnq_quantize_fp8_groups)
@@ -12,10 +12,14 @@ aligned to 256 rows), or the masked one for `moe_masked`).  Weights are model
 parameters: quantized to 128x128 blocks once, before timing
 (lnq_quantize_fp8_blocks).
 
-Default workload (`prefill`): the dense-transformer prefill linears at M = 2048
-tokens, K = 4096 -- QKV N=6144, O N=4096, gate_up N=24576, down K=12288 -> N=4096.
-A ~ N(0,1), W ~ N(0,0.02), bf16, seeded.  The step touches ~500 MB, more than
-the 126 MB L2, so no extra L2 flush is used between steps.
+Default (`--workload all`): every timed workload, one after the other, in one JSON
+line.  The headline (the line's own value, roofline, e2e and cpu_baseline) is the
+largest single-GPU workload, the square 8192^3 GEMM with 5% outlier groups; the
+prefill linears at M = 2048 (QKV N=6144, O N=4096, gate_up N=24576, down K=12288 ->
+N=4096), the decode linears (M = 1, 8, 32, 64; N=12288, K=4096) and the 32-expert
+MoE GEMM follow under `configs`, each with the same keys.  A ~ N(0,1), W ~
+N(0,0.02) (square: N(0,1) with outliers), bf16, seeded.  Every workload's step
+touches more than the 126 MB L2, so no extra L2 flush is used between steps.
 
 Multi-GPU (torchrun): every rank runs its own replica of the workload (its own
 tokens, replicated weights); no collective is on the data path.  The timed
@@ -135,7 +139,7 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples = []
         self.reasons = set()
         self.period = period_s
@@ -441,7 +445,234 @@ def is_hbm_bound(name: str) -> bool:
     return name in ("decode", "moe_masked")
 
 
+# The default run: every timed workload of the block-scaled FP8 linear, the largest
+# single-GPU one (square 8192^3) first as the headline.
+ALL_WORKLOADS = ("square", "prefill", "decode", "moe")
+
+# How each workload keeps the timed kernels reading their operands from HBM rather than L2.
+L2_NOTE = {
+    "square": "inputs larger than L2: A and W E4M3 67 MB each, D 134 MB, and the step's quantize "
+              "reads 134 MB of bf16 between GEMMs (126 MB L2); no extra flush",
+    "prefill": "working set per step ~500 MB > 126 MB L2 (four linears); no extra flush",
+    "decode": "four distinct 50 MB weights per step (200 MB > 126 MB L2), each read once per step; "
+              "no extra flush",
+    "moe": "1.1 GB of expert weights and activations per step > 126 MB L2; no extra flush",
+    "moe_psum": "1.1 GB of expert weights and activations per step > 126 MB L2; no extra flush",
+    "moe_masked": "32 experts' weights (940 MB) per step > 126 MB L2; no extra flush",
+    "tiny": "tiny: fits in L2 (parity-only workload)",
+}
+
+
 # --------------------------------------------------------------------------- our arm
+
+def make_units(name: str, args, dev):
+    cfgs, kind = workload_units(name)
+    return [Grouped(c, dev, recipe=args.recipe) if kind == "grouped"
+            else Grouped(c, dev, alignment=256) if kind == "psum"
+            else Masked(c, dev) if kind == "masked"
+            else Linear(c, dev, split=args.split, fp8_out=args.epilogue == "fp8",
+                        silu=args.epilogue == "silu", recipe=args.recipe) for c in cfgs]
+
+
+def describe_times(ms):
+    """min / median / mean of a list of per-launch milliseconds."""
+    return {"min": round(min(ms), 5), "median": round(statistics.median(ms), 5),
+            "mean": round(statistics.mean(ms), 5), "reps": len(ms)}
+
+
+def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seconds: float):
+    """Everything the bench reports for one workload, as a dict (the same keys as the
+    top-level JSON line, without `metric`).
+
+    * value: the step (quantize + GEMM of every linear) over K steps between two events,
+      with every kernel chained by programmatic dependent launch; max over ranks.
+    * kernels: each kernel between its own two events, over max(K, 50) steps (min and
+      median per launch); and the GEMMs alone back to back (chained as in the step, no
+      quantize between them), over the same number of repetitions: their mean period
+      per launch is the duration `roofline.achieved` divides by.
+    * e2e: the step through the public calls with the bf16 activations copied in from
+      pinned host memory and the outputs copied back, every step.
+    """
+    import moe_grouped_gemm_quantize_b200 as lnq
+
+    units = make_units(name, args, dev)
+    stream = torch.cuda.current_stream(dev)
+    calls = [u.calls(stream.cuda_stream) for u in units]
+    n_units = len(units)
+    flops_step = sum(u.flops for u in units)
+    bytes_step = sum(u.gemm_bytes for u in units)
+    hbm = is_hbm_bound(name)
+
+    def run(fn_args, what):
+        fn, a = fn_args
+        rc = fn(*a)
+        if rc:
+            raise lnq.LnqError(rc, f"{name} {what}")
+
+    def launch_step(ev=None):
+        for i, (q, g) in enumerate(calls):
+            if ev is not None:
+                ev[2 * i].record(stream)
+            run(q, "quantize")
+            if ev is not None:
+                ev[2 * i + 1].record(stream)
+            run(g, "gemm")
+        if ev is not None:
+            ev[2 * n_units].record(stream)
+
+    for _ in range(args.warmup):
+        launch_step()
+    torch.cuda.synchronize()
+    if lnq.lnq_get_last_device_error() != 0:
+        raise RuntimeError(f"{name}: device reported an error during warm-up")
+
+    K = args.steps
+    R = max(K, args.kernel_reps)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        # ---- the timed region: K steps between two events on the launching stream
+        barrier(dist)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(K):
+            launch_step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(dist)
+        ms_local = t0.elapsed_time(t1)
+        if lnq.lnq_get_last_device_error() != 0:
+            raise RuntimeError(f"{name}: device reported an error in the timed region")
+
+        # ---- each kernel between its own events (no overlap with its neighbours)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_units + 1)] for _ in range(R)]
+        torch.cuda.synchronize()
+        for r in range(R):
+            launch_step(evs[r])
+        torch.cuda.synchronize()
+        per_gemm = [[evs[r][2 * i + 1].elapsed_time(evs[r][2 * i + 2]) for r in range(R)] for i in range(n_units)]
+        per_quant = [[evs[r][2 * i].elapsed_time(evs[r][2 * i + 1]) for r in range(R)] for i in range(n_units)]
+
+        # ---- the GEMMs alone, back to back as the step chains them
+        for _ in range(3):
+            for _, g in calls:
+                run(g, "gemm")
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        c0.record(stream)
+        for _ in range(R):
+            for _, g in calls:
+                run(g, "gemm")
+        c1.record(stream)
+        torch.cuda.synchronize()
+        chained_ms = c0.elapsed_time(c1)
+        if lnq.lnq_get_last_device_error() != 0:
+            raise RuntimeError(f"{name}: device reported an error in the kernel loops")
+    ms = max_over_ranks(ms_local, dist, dev)
+    chained_ms = max_over_ranks(chained_ms, dist, dev)
+
+    # ---- end to end through the public calls: host inputs in, host outputs back
+    e2e = None
+    if not args.no_e2e:
+        Ke = max(1, min(K, args.e2e_steps))
+        for u in units:                       # warm the copy paths
+            u.x.copy_(u.host_x, non_blocking=True)
+            u.copy_out()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier(dist)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(Ke):
+            for u, (q, g) in zip(units, calls):
+                u.x.copy_(u.host_x, non_blocking=True)
+                run(q, "e2e quantize")
+                run(g, "e2e gemm")
+                u.copy_out()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(dist)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        if hbm:
+            ev_val, ev_unit = job_throughput(bytes_step, Ke, world, e_ms, 1e9), "GB/s"
+        else:
+            ev_val, ev_unit = job_throughput(flops_step, Ke, world, e_ms, 1e12), "TFLOP/s"
+        e2e = {"value": round(ev_val, 3), "unit": ev_unit, "steps": Ke,
+               "h2d_bytes_per_step": int(sum(u.h2d_bytes for u in units)),
+               "d2h_bytes_per_step": int(sum(u.d2h_bytes for u in units)),
+               "note": "pinned host bf16 activations copied in and the outputs copied back "
+                       "every step; weights resident (model parameters)"}
+
+    # ---- numbers
+    peaks, peak_src = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    gemm_period_ms = chained_ms / (R * n_units)
+    if hbm:
+        value = job_throughput(bytes_step, K, world, ms, 1e9)
+        unit = "GB/s"
+        ach = bytes_step * R / (chained_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 4)}
+        peak_note = f"HBM copy bandwidth ({peak_src}; burst)"
+        iso = [bytes_step / n_units / (statistics.median(t) * 1e-3) / 1e9 for t in per_gemm]
+    else:
+        value = job_throughput(flops_step, K, world, ms, 1e12)
+        unit = "TFLOP/s"
+        ach = flops_step * R / (chained_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4)}
+        peak_note = (f"dense FP8 = {FP8_OVER_BF16:g} x bf16 cuBLAS burst {peaks['bf16_tflops']} "
+                     f"TFLOP/s ({peak_src})")
+        iso = [u.flops / (statistics.median(t) * 1e-3) / 1e12 for u, t in zip(units, per_gemm)]
+    ue8m0 = any(getattr(u, "ue8m0", False) for u in units)
+    kernel_name = "k_mx_block_gemm" if ue8m0 else "k_fp8_block_gemm"
+    roof["traffic"] = recorded_traffic(kernel_name, name)
+    roof["kernel"] = kernel_name
+    roof["peak_source"] = peak_note
+    roof["duration"] = ("mean period per GEMM launch over the workload's GEMMs launched back to "
+                        f"back {R} times (chained by programmatic dependent launch as in the step)")
+    roof["algorithmic_per_launch"] = ({"bytes": [int(u.gemm_bytes) for u in units]} if hbm
+                                      else {"flops": [float(u.flops) for u in units]})
+    roof["isolated_median"] = {"value": [round(x, 1) for x in iso], "unit": roof["unit"],
+                               "note": "each GEMM between its own two events (no overlap)"}
+    q_total = sum(statistics.median(t) for t in per_quant)
+    g_total = sum(statistics.median(t) for t in per_gemm)
+    quant_gbs = sum(u.quant_bytes for u in units) / (q_total * 1e-3) / 1e9
+    out = {
+        "value": round(value, 3),
+        "unit": unit,
+        "ms_per_step": round(ms / K, 5),
+        "steps": K,
+        "roofline": roof,
+        "kernels": {
+            "gemm_ms_per_launch": [describe_times(t) for t in per_gemm],
+            "quantize_ms_per_launch": [describe_times(t) for t in per_quant],
+            "gemm_chained_ms_per_launch": round(gemm_period_ms, 5),
+            "quantize_gbs": round(quant_gbs, 1),
+            "quantize_frac_of_hbm": round(quant_gbs / peaks["hbm_gbs"], 4),
+            "gemm_share_of_step": round(g_total / (g_total + q_total), 4),
+        },
+        "gpu_launches": K * 2 * n_units,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "desc": WORKLOAD_DESC[name],
+        "recipe": ("UE8M0 power-of-two scales in the tensor core" if ue8m0
+                   else "FP32 scales, per-128-K-block promotion"),
+        "epilogue": ("fp8 output (E4M3 + 1x128 scales)" if any(getattr(u, "fp8_out", False) for u in units)
+                     else "gate_up with SiLU.mul (bf16 h)" if any(getattr(u, "silu", False) for u in units)
+                     else "bf16 output"),
+        "decode_k_split": any(getattr(u, "work", None) is not None for u in units),
+        "l2": L2_NOTE[name],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(name, target_s=cpu_seconds)
+    del calls, units
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
 
 def run_ours(args, world, rank, local):
     import moe_grouped_gemm_quantize_b200 as lnq
@@ -460,182 +691,56 @@ def run_ours(args, world, rank, local):
     # writes them, so the GEMMs may stream them before the previous kernel completes
     lnq.lnq_set_weight_prefetch(not args.no_weight_prefetch)
 
-    cfgs, kind = workload_units(args.workload)
-    units = [Grouped(c, dev, recipe=args.recipe) if kind == "grouped" else Grouped(c, dev, alignment=256) if kind == "psum"
-             else Masked(c, dev) if kind == "masked"
-             else Linear(c, dev, split=args.split, fp8_out=args.epilogue == "fp8",
-                         silu=args.epilogue == "silu", recipe=args.recipe) for c in cfgs]
-    stream = torch.cuda.current_stream(dev)
-    sp = stream.cuda_stream
-    calls = [u.calls(sp) for u in units]
-    n_units = len(units)
-    flops_step = sum(u.flops for u in units)
-    bytes_step = sum(u.gemm_bytes for u in units)
-
-    def launch_step(ev=None):
-        for i, ((qf, qa), (gf, ga)) in enumerate(calls):
-            if ev is not None:
-                ev[2 * i].record(stream)
-            rc = qf(*qa)
-            if rc:
-                raise lnq.LnqError(rc, "quantize")
-            if ev is not None:
-                ev[2 * i + 1].record(stream)
-            rc = gf(*ga)
-            if rc:
-                raise lnq.LnqError(rc, "gemm")
-        if ev is not None:
-            ev[2 * n_units].record(stream)
-
-    for _ in range(args.warmup):
-        launch_step()
-    torch.cuda.synchronize()
-    if lnq.lnq_get_last_device_error() != 0:
-        raise RuntimeError("device reported an error during warm-up")
-
-    # ---- timed region (device time, CUDA events on the launching stream).  Events only
-    # bracket the K steps: an event between two kernels would stop the next one from
-    # starting early (programmatic dependent launch), so the per-kernel times come from
-    # a second timed loop below.
-    K = args.steps
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    barrier(dist)
-    torch.cuda.synchronize()
-    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
-        t0.record(stream)
-        for k in range(K):
-            launch_step()
-        t1.record(stream)
-        torch.cuda.synchronize()
-    barrier(dist)
-    ms_local = t0.elapsed_time(t1)
-    if lnq.lnq_get_last_device_error() != 0:
-        raise RuntimeError("device reported an error in the timed region")
-    ms = max_over_ranks(ms_local, dist, dev)
-
-    # ---- per-kernel times: K more steps with an event around every kernel
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_units + 1)] for _ in range(K)]
-    torch.cuda.synchronize()
-    for k in range(K):
-        launch_step(evs[k])
-    torch.cuda.synchronize()
-    q_ms = sum(evs[k][2 * i].elapsed_time(evs[k][2 * i + 1]) for k in range(K) for i in range(n_units))
-    g_ms = sum(evs[k][2 * i + 1].elapsed_time(evs[k][2 * i + 2]) for k in range(K)
-               for i in range(n_units))
-    per_gemm = [statistics.mean(evs[k][2 * i + 1].elapsed_time(evs[k][2 * i + 2]) for k in range(K))
-                for i in range(n_units)]
-    per_quant = [statistics.mean(evs[k][2 * i].elapsed_time(evs[k][2 * i + 1]) for k in range(K))
-                 for i in range(n_units)]
-
-    # ---- end to end through the public API: host inputs in, host outputs back
-    e2e = None
-    if not args.no_e2e:
-        Ke = max(1, min(K, args.e2e_steps))
-        for u in units:                       # warm the copy paths
-            u.x.copy_(u.host_x, non_blocking=True)
-            u.copy_out()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        barrier(dist)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(Ke):
-            for u, ((qf, qa), (gf, ga)) in zip(units, calls):
-                u.x.copy_(u.host_x, non_blocking=True)
-                rc = qf(*qa) or gf(*ga)
-                if rc:
-                    raise lnq.LnqError(rc, "e2e")
-                u.copy_out()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier(dist)
-        e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
-        if is_hbm_bound(args.workload):
-            ev_val = job_throughput(bytes_step, Ke, world, e_ms, 1e9)
-            ev_unit = "GB/s"
-        else:
-            ev_val = job_throughput(flops_step, Ke, world, e_ms, 1e12)
-            ev_unit = "TFLOP/s"
-        e2e = {"value": round(ev_val, 3), "unit": ev_unit, "steps": Ke,
-               "h2d_bytes_per_step": int(sum(u.h2d_bytes for u in units)),
-               "d2h_bytes_per_step": int(sum(u.d2h_bytes for u in units)),
-               "note": "pinned host bf16 activations copied in and bf16 outputs copied back "
-                       "every step; weights resident (model parameters)"}
-
-    # ---- numbers
-    peaks, peak_src = load_peaks()
-    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
-    if is_hbm_bound(args.workload):
-        value = job_throughput(bytes_step, K, world, ms, 1e9)
-        unit = "GB/s"
-        ach = bytes_step * K / (g_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(ach / peaks["hbm_gbs"], 4)}
-        peak_note = f"HBM copy bandwidth ({peak_src})"
-    else:
-        value = job_throughput(flops_step, K, world, ms, 1e12)
-        unit = "TFLOP/s"
-        ach = flops_step * K / (g_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1),
-                "unit": "TFLOP/s", "frac": round(ach / fp8_peak, 4)}
-        peak_note = (f"dense FP8 = {FP8_OVER_BF16:g} x bf16 cuBLAS burst {peaks['bf16_tflops']} "
-                     f"TFLOP/s ({peak_src})")
-    ue8m0 = any(getattr(u, "ue8m0", False) for u in units)
-    kernel_name = "k_mx_block_gemm" if ue8m0 else "k_fp8_block_gemm"
-    traffic = recorded_traffic(kernel_name, args.workload)
-    roof["traffic"] = traffic
-    roof["kernel"] = kernel_name
-    roof["peak_source"] = peak_note
-    roof["algorithmic_per_launch"] = ({"bytes": [int(u.gemm_bytes) for u in units]}
-                                      if is_hbm_bound(args.workload)
-                                      else {"flops": [float(u.flops) for u in units]})
-    quant_gbs = sum(u.quant_bytes for u in units) * K / (q_ms * 1e-3) / 1e9
-
+    names = list(ALL_WORKLOADS) if args.workload == "all" else [args.workload]
+    results = {}
+    for name in names:
+        share = args.cpu_seconds if len(names) == 1 else (
+            args.cpu_seconds / 2 if name == names[0] else args.cpu_seconds / (2 * (len(names) - 1)))
+        results[name] = measure_workload(name, args, dev, dist, world, rank, share)
+    head_name = names[0]
+    head = results[head_name]
     out = {
         "metric": METRIC,
-        "value": round(value, 3),
-        "unit": unit,
+        "value": head["value"],
+        "unit": head["unit"],
         "n_gpus": world,
-        "steps": K,
+        "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms / K, 5),
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": ("e4m3 x e4m3 with UE8M0 block scales -> f32 accumulate, bf16 out" if ue8m0
+        "dtype": ("e4m3 x e4m3 with UE8M0 block scales -> f32 accumulate, bf16 out" if args.recipe == "ue8m0"
                   else "e4m3 x e4m3 -> f32 accumulate, bf16 out"),
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, bf16)",
-        "config": {"workload": args.workload, "desc": WORKLOAD_DESC[args.workload],
+        "config": {"workload": (f"{head_name} (headline; every workload under `configs`)"
+                                if len(names) > 1 else head_name),
+                   "desc": head["desc"],
+                   "workloads": names,
                    "dense_cta_pairs": args.cta_pairs,
                    "grouped_cta_pairs": args.grouped_cta_pairs,
                    "weight_prefetch": not args.no_weight_prefetch,
-                   "decode_k_split": args.split and any(getattr(u, "work", None) is not None
-                                                         for u in units),
-                   "epilogue": ("fp8 output (E4M3 + 1x128 scales)" if any(getattr(u, "fp8_out", False) for u in units)
-                                else "gate_up with SiLU.mul (bf16 h)" if any(getattr(u, "silu", False) for u in units)
-                                else "bf16 output"),
-                   "recipe": ("UE8M0 power-of-two scales in the tensor core" if ue8m0
-                              else "FP32 scales, per-128-K-block promotion"),
+                   "decode_k_split": head["decode_k_split"],
+                   "epilogue": head["epilogue"],
+                   "recipe": head["recipe"],
                    "parallelism": f"replicas x{world} (independent tokens per rank)",
-                   "l2": "working set per step > 126 MB L2; no extra flush"},
-        "roofline": roof,
-        "kernels": {
-            "gemm_ms_per_launch": [round(x, 5) for x in per_gemm],
-            "quantize_ms_per_launch": [round(x, 5) for x in per_quant],
-            "quantize_gbs": round(quant_gbs, 1),
-            "quantize_frac_of_hbm": round(quant_gbs / peaks["hbm_gbs"], 4),
-            "gemm_share_of_step": round(g_ms / (g_ms + q_ms), 4),
-        },
-        "gpu_launches": K * 2 * n_units,
-        "timing": "value: K steps between two events (kernels chained by programmatic dependent "
-                  "launch); roofline and kernels: K further steps with an event around each kernel",
-        "clocks": clocks.summary(),
-        "e2e": e2e,
+                   "l2": head["l2"]},
+        "roofline": head["roofline"],
+        "kernels": head["kernels"],
+        "gpu_launches": head["gpu_launches"],
+        "timing": ("value: K steps between two events (kernels chained by programmatic dependent "
+                   "launch), max over ranks; roofline: the GEMMs alone back to back, mean period per "
+                   "launch; kernels: each kernel between its own events over max(K, 50) steps "
+                   "(min, median)"),
+        "clocks": head["clocks"],
+        "e2e": head["e2e"],
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args.workload, target_s=args.cpu_seconds)
+    if "cpu_baseline" in head:
+        out["cpu_baseline"] = head["cpu_baseline"]
+    if len(names) > 1:
+        out["configs"] = {n: {k: v for k, v in r.items() if k not in ("desc",)} | {"desc": r["desc"]}
+                          for n, r in results.items()}
+        out["gpu_launches_all_workloads"] = sum(r["gpu_launches"] for r in results.values())
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist is not None:
@@ -726,29 +831,37 @@ def cpu_baseline(workload: str, target_s: float = 10.0):
                       f"(quantize + FP64 product, weights pre-quantized), {dt:.2f} s"}
 
 
+def reference_sample(workload: str, steps: int, warmup: int):
+    """The oracle on one bounded sample per step: the first 16 activation rows x the first
+    1024 output columns of every linear of the workload (fewer where it has fewer)."""
+    rows, cols = 16, 1024
+    items = oracle_sample(oracle_inputs(workload, rows), rows, cols)
+    for _ in range(warmup):
+        oracle_step(items)
+    t = time.perf_counter()
+    for _ in range(steps):
+        oracle_step(items)
+    dt = time.perf_counter() - t
+    flops, byts = measure_oracle(items, dt, steps)
+    if is_hbm_bound(workload):
+        val, unit = byts / dt / 1e9, "GB/s"
+    else:
+        val, unit = flops / dt / 1e12, "TFLOP/s"
+    return val, unit, dt / steps * 1e3, (f"first {rows} activation rows x first {cols} output columns of "
+                                         f"each linear per step (quantize + FP64 product, weights "
+                                         f"pre-quantized)")
+
+
 def run_reference(args, world, rank, local):
     """The reference arm: the CPU oracle on a bounded sample, on rank 0 only."""
     if rank != 0:
         return
     import oracle
     oracle.build()
-    # each step: the first 16 activation rows x the first 1024 output columns of every
-    # linear of the workload (fewer where the workload has fewer)
-    rows, cols = 16, 1024
-    items = oracle_sample(oracle_inputs(args.workload, rows), rows, cols)
-    for _ in range(args.warmup):
-        oracle_step(items)
-    t = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(items)
-    dt = time.perf_counter() - t
-    flops, byts = measure_oracle(items, dt, args.steps)
-    if is_hbm_bound(args.workload):
-        val, unit = byts / dt / 1e9, "GB/s"
-    else:
-        val, unit = flops / dt / 1e12, "TFLOP/s"
-    sample = (f"first {rows} activation rows x first {cols} output columns of each linear per step "
-              f"(quantize + FP64 product, weights pre-quantized)")
+    names = list(ALL_WORKLOADS) if args.workload == "all" else [args.workload]
+    results = {n: reference_sample(n, args.steps, args.warmup) for n in names}
+    val, unit, ms_step, sample = results[names[0]]
+    cores = oracle.num_threads()
     out = {
         "impl": "reference",
         "metric": METRIC,
@@ -757,28 +870,37 @@ def run_reference(args, world, rank, local):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": dt / args.steps * 1e3,
+        "ms_per_step": ms_step,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded)",
-        "config": {"workload": args.workload, "desc": WORKLOAD_DESC[args.workload]},
-        "cpu_baseline": {"value": val, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": sample},
+        "config": {"workload": (f"{names[0]} (headline; every workload under `configs`)"
+                                if len(names) > 1 else names[0]),
+                   "desc": WORKLOAD_DESC[names[0]], "workloads": names},
+        "cpu_baseline": {"value": val, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+    if len(names) > 1:
+        out["configs"] = {n: {"value": v, "unit": u, "ms_per_step": m, "desc": WORKLOAD_DESC[n],
+                              "cpu_baseline": {"value": v, "unit": u, "cores": cores, "kind": "oracle",
+                                               "sample": smp}}
+                          for n, (v, u, m, smp) in results.items()}
     print(json.dumps(out), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["prefill", "decode", "moe", "moe_psum", "moe_masked", "square", "tiny"],
-                    default="prefill")
+    ap.add_argument("--workload", choices=["all", "prefill", "decode", "moe", "moe_psum", "moe_masked", "square",
+                                           "tiny"],
+                    default="all", help="all (the default): square (headline), prefill, decode and moe")
+    ap.add_argument("--kernel-reps", type=int, default=50,
+                    help="repetitions of the per-kernel timing loops (at least the number of steps)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)

@@ -20,19 +20,23 @@ REL_MAX = 2e-2
 MASK_FRAC = 1e-2
 
 
-def gemm_errors(d: np.ndarray, ref: np.ndarray):
+def gemm_errors(d: np.ndarray, ref: np.ndarray, ref_absmax: float | None = None):
+    """(Frobenius relative error, max relative error over the masked elements).  The mask
+    keeps |D_ref| > 1e-2 * max|D_ref|, the max taken over the whole product: pass
+    `ref_absmax` when d and ref are a part of it (rows of a grouped product)."""
     d = np.asarray(d, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert d.shape == ref.shape
     assert np.all(np.isfinite(d)), "non-finite output"
     fro = np.linalg.norm(d - ref) / max(np.linalg.norm(ref), 1e-300)
-    mask = np.abs(ref) > MASK_FRAC * np.abs(ref).max()
+    top = np.abs(ref).max() if ref_absmax is None else ref_absmax
+    mask = np.abs(ref) > MASK_FRAC * top
     mx = float((np.abs(d - ref)[mask] / np.abs(ref)[mask]).max()) if mask.any() else 0.0
     return float(fro), mx
 
 
-def assert_gemm_close(d, ref, what=""):
-    fro, mx = gemm_errors(d, ref)
+def assert_gemm_close(d, ref, what="", ref_absmax: float | None = None):
+    fro, mx = gemm_errors(d, ref, ref_absmax)
     assert fro <= REL_FRO, f"{what}: Frobenius relative error {fro:.3e} > {REL_FRO}"
     assert mx <= REL_MAX, f"{what}: max relative error {mx:.3e} > {REL_MAX}"
     return fro, mx

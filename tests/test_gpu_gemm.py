@@ -2,10 +2,14 @@
 
 The oracle quantizes the same seeded bf16 inputs itself and computes D in FP64;
 the CUDA path quantizes with its own kernels (bit-exact with the oracle, see
-test_gpu_quantize) and multiplies.  Small and ragged shapes are compared element
-by element; the full workloads, in the launch configuration the benchmark times,
-on sampled points (random points plus one whole row and one whole column).
+test_gpu_quantize) and multiplies.  Every output is compared element by element
+over the whole of D: the small and ragged shapes, a shape of many more tiles than
+SMs (so every persistent CTA runs several tiles), and the full workloads in every
+launch configuration (the benchmark's included); the full-size references are
+computed once per session (full_refs).
 """
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -13,7 +17,8 @@ import torch
 import moe_grouped_gemm_quantize_b200 as lnq
 import oracle
 from moe_grouped_gemm_quantize_b200 import synthetic
-from parity import assert_gemm_close, codes, oracle_quantize_a, oracle_quantize_w, sample_points, to_f64
+import full_refs
+from parity import assert_gemm_close, codes, oracle_quantize_a, oracle_quantize_w, to_f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -110,37 +115,46 @@ def test_deterministic():
     assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
 
 
-def check_sampled(a, w, what, count=20000, seed=0):
+def check_workload(name, what=None):
+    """The named workload's whole D against its cached full oracle reference."""
+    a, w = full_refs.linear_inputs(name)
     d, _ = gpu_linear(a, w)
-    qa, sa = oracle_quantize_a(a)
-    qb, sb = oracle_quantize_w(w)
-    M, N = d.shape
-    rows, cols = sample_points(M, N, count, seed, full_row=M - 1, full_col=N // 2 + 1)
-    ref = oracle.gemm_nt_points(qa, sa, qb, sb, rows, cols)
-    got = to_f64(d)[rows, cols]
-    return assert_gemm_close(got, ref, what)
+    return assert_gemm_close(to_f64(d), full_refs.linear_ref(name), what or name)
 
 
 @pytest.mark.parametrize("idx", range(4))
-def test_prefill_workloads_sampled(idx, dense_pairs):
-    cfg = synthetic.PREFILL[idx]
-    a, w = synthetic.make_linear_inputs(cfg)
-    check_sampled(a, w, cfg.name)
+def test_prefill_workloads_full(idx, dense_pairs):
+    check_workload(synthetic.PREFILL[idx].name)
 
 
-def test_decode_workloads(weight_prefetch):
-    for cfg in synthetic.DECODE:
-        a, w = synthetic.make_linear_inputs(cfg)
-        if cfg.M <= 8:
-            check_full(a, w, cfg.name)
-        else:
-            check_sampled(a, w, cfg.name)
+@pytest.mark.parametrize("idx", range(4))
+def test_decode_workloads_full(idx, weight_prefetch):
+    check_workload(synthetic.DECODE[idx].name)
 
 
-def test_square_outlier_workload_sampled(dense_pairs):
-    cfg = synthetic.SQUARE
-    a, w = synthetic.make_linear_inputs(cfg)
-    check_sampled(a, w, cfg.name, count=30000)
+def test_square_outlier_workload_full(dense_pairs):
+    check_workload(synthetic.SQUARE.name)
+
+
+@functools.lru_cache(maxsize=None)
+def many_tiles_case():
+    # 4096 x 8192 output at K = 256: 1024 tiles of 128 x 256 (512 CTA-pair tiles of
+    # 256 x 256), several per persistent CTA, so the accumulator ring, its phases and the
+    # tile boundary are exercised under an element-by-element check
+    M, N, K = 4096, 8192, 256
+    a = synthetic.gaussian_bf16((M, K), 1.0, seed=401)
+    w = synthetic.gaussian_bf16((N, K), 0.02, seed=402)
+    qa, sa = oracle_quantize_a(a)
+    qb, sb = oracle_quantize_w(w)
+    return a, w, oracle.gemm_nt(qa, sa, qb, sb)
+
+
+def test_many_tiles_per_cta_elementwise(dense_pairs, weight_prefetch):
+    a, w, ref = many_tiles_case()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert (a.shape[0] // 256) * (w.shape[0] // 256) > 3 * sms // 2
+    d, _ = gpu_linear(a, w)
+    assert_gemm_close(to_f64(d), ref, f"many tiles, configuration {dense_pairs}")
 
 
 def test_timeout_path_reports_and_recovers():
@@ -199,18 +213,10 @@ def test_decode_split_is_deterministic_and_reuses_its_workspace():
 
 def test_decode_split_workloads(weight_prefetch):
     for cfg in synthetic.DECODE:
-        a, w = synthetic.make_linear_inputs(cfg)
+        a, w = full_refs.linear_inputs(cfg.name)
         d, work, (aq, sa, wq, ws) = gpu_linear_split(a, w)
         assert work is not None
-        qa, sao = oracle_quantize_a(a)
-        qb, sbo = oracle_quantize_w(w)
-        if cfg.M <= 8:
-            ref = oracle.gemm_nt(qa, sao, qb, sbo)
-            assert_gemm_close(to_f64(d), ref, cfg.name + " split")
-        else:
-            rows, cols = sample_points(cfg.M, cfg.N, 20000, 0, full_row=cfg.M - 1, full_col=cfg.N // 2 + 1)
-            ref = oracle.gemm_nt_points(qa, sao, qb, sbo, rows, cols)
-            assert_gemm_close(to_f64(d)[rows, cols], ref, cfg.name + " split")
+        assert_gemm_close(to_f64(d), full_refs.linear_ref(cfg.name), cfg.name + " split")
         torch.cuda.synchronize()
         assert counters_zero(work, cfg.M, cfg.N)
 
@@ -268,7 +274,6 @@ def test_one_workspace_serves_products_of_different_shapes():
         assert lnq.lnq_get_last_device_error() == 0
         qa, sao = oracle_quantize_a(a)
         qb, sbo = oracle_quantize_w(w)
-        rows, cols = sample_points(M, N, 4000, i, full_row=M - 1, full_col=N // 2)
-        ref = oracle.gemm_nt_points(qa, sao, qb, sbo, rows, cols)
-        assert_gemm_close(to_f64(d)[rows, cols], ref, f"shared workspace {M}x{N}x{K}")
+        ref = oracle.gemm_nt(qa, sao, qb, sbo)
+        assert_gemm_close(to_f64(d), ref, f"shared workspace {M}x{N}x{K}")
         assert counters_zero(work, M, N)

@@ -2,9 +2,9 @@
 
 Layout (deepgemm-rust README, "Grouped (contiguous) MoE GEMM"; Triton_Grouped_GEMM
 README, "Example DeepGEMM layout creation"): each group's rows start at a multiple
-of 128, pad rows carry id -1.  Rows of real tokens are compared with the oracle;
-pad rows inside a block are unspecified; blocks whose first row is -1 must not be
-written at all.
+of 128, pad rows carry id -1.  Rows of real tokens are compared with the oracle
+element by element (all of them at the MoE workload size); pad rows inside a block
+are unspecified; blocks whose first row is -1 must not be written at all.
 """
 import numpy as np
 import pytest
@@ -13,7 +13,8 @@ import torch
 import moe_grouped_gemm_quantize_b200 as lnq
 import oracle
 from moe_grouped_gemm_quantize_b200 import synthetic
-from parity import assert_gemm_close, oracle_quantize_a, oracle_quantize_w, sample_points, to_f64
+import full_refs
+from parity import assert_gemm_close, oracle_quantize_a, oracle_quantize_w, to_f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -90,16 +91,14 @@ def test_single_group_equals_dense():
     assert np.array_equal(d, to_f64(dd))
 
 
-def test_moe_workload_sampled():
+def test_moe_workload_full():
+    # every token row of the 32-expert MoE workload, element by element
     cfg = synthetic.MOE
-    a, w, m_indices, sizes = synthetic.make_moe_inputs(cfg)
-    G = cfg.groups
-    d = run_gpu(a, w, m_indices, G)
-    qa, sa = oracle_quantize_a(a)
-    qb, sb = oracle_quantize_w_grouped(w, G)
-    real_rows = np.nonzero(m_indices >= 0)[0]
-    rows, cols = sample_points(real_rows.size, cfg.N, 30000, seed=1, full_row=real_rows.size - 1,
-                               full_col=cfg.N - 1)
-    rows = real_rows[rows]
-    ref = oracle.m_grouped_gemm_points(qa, sa, qb, sb, m_indices, G, rows, cols)
-    assert_gemm_close(d[rows, cols], ref, cfg.name)
+    a, w, m_indices, _, _ = full_refs.moe_inputs()
+    d = run_gpu(a, w, m_indices, cfg.groups)
+    ref = full_refs.moe_ref()
+    real = m_indices >= 0
+    assert np.array_equal(real, ~np.isnan(ref[:, 0]))
+    assert_gemm_close(d[real], ref[real], cfg.name)
+    led_by_pad = np.repeat(m_indices[::128] < 0, 128)
+    assert np.all(np.isnan(d[led_by_pad]))

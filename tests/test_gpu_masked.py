@@ -3,7 +3,7 @@
 Layout (deepgemm-rust README, "What's implemented", m_grouped_fp8_gemm_nt_masked):
 every group has a buffer of M_max rows of which the first masked_m[g] hold tokens;
 the counts stay on the device.  Rows of real tokens are compared with the oracle
-element by element (or on sampled points at the workload size); the other rows of
+element by element (all of them at the workload size); the other rows of
 D must keep what was there before the call.  The rows past a count hold random
 values, which must not reach any real row.
 """
@@ -14,7 +14,8 @@ import torch
 import moe_grouped_gemm_quantize_b200 as lnq
 import oracle
 from moe_grouped_gemm_quantize_b200 import synthetic
-from parity import assert_gemm_close, oracle_quantize_a, oracle_quantize_w, sample_points, to_f64
+import full_refs
+from parity import assert_gemm_close, oracle_quantize_a, oracle_quantize_w, to_f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -66,8 +67,10 @@ def test_masked_elementwise(masked, M_max, N, K):
     assert np.all(np.isnan(got[~valid]))
 
 
-def test_decode_moe_workload_sampled():
-    # 32 experts with 128-row buffers, 2048 routed tokens (multinomial, seed 3)
+def test_decode_moe_workload_full():
+    # 32 experts with 128-row buffers, 2048 routed tokens (multinomial, seed 3): every
+    # token row is compared, each group's rows with the dense oracle product of its
+    # weights (the definition of the masked product)
     G, M_max, N, K = 32, 128, 4096, 7168
     counts = np.minimum(np.random.default_rng(3).multinomial(2048, [1.0 / G] * G), M_max)
     masked = [int(c) for c in counts]
@@ -76,13 +79,11 @@ def test_decode_moe_workload_sampled():
     assert lnq.lnq_get_last_device_error() == 0
     qa, sa = oracle_quantize_a(a)
     qb, sb = oracle_quantize_w_grouped(w, G)
+    starts = np.arange(G) * M_max
+    ref = full_refs.grouped_ref(qa, sa, qb, sb, starts, masked, N)
     real = np.concatenate([np.arange(g * M_max, g * M_max + c) for g, c in enumerate(masked)])
-    rng = np.random.default_rng(5)
-    rows = rng.choice(real, 20000)
-    cols = rng.integers(0, N, 20000)
-    ref = oracle.m_grouped_gemm_masked_points(qa, sa, qb, sb, masked, M_max, rows, cols)
     got = to_f64(d)
-    assert_gemm_close(got[rows, cols], ref, "masked decode MoE")
+    assert_gemm_close(got[real], ref[real], "masked decode MoE")
     pad = np.setdiff1d(np.arange(G * M_max), real)
     assert np.all(np.isnan(got[pad]))
 

@@ -9,11 +9,11 @@ by the block-scaled MMA) and "What's implemented" (gran-128 on either side).
   layout.  Pad rows of the last block carry the byte of p = 1.
 * The GEMM (tcgen05.mma kind::mxf8f6f4.block_scale) is compared with the oracle's FP64
   product of the same codes and power-of-two scales, within the GEMM tolerance, element by
-  element on ragged shapes and at sampled points on a prefill linear.
+  element on ragged shapes and over the whole output of a prefill linear.
 * The M-grouped contiguous form (each 128-row block takes the group of its first row) is
   compared with the oracle's grouped product on rows with a group id, element by element on
-  small layouts and at sampled points on the 32-expert MoE workload; blocks led by -1 stay
-  untouched.
+  small layouts and on every token row of the 32-expert MoE workload; blocks led by -1
+  stay untouched.
 """
 import numpy as np
 import pytest
@@ -22,6 +22,7 @@ import torch
 import moe_grouped_gemm_quantize_b200 as lnq
 import oracle
 from moe_grouped_gemm_quantize_b200 import synthetic
+import full_refs
 from parity import assert_gemm_close, codes, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -94,18 +95,12 @@ def test_gemm_elementwise(M, N, K):
     assert_gemm_close(to_f64(d), oracle_gemm(a, w), f"ue8m0 {M}x{N}x{K}")
 
 
-def test_gemm_prefill_sampled():
+def test_gemm_prefill_full():
     cfg = synthetic.PREFILL[0]
-    a, w = synthetic.make_linear_inputs(cfg)
+    a, w = full_refs.linear_inputs(cfg.name)
     d = run_gemm(a, w)
     assert lnq.lnq_get_last_device_error() == 0
-    qa, ea = oracle.quantize_ue8m0_groups(synthetic.bf16_bits(a))
-    qb, eb = oracle.quantize_ue8m0_blocks(synthetic.bf16_bits(w))
-    rng = np.random.default_rng(17)
-    rows = np.concatenate([rng.integers(0, cfg.M, 20000), np.full(cfg.N, 7)])
-    cols = np.concatenate([rng.integers(0, cfg.N, 20000), np.arange(cfg.N)])
-    ref = oracle.gemm_nt_points(qa, oracle.ue8m0_value(ea), qb, oracle.ue8m0_value(eb), rows, cols)
-    assert_gemm_close(to_f64(d)[rows, cols], ref, "ue8m0 prefill QKV")
+    assert_gemm_close(to_f64(d), oracle_gemm(a, w), "ue8m0 prefill QKV")
 
 
 def test_repeated_runs_are_identical():
@@ -144,17 +139,15 @@ def test_grouped_elementwise(sizes, N, K):
     assert np.all(np.isnan(got[led_by_pad]))
 
 
-def test_grouped_moe_workload_sampled():
+def test_grouped_moe_workload_full():
+    # every token row of the 32-expert MoE workload; each group's rows against the
+    # dense oracle product with its weights and power-of-two scales
     cfg = synthetic.MOE
-    a, w, m_indices, sizes = synthetic.make_moe_inputs(cfg)
+    a, w, m_indices, sizes, starts = full_refs.moe_inputs()
     d = run_grouped(a, w, m_indices, cfg.groups)
     assert lnq.lnq_get_last_device_error() == 0
     qa, ea = oracle.quantize_ue8m0_groups(synthetic.bf16_bits(a))
     qb, eb = oracle.quantize_ue8m0_blocks(synthetic.bf16_bits(w))
-    rng = np.random.default_rng(23)
-    real = np.flatnonzero(m_indices >= 0)
-    rows = rng.choice(real, 20000)
-    cols = rng.integers(0, cfg.N, 20000)
-    ref = oracle.m_grouped_gemm_points(qa, oracle.ue8m0_value(ea), qb, oracle.ue8m0_value(eb), m_indices,
-                                       cfg.groups, rows, cols)
-    assert_gemm_close(to_f64(d)[rows, cols], ref, "ue8m0 MoE workload")
+    ref = full_refs.grouped_ref(qa, oracle.ue8m0_value(ea), qb, oracle.ue8m0_value(eb), starts, sizes, cfg.N)
+    real = m_indices >= 0
+    assert_gemm_close(to_f64(d)[real], ref[real], "ue8m0 MoE workload")

@@ -5,9 +5,9 @@ sum of the earlier groups' counts rounded up to the alignment (deepgemm-rust REA
 "The mk_alignment knob (MoE tile width)", and its psum-layout contiguous entry point).
 Tiles are 128 rows, those of pad rows only skipped; with alignment 256, N >= 256 and
 the grouped pairs knob set, 256 x 256 tiles on CTA pairs.  Both schedules run every
-case.  Token rows are
-compared with the oracle element by element (sampled points at the workload size);
-pad rows and rows past the last group must keep what was there before the call.
+case.  Token rows are compared with the oracle element by element (all of them at the
+workload size); pad rows and rows past the last group must keep what was there
+before the call.
 """
 import numpy as np
 import pytest
@@ -16,6 +16,7 @@ import torch
 import moe_grouped_gemm_quantize_b200 as lnq
 import oracle
 from moe_grouped_gemm_quantize_b200 import synthetic
+import full_refs
 from parity import assert_gemm_close, oracle_quantize_a, oracle_quantize_w, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -115,29 +116,25 @@ def test_128_alignment_matches_the_group_id_layout_bit_for_bit():
 
 
 @pytest.mark.parametrize("pairs", [0, 1])
-def test_moe_workload_sampled(pairs):
-    # 32 experts, 16384 routed tokens (multinomial, seed 0), 256-row alignment
+def test_moe_workload_full(pairs):
+    # the 32-expert MoE workload (16384 tokens, multinomial seed 0) moved into the
+    # prefix-sum arena with 256-row alignment: every token row is compared with the
+    # group-id layout's full reference (the same tokens, the same weights)
     cfg = synthetic.MOE
-    sizes = cfg.group_sizes()
+    a128, w, _, sizes, starts128 = full_refs.moe_inputs()
     G, N, K = cfg.groups, cfg.N, cfg.K
     psum, starts, M_total = synthetic.psum_layout(sizes, 256)
-    a = synthetic.gaussian_bf16((M_total, K), 1.0, seed=cfg.a_seed)
-    w = synthetic.gaussian_bf16((G * N, K), 0.02, seed=cfg.w_seed)
+    a = torch.zeros((M_total, K), dtype=torch.bfloat16)
+    src = np.concatenate([np.arange(s, s + n) for s, n in zip(starts128, sizes)])
+    dst = np.concatenate([np.arange(s, s + n) for s, n in zip(starts, sizes)])
+    a[torch.from_numpy(dst)] = a128[torch.from_numpy(src)]
     d = run_gpu(a, w, psum, 256, G, pairs)
     assert lnq.lnq_get_last_device_error() == 0
-    qa, sa = oracle_quantize_a(a)
-    qb, sb = oracle_quantize_w_grouped(w, G)
-    real = token_rows(sizes, starts)
-    owner = np.full(M_total, -1, np.int32)
-    for g, (s, n) in enumerate(zip(starts, sizes)):
-        owner[s:s + n] = g
-    rng = np.random.default_rng(9)
-    rows = rng.choice(real, 20000)
-    cols = rng.integers(0, N, 20000)
-    ref = oracle.m_grouped_gemm_points(qa, sa, qb, sb, owner, G, rows, cols)
+    ref = full_refs.moe_ref()
     got = to_f64(d)
-    assert_gemm_close(got[rows, cols], ref, "psum MoE workload")
-    pad = np.setdiff1d(np.arange(M_total), real)
+    assert np.array_equal(np.sort(dst), token_rows(sizes, starts))
+    assert_gemm_close(got[dst], ref[src], f"psum MoE workload, pairs={pairs}")
+    pad = np.setdiff1d(np.arange(M_total), dst)
     assert np.all(np.isnan(got[pad][:, :64]))
 
 
