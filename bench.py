@@ -484,19 +484,27 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
     """Everything the bench reports for one workload, as a dict (the same keys as the
     top-level JSON line, without `metric`).
 
-    * value: the step (quantize + GEMM of every linear) over K steps between two events,
-      with every kernel chained by programmatic dependent launch; max over ranks.
-    * kernels: each kernel between its own two events, over max(K, 50) steps (min and
-      median per launch); and the GEMMs alone back to back (chained as in the step, no
-      quantize between them), over the same number of repetitions: their mean period
-      per launch is the duration `roofline.achieved` divides by.
-    * e2e: the step through the public calls with the bf16 activations copied in from
-      pinned host memory and the outputs copied back, every step.
+    * value: the step (quantize + GEMM of every linear) captured once in a CUDA graph
+      and replayed K times between two events, every kernel chained by programmatic
+      dependent launch; max over ranks.
+    * kernels: each kernel alone, a graph of that one launch replayed max(K, 50) times,
+      each replay between its own two events (min and median per launch); and the GEMMs
+      alone, max(K, 50) rounds of the workload's GEMMs back to back in one graph (chained
+      as in the step, no quantize between them): their mean period per launch is the
+      duration `roofline.achieved` divides by.  Graphs keep the host's launch cost (the
+      argument marshalling and tensor-map encoding of each C-ABI call) out of the
+      device timeline, which would otherwise starve the GPU on the microsecond decode
+      kernels.
+    * e2e: the step through the public calls, issued from the host every step (no graph),
+      with the bf16 activations copied in from pinned host memory and the outputs
+      copied back.
     """
     import moe_grouped_gemm_quantize_b200 as lnq
 
     units = make_units(name, args, dev)
-    stream = torch.cuda.current_stream(dev)
+    # every call is marshalled for one dedicated stream, on which the graphs are captured
+    # and replayed
+    stream = torch.cuda.Stream(dev)
     calls = [u.calls(stream.cuda_stream) for u in units]
     n_units = len(units)
     flops_step = sum(u.flops for u in units)
@@ -509,16 +517,16 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
         if rc:
             raise lnq.LnqError(rc, f"{name} {what}")
 
-    def launch_step(ev=None):
-        for i, (q, g) in enumerate(calls):
-            if ev is not None:
-                ev[2 * i].record(stream)
+    def launch_step():
+        for q, g in calls:
             run(q, "quantize")
-            if ev is not None:
-                ev[2 * i + 1].record(stream)
             run(g, "gemm")
-        if ev is not None:
-            ev[2 * n_units].record(stream)
+
+    def capture(fn):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            fn()
+        return graph
 
     for _ in range(args.warmup):
         launch_step()
@@ -528,15 +536,28 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
 
     K = args.steps
     R = max(K, args.kernel_reps)
+    g_step = capture(launch_step)
+    g_chain = capture(lambda: [run(g, "gemm") for _ in range(R) for _, g in calls])
+    g_quant = [capture(lambda q=q: run(q, "quantize")) for q, _ in calls]
+    g_gemm = [capture(lambda g=g: run(g, "gemm")) for _, g in calls]
+    torch.cuda.synchronize()
+
+    def replay(graph, times=1):
+        with torch.cuda.stream(stream):
+            for _ in range(times):
+                graph.replay()
+
+    replay(g_step, 3)
+    replay(g_chain)
+    torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
-        # ---- the timed region: K steps between two events on the launching stream
+        # ---- the timed region: K replays of the step between two events on its stream
         barrier(dist)
         torch.cuda.synchronize()
         t0.record(stream)
-        for _ in range(K):
-            launch_step()
+        replay(g_step, K)
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(dist)
@@ -544,31 +565,37 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
         if lnq.lnq_get_last_device_error() != 0:
             raise RuntimeError(f"{name}: device reported an error in the timed region")
 
-        # ---- each kernel between its own events (no overlap with its neighbours)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_units + 1)] for _ in range(R)]
+        # ---- each kernel alone, between its own events
+        per_gemm = [[] for _ in range(n_units)]
+        per_quant = [[] for _ in range(n_units)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4 * n_units)] for _ in range(R)]
+        for r in range(R):
+            e = evs[r]
+            for i in range(n_units):
+                e[4 * i].record(stream)
+                replay(g_quant[i])
+                e[4 * i + 1].record(stream)
+                e[4 * i + 2].record(stream)
+                replay(g_gemm[i])
+                e[4 * i + 3].record(stream)
         torch.cuda.synchronize()
         for r in range(R):
-            launch_step(evs[r])
-        torch.cuda.synchronize()
-        per_gemm = [[evs[r][2 * i + 1].elapsed_time(evs[r][2 * i + 2]) for r in range(R)] for i in range(n_units)]
-        per_quant = [[evs[r][2 * i].elapsed_time(evs[r][2 * i + 1]) for r in range(R)] for i in range(n_units)]
+            for i in range(n_units):
+                per_quant[i].append(evs[r][4 * i].elapsed_time(evs[r][4 * i + 1]))
+                per_gemm[i].append(evs[r][4 * i + 2].elapsed_time(evs[r][4 * i + 3]))
 
-        # ---- the GEMMs alone, back to back as the step chains them
-        for _ in range(3):
-            for _, g in calls:
-                run(g, "gemm")
+        # ---- the GEMMs alone, R rounds back to back as the step chains them
         c0 = torch.cuda.Event(enable_timing=True)
         c1 = torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         c0.record(stream)
-        for _ in range(R):
-            for _, g in calls:
-                run(g, "gemm")
+        replay(g_chain)
         c1.record(stream)
         torch.cuda.synchronize()
         chained_ms = c0.elapsed_time(c1)
         if lnq.lnq_get_last_device_error() != 0:
             raise RuntimeError(f"{name}: device reported an error in the kernel loops")
+    del g_step, g_chain, g_quant, g_gemm
     ms = max_over_ranks(ms_local, dist, dev)
     chained_ms = max_over_ranks(chained_ms, dist, dev)
 
@@ -576,21 +603,23 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
     e2e = None
     if not args.no_e2e:
         Ke = max(1, min(K, args.e2e_steps))
-        for u in units:                       # warm the copy paths
-            u.x.copy_(u.host_x, non_blocking=True)
-            u.copy_out()
+        with torch.cuda.stream(stream):
+            for u in units:                   # warm the copy paths
+                u.x.copy_(u.host_x, non_blocking=True)
+                u.copy_out()
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         barrier(dist)
         torch.cuda.synchronize()
         e0.record(stream)
-        for _ in range(Ke):
-            for u, (q, g) in zip(units, calls):
-                u.x.copy_(u.host_x, non_blocking=True)
-                run(q, "e2e quantize")
-                run(g, "e2e gemm")
-                u.copy_out()
+        with torch.cuda.stream(stream):
+            for _ in range(Ke):
+                for u, (q, g) in zip(units, calls):
+                    u.x.copy_(u.host_x, non_blocking=True)
+                    run(q, "e2e quantize")
+                    run(g, "e2e gemm")
+                    u.copy_out()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(dist)
@@ -631,12 +660,13 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
     roof["traffic"] = recorded_traffic(kernel_name, name)
     roof["kernel"] = kernel_name
     roof["peak_source"] = peak_note
-    roof["duration"] = ("mean period per GEMM launch over the workload's GEMMs launched back to "
-                        f"back {R} times (chained by programmatic dependent launch as in the step)")
+    roof["duration"] = ("mean period per GEMM launch over the workload's GEMMs captured back to "
+                        f"back {R} times in one CUDA graph (chained by programmatic dependent launch "
+                        "as in the step)")
     roof["algorithmic_per_launch"] = ({"bytes": [int(u.gemm_bytes) for u in units]} if hbm
                                       else {"flops": [float(u.flops) for u in units]})
     roof["isolated_median"] = {"value": [round(x, 1) for x in iso], "unit": roof["unit"],
-                               "note": "each GEMM between its own two events (no overlap)"}
+                               "note": "each GEMM alone (a one-launch graph between its own two events)"}
     q_total = sum(statistics.median(t) for t in per_quant)
     g_total = sum(statistics.median(t) for t in per_gemm)
     quant_gbs = sum(u.quant_bytes for u in units) / (q_total * 1e-3) / 1e9
@@ -728,10 +758,11 @@ def run_ours(args, world, rank, local):
         "roofline": head["roofline"],
         "kernels": head["kernels"],
         "gpu_launches": head["gpu_launches"],
-        "timing": ("value: K steps between two events (kernels chained by programmatic dependent "
-                   "launch), max over ranks; roofline: the GEMMs alone back to back, mean period per "
-                   "launch; kernels: each kernel between its own events over max(K, 50) steps "
-                   "(min, median)"),
+        "timing": ("value: one step captured in a CUDA graph, replayed K times between two events "
+                   "(kernels chained by programmatic dependent launch), max over ranks; roofline: "
+                   "max(K, 50) rounds of the GEMMs back to back in one graph, mean period per launch; "
+                   "kernels: each kernel alone in a graph, each replay between its own events "
+                   "(min, median over max(K, 50)); e2e: host-issued calls with host copies"),
         "clocks": head["clocks"],
         "e2e": head["e2e"],
     }

@@ -203,10 +203,10 @@ using CfgGrouped128 = GemmCfg<128, 6, 2, false, true>;
 using CfgGroupedPair256 = GemmCfg<256, 6, 2, false, true, true>;
 using CfgSilu = GemmCfg<256, 4, 2, false, false, false, 1, false, true>;
 using CfgSiluPair = GemmCfg<256, 6, 2, false, false, true, 1, false, true>;
-using CfgSwap32 = GemmCfg<32, 10, 1, true, false>;
-using CfgSwap64 = GemmCfg<64, 8, 1, true, false>;
-using CfgSwap32Split = GemmCfg<32, 10, 1, true, false, false, 1, true>;
-using CfgSwap64Split = GemmCfg<64, 8, 1, true, false, false, 1, true>;
+using CfgSwap32 = GemmCfg<32, 5, 2, true, false>;
+using CfgSwap64 = GemmCfg<64, 4, 2, true, false>;
+using CfgSwap32Split = GemmCfg<32, 5, 2, true, false, false, 1, true>;
+using CfgSwap64Split = GemmCfg<64, 4, 2, true, false, false, 1, true>;
 
 constexpr int64_t kMaxRows = (int64_t{1} << 31) - 256;
 // Split workspace: one int32 counter per weight tile in a fixed region at its start.

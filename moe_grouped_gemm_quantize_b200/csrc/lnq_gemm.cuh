@@ -113,13 +113,16 @@ struct GemmCfg {
     static_assert(!(SWAP && GROUPED), "decode configuration is dense only");
     static_assert(!(PAIR && SWAP), "CTA pairs serve the dense and grouped configurations");
     static_assert(BNQ % 16 == 0 && BNQ >= 16 && BNQ <= 256, "MMA N for M=128/256");
-    static_assert(!SWAP || EPI_WG == 1, "decode epilogue: one thread per weight row");
-    static_assert(!SWAP || BNQ % 32 == 0, "decode tiles read TMEM in 32-column chunks");
+    static_assert(!SWAP || (BNQ / EPI_WG) % 16 == 0, "decode threads read TMEM in 16-column loads");
     static_assert(SWAP || BNQ % 128 == 0, "dense tiles cover whole 128-column scale blocks");
 
     static constexpr int kP = 128;                // P rows per CTA (MMA M per CTA)
     static constexpr int kTileM = PAIR ? 256 : 128;  // P rows per tile
-    static constexpr int kBK = 128;               // K elements (bytes) per stage
+    static constexpr int kBK = 128;               // K elements (bytes) per K block
+    // K blocks per pipeline stage: decode tiles stream two weight boxes per stage (one
+    // barrier wait, one expect-tx arrival and one commit for 32 KB of weights), and the
+    // epilogue promotes the stage's two K blocks together
+    static constexpr int kKbPerStage = SWAP ? 2 : 1;
     static constexpr int kPBytes = kP * kBK;
     static constexpr int kQRowsPerCta = PAIR ? BNQ / 2 : BNQ;
     static constexpr int kQBytes = kQRowsPerCta * kBK;
@@ -140,8 +143,9 @@ struct GemmCfg {
     static constexpr int kScaleSlotFloats = kScaleBatch * kScaleKbFloats;
     static_assert(kScaleKbFloats % 4 == 0, "16-byte aligned scale runs");
     static constexpr int kCW = BNQ / EPI_WG;      // accumulator columns per epilogue thread
-    // TMEM columns per load in the promotion (each load issued one chunk ahead)
-    static constexpr int kLdCols = 32;
+    // TMEM columns per load in the promotion (each load issued one chunk ahead); a decode
+    // thread loads all of its columns of a K block at once
+    static constexpr int kLdCols = SWAP ? kCW : 32;
     static_assert(kCW % kLdCols == 0, "promotion chunks tile the thread's columns");
     // TMEM column of the thread's promotion chunk c, from its first column: SiLU.mul
     // threads take kCW/2 gate columns and the kCW/2 up columns 128 further on
@@ -175,8 +179,8 @@ struct GemmCfg {
 
     // shared-memory layout (offsets from a 1024-byte aligned base)
     static constexpr int kOffP = 0;
-    static constexpr int kOffQ = kOffP + STAGES * kPBytes;
-    static constexpr int kOffScale = kOffQ + STAGES * kQBytes;
+    static constexpr int kOffQ = kOffP + STAGES * kKbPerStage * kPBytes;
+    static constexpr int kOffScale = kOffQ + STAGES * kKbPerStage * kQBytes;
     static constexpr int kOffBar = kOffScale + kScaleStages * kScaleSlotFloats * 4;
     static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs * kSlices + 2 * kScaleStages + 1 + (SPLITK ? 2 : 0);
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -428,16 +432,16 @@ __device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint3
 }
 
 // Decode tile store: this thread holds weight row n = p0 + row for the tile's
-// tokens q0 .. q0 + kCW - 1; D is [M][N], so each token's row gets one bf16.
+// tokens q0 + col0 .. q0 + col0 + kCW - 1; D is [M][N], so each token's row gets one bf16.
 template <class C>
-__device__ __forceinline__ void store_decode_tile(const GemmArgs& args, const TileCoord& tc, int row,
+__device__ __forceinline__ void store_decode_tile(const GemmArgs& args, const TileCoord& tc, int row, int col0,
                                                   const float2 (&acc)[C::kCW / 2]) {
     const int n = tc.p0 + row;
     if (n >= args.N) return;
     const float bias = args.bias != nullptr ? bf16_lo(static_cast<uint32_t>(args.bias[n])) : 0.f;
 #pragma unroll
     for (int j = 0; j < C::kCW; ++j) {
-        const int m = tc.q0 + j;
+        const int m = tc.q0 + col0 + j;
         const float v = ((j & 1) ? acc[j >> 1].y : acc[j >> 1].x) + bias;
         if (m < args.M)
             args.d[static_cast<long long>(m) * args.N + n] =
@@ -463,6 +467,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     const uint32_t s_base = smem_u32(smem);
     const uint32_t sP = s_base + C::kOffP;
     const uint32_t sQ = s_base + C::kOffQ;
+    // K block h of ring stage s, P and Q operands
+    auto p_at = [&](int s, int h) { return sP + static_cast<uint32_t>((s * C::kKbPerStage + h) * C::kPBytes); };
+    auto q_at = [&](int s, int h) { return sQ + static_cast<uint32_t>((s * C::kKbPerStage + h) * C::kQBytes); };
     float* scale_slots = reinterpret_cast<float*>(smem + C::kOffScale);
     const uint32_t bars = s_base + C::kOffBar;
     auto full_bar = [&](int s) { return bars + 8u * s; };
@@ -563,19 +570,22 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     Segment sg0;
                     if (segment<C>(args, unit, units, 0, sg0)) {
                         const TileCoord tc = tile_coord<C>(args, sg0.t, rank);
-                        prefetched = min(C::STAGES, sg0.kb_hi - sg0.kb_lo);
+                        constexpr int KBS = C::kKbPerStage;
+                        prefetched = min(C::STAGES, (sg0.kb_hi - sg0.kb_lo + KBS - 1) / KBS);
                         if (elect_one()) {
                             for (int s = 0; s < prefetched; ++s) {
-                                mbar_arrive_expect_tx(full_bar(s), C::kPBytes + C::kQBytes);
-                                if constexpr (C::SWAP) {
-                                    tma_load_2d(sP + s * C::kPBytes, &map_p, full_bar(s),
-                                                (sg0.kb_lo + s) * C::kBK, tc.p0);
-                                } else {
-                                    tma_load_2d(sQ + s * C::kQBytes, &map_q, full_bar(s),
-                                                (sg0.kb_lo + s) * C::kBK, tc.q0);
-                                    if constexpr (C::SILU)  // the up rows of the same outputs
-                                        tma_load_2d(sQ + s * C::kQBytes + C::kQBoxRows * C::kBK, &map_q,
-                                                    full_bar(s), (sg0.kb_lo + s) * C::kBK, tc.q0 + args.N);
+                                const int kb0 = sg0.kb_lo + s * KBS;
+                                const int nk = min(KBS, sg0.kb_hi - kb0);
+                                mbar_arrive_expect_tx(full_bar(s), nk * (C::kPBytes + C::kQBytes));
+                                for (int h = 0; h < nk; ++h) {
+                                    if constexpr (C::SWAP) {
+                                        tma_load_2d(p_at(s, h), &map_p, full_bar(s), (kb0 + h) * C::kBK, tc.p0);
+                                    } else {
+                                        tma_load_2d(q_at(s, h), &map_q, full_bar(s), (kb0 + h) * C::kBK, tc.q0);
+                                        if constexpr (C::SILU)  // the up rows of the same outputs
+                                            tma_load_2d(q_at(s, h) + C::kQBoxRows * C::kBK, &map_q, full_bar(s),
+                                                        (kb0 + h) * C::kBK, tc.q0 + args.N);
+                                    }
                                 }
                             }
                         }
@@ -600,17 +610,18 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     p_row = tc.p0;
                     q_row = tc.group * args.N + tc.q0 + static_cast<int>(rank) * C::kSliceQRows;
                 }
-                for (int kb = sg.kb_lo; kb < sg.kb_hi; ++kb) {
+                for (int kb = sg.kb_lo; kb < sg.kb_hi; kb += C::kKbPerStage) {
+                    const int nk = min(C::kKbPerStage, sg.kb_hi - kb);
                     if (prefetched > 0) {
                         // stage already armed and its weight half in flight: load the activations
                         if constexpr (!C::PAIR) {
                             if (elect_one()) {
-                                if constexpr (C::SWAP)
-                                    tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK,
-                                                q_row);
-                                else
-                                    tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK,
-                                                p_row);
+                                for (int h = 0; h < nk; ++h) {
+                                    if constexpr (C::SWAP)
+                                        tma_load_2d(q_at(stage, h), &map_q, full_bar(stage), (kb + h) * C::kBK, q_row);
+                                    else
+                                        tma_load_2d(p_at(stage, h), &map_p, full_bar(stage), (kb + h) * C::kBK, p_row);
+                                }
                             }
                             __syncwarp();
                         }
@@ -626,19 +637,21 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                                 if (rank == 0)
                                     mbar_arrive_expect_tx(full_bar(stage), 2 * (C::kPBytes + C::kQBytes));
                                 const uint32_t leader_full = mapa_shared(full_bar(stage), 0);
-                                tma_load_2d_pair(sP + stage * C::kPBytes, &map_p, leader_full, kb * C::kBK, p_row);
+                                tma_load_2d_pair(p_at(stage, 0), &map_p, leader_full, kb * C::kBK, p_row);
                                 // slice h of the tile's N: this CTA holds its kSliceQRows rows of it
 #pragma unroll
                                 for (int h = 0; h < C::kSlices; ++h)
-                                    tma_load_2d_pair(sQ + stage * C::kQBytes + h * C::kSliceQRows * C::kBK, &map_q,
+                                    tma_load_2d_pair(q_at(stage, 0) + h * C::kSliceQRows * C::kBK, &map_q,
                                                      leader_full, kb * C::kBK, q_row + h * C::kSliceN);
                             } else {
-                                mbar_arrive_expect_tx(full_bar(stage), C::kPBytes + C::kQBytes);
-                                tma_load_2d(sP + stage * C::kPBytes, &map_p, full_bar(stage), kb * C::kBK, p_row);
-                                tma_load_2d(sQ + stage * C::kQBytes, &map_q, full_bar(stage), kb * C::kBK, q_row);
-                                if constexpr (C::SILU && !C::PAIR)  // the up rows of the same outputs
-                                    tma_load_2d(sQ + stage * C::kQBytes + C::kQBoxRows * C::kBK, &map_q,
-                                                full_bar(stage), kb * C::kBK, q_row + args.N);
+                                mbar_arrive_expect_tx(full_bar(stage), nk * (C::kPBytes + C::kQBytes));
+                                for (int h = 0; h < nk; ++h) {
+                                    tma_load_2d(p_at(stage, h), &map_p, full_bar(stage), (kb + h) * C::kBK, p_row);
+                                    tma_load_2d(q_at(stage, h), &map_q, full_bar(stage), (kb + h) * C::kBK, q_row);
+                                    if constexpr (C::SILU && !C::PAIR)  // the up rows of the same outputs
+                                        tma_load_2d(q_at(stage, h) + C::kQBoxRows * C::kBK, &map_q, full_bar(stage),
+                                                    (kb + h) * C::kBK, q_row + args.N);
+                                }
                             }
                         }
                         __syncwarp();
@@ -678,62 +691,70 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         constexpr int kIssuers = 2;
         if (rank == 0) {
             int stage = 0, abuf = 0;
-            int gk = 0;  // K blocks seen, for the alternation
+            int gs = 0;  // ring stages seen, for the alternation
             uint32_t phase = 0, aphase = 0;
             bool ok = true;
             const uint64_t adesc0 = sw128_kmajor_desc(sP);
             const uint64_t bdesc0 = sw128_kmajor_desc(sQ);
+            auto next_acc = [&]() {
+                if (++abuf == C::kAccBufs) {
+                    abuf = 0;
+                    aphase ^= 1u;
+                }
+            };
             Segment sg;
             for (int i = 0; ok && segment<C>(args, unit, units, i, sg); ++i) {
                 const TileCoord tc = tile_coord<C>(args, sg.t, 0);
                 if (tc.group < 0) continue;
-                for (int kb = sg.kb_lo; kb < sg.kb_hi && ok; ++kb) {
-                    if (gk++ % kIssuers != midx) {
-                        // the other issuer's K block
+                for (int kb = sg.kb_lo; kb < sg.kb_hi && ok; kb += C::kKbPerStage) {
+                    const int nk = min(C::kKbPerStage, sg.kb_hi - kb);
+                    if (gs++ % kIssuers != midx) {
+                        // the other issuer's stage and its K blocks' accumulators
                         if (++stage == C::STAGES) {
                             stage = 0;
                             phase ^= 1u;
                         }
-                        if (++abuf == C::kAccBufs) {
-                            abuf = 0;
-                            aphase ^= 1u;
-                        }
+                        for (int hk = 0; hk < nk; ++hk) next_acc();
                         continue;
                     }
                     if (!mbar_wait_warp(full_bar(stage), phase, wctx)) {
                         ok = false;
                         break;
                     }
-                    // descriptor start fields advance by (byte offset >> 4)
-                    const uint64_t adesc = adesc0 + static_cast<uint64_t>((stage * C::kPBytes) >> 4);
+                    for (int hk = 0; hk < nk && ok; ++hk) {
+                        // descriptor start fields advance by (byte offset >> 4)
+                        const int sk = stage * C::kKbPerStage + hk;
+                        const uint64_t adesc = adesc0 + static_cast<uint64_t>((sk * C::kPBytes) >> 4);
 #pragma unroll
-                    for (int h = 0; h < C::kSlices; ++h) {
-                        const int slot = abuf * C::kSlices + h;
-                        if (!mbar_wait_warp(tempty_bar(slot), aphase ^ 1u, wctx)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::BNQ + h * C::kSliceN);
-                        const uint64_t bdesc =
-                            bdesc0 + static_cast<uint64_t>((stage * C::kQBytes + h * C::kSliceQRows * C::kBK) >> 4);
-                        if (elect_one()) {
-                            if constexpr (C::PAIR) {
-#pragma unroll
-                                for (int k = 0; k < C::kBK / 32; ++k)
-                                    mma_f8f6f4_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
-                                                    k > 0 ? 1u : 0u);
-                                mma_commit_pair(mapa_shared(tfull_bar(slot), 0));
-                                mma_commit_pair(mapa_shared(tfull_bar(slot), 1));
-                            } else {
-#pragma unroll
-                                for (int k = 0; k < C::kBK / 32; ++k)
-                                    mma_f8f6f4(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
-                                               k > 0 ? 1u : 0u);
-                                mma_commit(tfull_bar(slot));
+                        for (int h = 0; h < C::kSlices; ++h) {
+                            const int slot = abuf * C::kSlices + h;
+                            if (!mbar_wait_warp(tempty_bar(slot), aphase ^ 1u, wctx)) {
+                                ok = false;
+                                break;
                             }
+                            tc_fence_after();
+                            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * C::BNQ + h * C::kSliceN);
+                            const uint64_t bdesc =
+                                bdesc0 + static_cast<uint64_t>((sk * C::kQBytes + h * C::kSliceQRows * C::kBK) >> 4);
+                            if (elect_one()) {
+                                if constexpr (C::PAIR) {
+#pragma unroll
+                                    for (int k = 0; k < C::kBK / 32; ++k)
+                                        mma_f8f6f4_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
+                                                        k > 0 ? 1u : 0u);
+                                    mma_commit_pair(mapa_shared(tfull_bar(slot), 0));
+                                    mma_commit_pair(mapa_shared(tfull_bar(slot), 1));
+                                } else {
+#pragma unroll
+                                    for (int k = 0; k < C::kBK / 32; ++k)
+                                        mma_f8f6f4(d_tmem, adesc + 2u * k, bdesc + 2u * k, C::kIdesc,
+                                                   k > 0 ? 1u : 0u);
+                                    mma_commit(tfull_bar(slot));
+                                }
+                            }
+                            __syncwarp();
                         }
-                        __syncwarp();
+                        next_acc();
                     }
                     if (!ok) break;
                     // the stage is free once every slice's MMAs have read it
@@ -749,10 +770,6 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
-                    }
-                    if (++abuf == C::kAccBufs) {
-                        abuf = 0;
-                        aphase ^= 1u;
                     }
                 }
             }
@@ -847,7 +864,69 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 #pragma unroll
             for (int i = 0; i < C::kCW / 2; ++i) acc[i] = make_float2(0.f, 0.f);
             int j = 0;  // K block within the scale slot's batch
-            for (int kb = sg.kb_lo; kb < sg.kb_hi; ++kb) {
+            for (int kb = sg.kb_lo; kb < sg.kb_hi; kb += C::kKbPerStage) {
+                if constexpr (C::SWAP) {
+                    // Decode: the ring stage's K blocks (two, or one at the end of a run) are
+                    // promoted together: both partials are loaded before either is waited
+                    // on, both accumulators released, then both multiplied in.  This
+                    // thread's columns are tokens wg*kCW .. wg*kCW + kCW - 1 of the tile.
+                    const int nk = min(C::kKbPerStage, sg.kb_hi - kb);
+                    const bool batch_last = (j + nk == C::kScaleBatch) || (kb + nk == sg.kb_hi);
+                    int abuf1 = abuf + 1;
+                    uint32_t aphase1 = aphase;
+                    if (abuf1 == C::kAccBufs) {
+                        abuf1 = 0;
+                        aphase1 ^= 1u;
+                    }
+                    if ((j == 0 && !mbar_wait(sfull_bar(sstage), sphase, wctx)) ||
+                        !mbar_wait(tfull_bar(abuf), aphase, wctx) ||
+                        (nk > 1 && !mbar_wait(tfull_bar(abuf1), aphase1, wctx))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float* slot = scale_slots + sstage * C::kScaleSlotFloats + j * C::kScaleKbFloats;
+                    const uint32_t col = static_cast<uint32_t>(C::wg_col(wg));
+                    uint32_t r0[C::kCW], r1[C::kCW];
+                    tmem_ld_async(tmem_base + t_lane + static_cast<uint32_t>(abuf * C::BNQ) + col, r0);
+                    if (nk > 1) tmem_ld_async(tmem_base + t_lane + static_cast<uint32_t>(abuf1 * C::BNQ) + col, r1);
+                    tmem_wait_ld(r0);
+                    if (nk > 1) tmem_wait_ld(r1);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive_relaxed(tempty_bar(abuf));
+                        if (nk > 1) mbar_arrive_relaxed(tempty_bar(abuf1));
+                    }
+                    {
+                        const float sb = slot[C::kSbOffset];
+                        promote_chunk<C, C::kCW>(acc, r0, 0, slot + wg * C::kCW, make_float2(sb, sb));
+                    }
+                    if (nk > 1) {
+                        const float* slot1 = slot + C::kScaleKbFloats;
+                        const float sb = slot1[C::kSbOffset];
+                        promote_chunk<C, C::kCW>(acc, r1, 0, slot1 + wg * C::kCW, make_float2(sb, sb));
+                    }
+                    // the per-token scales were read by the FMAs above: the slot may go
+                    if (batch_last) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_relaxed(sempty_bar(sstage));
+                        j = 0;
+                        if (++sstage == C::kScaleStages) {
+                            sstage = 0;
+                            sphase ^= 1u;
+                        }
+                    } else {
+                        j += nk;
+                    }
+                    abuf = abuf1;
+                    aphase = aphase1;
+                    if (nk > 1 && ++abuf == C::kAccBufs) {
+                        abuf = 0;
+                        aphase ^= 1u;
+                    }
+                    continue;
+                } else {
                 const bool batch_last = (j == C::kScaleBatch - 1) || (kb + 1 == sg.kb_hi);
                 const int slot_id = abuf * C::kSlices + (C::kSlices == 1 ? 0 : wg);
                 if ((j == 0 && !mbar_wait(sfull_bar(sstage), sphase, wctx)) ||
@@ -861,9 +940,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 // the accumulator slice and the scale slot are only read, and each arrival
                 // follows the completion of those reads: no release fence is needed (one
                 // would also wait for this warp's outstanding output stores).  The slice is
-                // released as soon as its last chunk is in registers; the scale slot after
-                // the last K block of its batch (after the FMAs in the decode configuration,
-                // which read per-token scales from it).
+                // released as soon as its last chunk is in registers, the scale slot after
+                // the last K block of its batch.
                 const uint32_t sempty = sempty_bar(sstage);
                 promote_k_block<C>(acc, taddr, slot, row, wg, [&]() {
                     tc_fence_before();
@@ -871,18 +949,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     if (lane == 0) {
                         if constexpr (C::PAIR) mbar_arrive_cluster_relaxed(mapa_shared(tempty_bar(slot_id), 0));
                         else mbar_arrive_relaxed(tempty_bar(slot_id));
-                        // dense: the scales were read before the first TMEM load
-                        if constexpr (!C::SWAP) {
-                            if (batch_last) mbar_arrive_relaxed(sempty);
-                        }
+                        // the scales were read before the first TMEM load
+                        if (batch_last) mbar_arrive_relaxed(sempty);
                     }
                 });
-                if constexpr (C::SWAP) {
-                    if (batch_last) {
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_relaxed(sempty);
-                    }
-                }
                 if (batch_last) {
                     j = 0;
                     if (++sstage == C::kScaleStages) {
@@ -895,6 +965,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 if (++abuf == C::kAccBufs) {
                     abuf = 0;
                     aphase ^= 1u;
+                }
                 }
             }
             if (!ok) break;
@@ -913,7 +984,8 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     auto part = [&](int sl) {
                         return reinterpret_cast<float4*>(
                             args.partials +
-                            ((static_cast<long long>(sg.t) * args.max_slots + sl) * C::kP + row) * C::kCW);
+                            ((static_cast<long long>(sg.t) * args.max_slots + sl) * C::kP + row) * C::BNQ +
+                            wg * C::kCW);
                     };
                     float4* mine = part(slot);
 #pragma unroll
@@ -1009,16 +1081,15 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                             for (int i = 0; i < 64; ++i)
                                 amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(h[i])), fabsf(bf16_hi(h[i]))));
                             const float sv = scale_of_amax(amax);
-                            const float rv = rcp_approx(sv);
+                            float r_lo = 0.f, r_hi = 0.f;
+                            if (sv >= 0x1p-125f) bracket_rcp(sv, r_lo, r_hi);
                             uint8_t* qrow = args.q_out + static_cast<long long>(m) * args.N + n0;
 #pragma unroll
                             for (int j = 0; j < 8; ++j) {
-                                float t0[8], t1[8];
                                 const uint4 r0 = make_uint4(h[8 * j + 0], h[8 * j + 1], h[8 * j + 2], h[8 * j + 3]);
                                 const uint4 r1 = make_uint4(h[8 * j + 4], h[8 * j + 5], h[8 * j + 6], h[8 * j + 7]);
-                                quotients8(r0, sv, rv, sv == 0.0f, !(sv >= 0x1p-125f), t0);
-                                quotients8(r1, sv, rv, sv == 0.0f, !(sv >= 0x1p-125f), t1);
-                                const uint2 p0 = pack8(t0), p1 = pack8(t1);
+                                const uint2 p0 = codes8(r0, sv, r_lo, r_hi, sv == 0.0f, !(sv >= 0x1p-125f));
+                                const uint2 p1 = codes8(r1, sv, r_lo, r_hi, sv == 0.0f, !(sv >= 0x1p-125f));
                                 *reinterpret_cast<uint4*>(qrow + 16 * j) = make_uint4(p0.x, p0.y, p1.x, p1.y);
                             }
                             args.sfa_out[static_cast<long long>(n0 >> 7) * args.M4_out + m] = sv;
@@ -1043,7 +1114,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     }
                 }
             } else {
-                store_decode_tile<C>(args, tc, row, acc);
+                store_decode_tile<C>(args, tc, row, wg * C::kCW, acc);
             }
         }
     }

@@ -34,17 +34,6 @@ __device__ __forceinline__ float quotient(float x, float s, bool zero_group) {
     return zero_group ? x : __fdiv_rn(x, s);
 }
 
-// True when the E4M3 rounding of t could differ from the E4M3 rounding of a
-// value at most 16 fp32 ulps away: t within 32 ulps of a rounding midpoint of
-// the normal E4M3 range (the 20 fp32 mantissa bits below the 3 E4M3 mantissa
-// bits within 32 of 0x80000), or |t| < 2^-6 (E4M3 subnormal range, where the
-// midpoints sit elsewhere).  Binade edges hold no midpoint, so one test covers
-// every exponent.
-__device__ __forceinline__ bool near_e4m3_midpoint(float t) {
-    const uint32_t b = __float_as_uint(t);
-    return ((b & 0xFFFFFu) - 0x7FFE0u) < 65u || fabsf(t) < 0x1p-6f;
-}
-
 // The correctly rounded amax / 448 from one multiplication and two FMAs: q0 =
 // RN(amax * c) with c = RN(1/448), then one correction step with the exact
 // remainder amax - 448 q0 (Markstein's division correction for a divisor known
@@ -64,15 +53,28 @@ __device__ __forceinline__ float rcp_approx(float s) {
     return r;
 }
 
-// Eight quotients x/s whose E4M3 codes equal those of the correctly rounded
-// quotients.  The fast path multiplies by r ~ 1/s: with r within 2^-21 of 1/s,
-// x*r and RN(x/s) are at most 16 ulps apart and take the same E4M3 code unless
-// x*r lies within 32 ulps of an E4M3 midpoint (a rounding test in the manner of
-// Ziv's correctly rounded elementary functions).  Then, and for tiny scales
-// where r would be subnormal or infinite, the eight values take the IEEE
-// division instead.
-__device__ __forceinline__ void quotients8(const uint4& raw, float s, float r, bool zero_group,
-                                           bool exact_group, float (&t)[8]) {
+
+__device__ __forceinline__ uint2 pack8(const float (&t)[8]) {
+    uint2 out;
+    out.x = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
+    out.y = e4m3x2(t[4], t[5]) | (e4m3x2(t[6], t[7]) << 16);
+    return out;
+}
+
+// Eight E4M3 codes (packed, the first value in the low byte) of the correctly rounded
+// quotients x/s of the bf16 values in `raw`.  r_lo and r_hi bracket 1/s: with r within
+// 2^-21 of 1/s (rcp.approx), r_lo = RN(r (1 - 2^-18)) and r_hi = RN(r (1 + 2^-18)), so for
+// every x the products RN(x r_lo) and RN(x r_hi) lie on either side of RN(x/s) (each
+// within about 2^-18 of x/s, further than RN(x/s) can be).  E4M3 rounding with
+// saturation is monotonic, so when both products take the same code, RN(x/s) takes it
+// too; otherwise (a quotient within about 32 fp32 ulps of an E4M3 rounding boundary,
+// about one value in 16000) the eight values take the IEEE division.  A product that is
+// an fp32 subnormal codes to +-0 at both ends, as the quotient does.  Scales below 2^-125,
+// whose reciprocal may overflow, take the division outright; an all-zero group (s = 0)
+// keeps the signed zeros.
+__device__ __forceinline__ uint2 codes8(const uint4& raw, float s, float r_lo, float r_hi, bool zero_group,
+                                        bool exact_group) {
+    float t[8];
     t[0] = bf16_lo(raw.x);
     t[1] = bf16_hi(raw.x);
     t[2] = bf16_lo(raw.y);
@@ -81,27 +83,46 @@ __device__ __forceinline__ void quotients8(const uint4& raw, float s, float r, b
     t[5] = bf16_hi(raw.z);
     t[6] = bf16_lo(raw.w);
     t[7] = bf16_hi(raw.w);
-    if (zero_group) return;  // all +-0: the codes keep the signs
-    float f[8];
-    bool risky = exact_group;
+    if (zero_group) return pack8(t);
+    if (!exact_group) {
+        float lo[8], hi[8];
+        const float2 rl = make_float2(r_lo, r_lo), rh = make_float2(r_hi, r_hi);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        f[j] = t[j] * r;
-        risky |= near_e4m3_midpoint(f[j]);
+        for (int j = 0; j < 4; ++j) {
+            const float2 x = make_float2(t[2 * j], t[2 * j + 1]);
+            const float2 a = __fmul2_rn(x, rl), b = __fmul2_rn(x, rh);
+            lo[2 * j] = a.x;
+            lo[2 * j + 1] = a.y;
+            hi[2 * j] = b.x;
+            hi[2 * j + 1] = b.y;
+        }
+        const uint2 a = pack8(lo), b = pack8(hi);
+        if (a.x == b.x && a.y == b.y) return a;
     }
-    if (risky) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] = __fdiv_rn(t[j], s);
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) t[j] = f[j];
+    for (int j = 0; j < 8; ++j) t[j] = __fdiv_rn(t[j], s);
+    return pack8(t);
 }
 
-__device__ __forceinline__ uint2 pack8(const float (&t)[8]) {
-    uint2 out;
-    out.x = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
-    out.y = e4m3x2(t[4], t[5]) | (e4m3x2(t[6], t[7]) << 16);
-    return out;
+// The two bracketing reciprocals of codes8 for a scale s >= 2^-125.
+__device__ __forceinline__ void bracket_rcp(float s, float& r_lo, float& r_hi) {
+    const float r = rcp_approx(s);
+    r_lo = __fmul_rn(r, 1.0f - 0x1p-18f);
+    r_hi = __fmul_rn(r, 1.0f + 0x1p-18f);
+}
+
+// Largest magnitude of two packed bf16 pairs, as a packed pair whose magnitudes are
+// max(|a|, |b|) lane by lane (the sign bits are not meaningful); exact.
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Largest |x| of the eight bf16 values in `raw` (exact).
+__device__ __forceinline__ float absmax8_packed(const uint4& raw) {
+    const uint32_t m = maxabs_bf16x2(maxabs_bf16x2(raw.x, raw.y), maxabs_bf16x2(raw.z, raw.w));
+    return fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
 }
 
 __device__ __forceinline__ float absmax8(const uint4& raw) {
@@ -237,7 +258,7 @@ __global__ void __launch_bounds__(kQuantThreads)
         float sv[kRowsPerWarp];
 #pragma unroll
         for (int i = 0; i < kRowsPerWarp; ++i) {
-            float amax = absmax8(raw[i]);
+            float amax = absmax8_packed(raw[i]);
 #pragma unroll
             for (int off = 8; off >= 1; off >>= 1)
                 amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
@@ -247,9 +268,10 @@ __global__ void __launch_bounds__(kQuantThreads)
         for (int i = 0; i < kRowsPerWarp; ++i) {
             const long long r = row0 + i;
             if (r < args.M && group_ok) {
-                float tq[8];
-                quotients8(raw[i], sv[i], rcp_approx(sv[i]), sv[i] == 0.0f, !(sv[i] >= 0x1p-125f), tq);
-                *reinterpret_cast<uint2*>(args.q + r * args.ld_q + col0 + lane * 8) = pack8(tq);
+                float r_lo, r_hi;
+                bracket_rcp(sv[i], r_lo, r_hi);
+                *reinterpret_cast<uint2*>(args.q + r * args.ld_q + col0 + lane * 8) =
+                    codes8(raw[i], sv[i], r_lo, r_hi, sv[i] == 0.0f, !(sv[i] >= 0x1p-125f));
             }
         }
         if ((lane & 15) == 0 && group_ok && row0 < args.M4)

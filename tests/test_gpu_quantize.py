@@ -74,6 +74,21 @@ def test_activation_edge_values():
     assert_same_a(x.to(torch.bfloat16))
 
 
+def test_subnormal_values_under_the_smallest_reciprocal_scales():
+    # scales just above 2^-125 (the smallest whose reciprocal is taken rather than the
+    # division) with the rest of each group bf16 subnormals: their quotients reach the
+    # E4M3 subnormal codes, so no input or product may be flushed to zero
+    rows = []
+    for m in (1.0, 1.25, 1.5, 3.0, 5.5, 7.9):
+        for sign in (1.0, -1.0):
+            row = np.zeros(128)
+            row[0] = 448.0 * 2.0 ** -125 * m
+            row[1:] = sign * np.arange(1, 128) * 2.0 ** -133
+            rows.append(row)
+    x = torch.tensor(np.stack(rows)).to(torch.bfloat16)
+    assert_same_a(x)
+
+
 def test_every_bf16_magnitude_with_unit_and_power_of_two_scales():
     # all non-negative finite bf16 bit patterns up to 448, both signs, in rows whose
     # amax is exactly 448 * 2^j: the scale is 2^j and each code is the E4M3 rounding
