@@ -720,6 +720,7 @@ def run_ours(args, world, rank, local):
     # the weights are model parameters quantized before timing: nothing in the step
     # writes them, so the GEMMs may stream them before the previous kernel completes
     lnq.lnq_set_weight_prefetch(not args.no_weight_prefetch)
+    lnq.lnq_set_tma_store(bool(args.tma_store))
 
     names = list(ALL_WORKLOADS) if args.workload == "all" else [args.workload]
     results = {}
@@ -750,6 +751,7 @@ def run_ours(args, world, rank, local):
                    "dense_cta_pairs": args.cta_pairs,
                    "grouped_cta_pairs": args.grouped_cta_pairs,
                    "weight_prefetch": not args.no_weight_prefetch,
+                   "output_store": "TMA store through shared memory" if args.tma_store else "row stores from registers",
                    "decode_k_split": head["decode_k_split"],
                    "epilogue": head["epilogue"],
                    "recipe": head["recipe"],
@@ -949,6 +951,9 @@ def main():
                          "power-of-two scales applied by the block-scaled MMA")
     ap.add_argument("--grouped-cta-pairs", type=int, default=0, choices=[0, 1],
                     help="moe_psum: 256x256 tiles on CTA pairs (1) or 128-row tiles (0)")
+    ap.add_argument("--tma-store", type=int, default=1, choices=[0, 1],
+                    help="dense and grouped GEMM outputs: 1 through shared memory and TMA stores, 0 each "
+                         "thread stores its own row")
     ap.add_argument("--cta-pairs", type=int, default=1, choices=[0, 1, 2],
                     help="dense GEMMs with M > 128: 0 one CTA per 128x256 tile, 1 CTA pairs on "
                          "256x256 tiles, 2 CTA pairs on 256x128 tiles")

@@ -438,6 +438,20 @@ int32_t lnq_set_grouped_cta_pairs(int32_t enable);
  */
 int32_t lnq_set_weight_prefetch(int32_t enable);
 
+/*
+ * Output path of the dense and grouped GEMMs (process-wide, default 1).  Non-zero:
+ * each epilogue warpgroup converts its 128 rows x 32 columns of the tile to bf16 (or
+ * its 64 E4M3 codes for the fused FP8 output) into an 8 KB shared-memory buffer in the
+ * 64-byte swizzle and writes it with one TMA store (cp.async.bulk.tensor), the box
+ * clipped at the M and N edges; 0: every epilogue thread writes its own output row
+ * with 16-byte stores.  Tiles of the masked and prefix-sum layouts whose rows end
+ * inside the output are always stored row by row.  Results are identical bit for bit;
+ * only the speed differs (the TMA stores were measured 1-7% faster per GEMM on the
+ * prefill, square and MoE workloads).  Decode tiles (M <= 64) always store directly.
+ * Returns the previous setting.
+ */
+int32_t lnq_set_tma_store(int32_t enable);
+
 /* Version of this ABI (major*10000 + minor*100 + patch). */
 int32_t lnq_abi_version(void);
 

@@ -32,7 +32,7 @@ __all__ = [
     "quantize_weights_ue8m0", "ue8m0_atoms",
     "lnq_m_grouped_fp8_gemm_masked", "lnq_get_last_device_error", "lnq_status_string",
     "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs",
-    "lnq_set_weight_prefetch",
+    "lnq_set_weight_prefetch", "lnq_set_tma_store",
     "quantize_activations", "quantize_weights",
     "quantize_weights_grouped", "linear",
     "m_grouped_linear", "ceil4",
@@ -99,7 +99,8 @@ def lib() -> ctypes.CDLL:
         L.lnq_abi_version.restype = ctypes.c_int32
         L.lnq_fp8_block_gemm_nt_workspace_bytes.argtypes = [I64, I64, I64, I32]
         L.lnq_fp8_block_gemm_nt_workspace_bytes.restype = I64
-        for knob in ("lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs", "lnq_set_weight_prefetch"):
+        for knob in ("lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs", "lnq_set_weight_prefetch",
+                     "lnq_set_tma_store"):
             getattr(L, knob).argtypes = [ctypes.c_int32]
             getattr(L, knob).restype = ctypes.c_int32
         _lib = L
@@ -463,6 +464,12 @@ def lnq_set_weight_prefetch(enable: bool) -> bool:
     """Let GEMMs stream their first weight stages before the previous kernel of the
     stream completes (weights must not be written by still-running kernels)."""
     return bool(lib().lnq_set_weight_prefetch(1 if enable else 0))
+
+
+def lnq_set_tma_store(enable: bool) -> bool:
+    """Dense and grouped GEMM outputs through shared memory and TMA stores (True, the
+    default) or stored row by row from registers (False).  Returns the previous setting."""
+    return bool(lib().lnq_set_tma_store(1 if enable else 0))
 
 
 def lnq_selftest_wait_timeout(timeout_ns: int, stream=None) -> None:

@@ -49,6 +49,8 @@ std::atomic<int> g_dense_pairs{1};
 std::atomic<int> g_grouped_pairs{0};
 // GEMMs may start streaming weights before the prior kernel completes.
 std::atomic<int> g_weight_prefetch{0};
+// Dense and grouped GEMM outputs go through shared memory and TMA stores when set.
+std::atomic<int> g_tma_store{1};
 DeviceInfo g_devices[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 
@@ -120,6 +122,21 @@ lnq_status encode_e4m3_map(CUtensorMap* map, const void* base, int64_t rows, int
     return r == CUDA_SUCCESS ? LNQ_OK : LNQ_ERR_CUDA;
 }
 
+// 2-D output tensor [rows][cols] of `elem_bytes`-byte elements (row stride = cols
+// elements), box of 64 bytes x 128 rows in the 64-byte swizzle: one epilogue
+// warpgroup's staging buffer of the TMA-store epilogue.
+lnq_status encode_out_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int elem_bytes) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * elem_bytes)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(64 / elem_bytes), 128u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
 template <class C>
 lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
                        const void* wgt, int64_t wgt_rows, int64_t K, GemmArgs args,
@@ -136,12 +153,22 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
                                  C::SILU ? C::kQBoxRows : (C::PAIR ? C::kSliceQRows : C::kQRowsPerCta));
     }
     if (st != LNQ_OK) return st;
+    // the output of the TMA-store epilogue (dense and grouped tiles; decode tiles store
+    // their transposed rows directly and never read this map)
+    CUtensorMap map_d;
+    std::memset(&map_d, 0, sizeof map_d);
+    if (!C::SWAP) {
+        st = args.q_out != nullptr ? encode_out_map(&map_d, args.q_out, args.M, args.N, 1)
+                                   : encode_out_map(&map_d, args.d, args.M, args.N, 2);
+        if (st != LNQ_OK) return st;
+    }
     static std::atomic<bool> attr_set[kMaxDevices];
     st = smem_attr_once(attr_set, dev.ordinal, k_fp8_block_gemm<C>, C::kSmemBytes);
     if (st != LNQ_OK) return st;
     args.status = dev.status;
     args.timeout_ns = kDefaultTimeoutNs;
     args.prefetch_weights = g_weight_prefetch.load(std::memory_order_relaxed);
+    args.tma_store = g_tma_store.load(std::memory_order_relaxed);
     if constexpr (C::PAIR) {
         // clusters of two CTAs sharing one MMA; as many pairs as can be resident
         constexpr int kCluster = 2;
@@ -169,7 +196,7 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
         const int clusters = args.num_tiles < resident ? args.num_tiles : resident;
         if (clusters <= 0) return LNQ_OK;
         cfg.gridDim = dim3(kCluster * clusters, 1, 1);
-        if (cudaLaunchKernelEx(&cfg, k_fp8_block_gemm<C>, map_p, map_q, args) != cudaSuccess)
+        if (cudaLaunchKernelEx(&cfg, k_fp8_block_gemm<C>, map_p, map_q, map_d, args) != cudaSuccess)
             return LNQ_ERR_CUDA;
         return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
     }
@@ -187,7 +214,7 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, k_fp8_block_gemm<C>, map_p, map_q, args) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, k_fp8_block_gemm<C>, map_p, map_q, map_d, args) != cudaSuccess)
         return LNQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
 }
@@ -261,6 +288,8 @@ extern "C" {
 int32_t lnq_abi_version(void) { return 10000; }
 
 int32_t lnq_set_weight_prefetch(int32_t enable) { return g_weight_prefetch.exchange(enable ? 1 : 0); }
+
+int32_t lnq_set_tma_store(int32_t enable) { return g_tma_store.exchange(enable ? 1 : 0); }
 
 int32_t lnq_set_grouped_cta_pairs(int32_t enable) {
     return g_grouped_pairs.exchange(enable == 1 ? 1 : 0);

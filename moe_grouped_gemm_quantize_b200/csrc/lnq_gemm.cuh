@@ -92,6 +92,9 @@ struct GemmArgs {
     uint8_t* q_out;        // [M][N] E4M3, or nullptr (bf16 D)
     float* sfa_out;        // [N/128][M4_out]
     long long M4_out;
+    // dense and grouped tiles: 1 = output through shared memory and TMA stores, 0 = each
+    // thread stores its own row
+    int tma_store;
 };
 
 template <int BNQ_, int STAGES_, int EPI_WG_, bool SWAP_, bool GROUPED_, bool PAIR_ = false,
@@ -181,7 +184,13 @@ struct GemmCfg {
     static constexpr int kOffP = 0;
     static constexpr int kOffQ = kOffP + STAGES * kKbPerStage * kPBytes;
     static constexpr int kOffScale = kOffQ + STAGES * kKbPerStage * kQBytes;
-    static constexpr int kOffBar = kOffScale + kScaleStages * kScaleSlotFloats * 4;
+    // Output staging for the TMA-store epilogue (dense and grouped tiles): per epilogue
+    // warpgroup one 8 KB buffer of 128 rows x 64 bytes (32 bf16 columns, or 64 E4M3
+    // codes) in the 64-byte swizzle, sent out by one TMA store per round.
+    static constexpr int kStageRowBytes = 64;
+    static constexpr int kStageBytes = 128 * kStageRowBytes;
+    static constexpr int kOffStage = (kOffScale + kScaleStages * kScaleSlotFloats * 4 + 1023) / 1024 * 1024;
+    static constexpr int kOffBar = kOffStage + (SWAP ? 0 : EPI_WG * kStageBytes);
     static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs * kSlices + 2 * kScaleStages + 1 + (SPLITK ? 2 : 0);
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -449,6 +458,30 @@ __device__ __forceinline__ void store_decode_tile(const GemmArgs& args, const Ti
     }
 }
 
+// One round of the TMA-store epilogue for one epilogue warpgroup: its 128 rows (thread
+// = row) of 64 bytes each go into the warpgroup's staging buffer `buf` (64-byte swizzle:
+// 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)) and out with one TMA store
+// of the box at (x, y), issued by the warpgroup's first thread.  The buffer is rewritten
+// only after the previous round's store has read it.  Named barrier `bar` (128 threads)
+// orders the rounds.
+__device__ __forceinline__ void stage_store_round(uint32_t buf, int row, bool leader, uint32_t bar,
+                                                  const uint32_t (&w)[16], const CUtensorMap* map, int x, int y) {
+    if (leader) bulk_wait_read_all();
+    asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+    const uint32_t rowaddr = buf + static_cast<uint32_t>(row * 64);
+    const uint32_t sw = static_cast<uint32_t>((row >> 1) & 3);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        st_shared_v4(rowaddr + ((static_cast<uint32_t>(c) ^ sw) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
+                     w[4 * c + 3]);
+    fence_proxy_async_shared();
+    asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+    if (leader) {
+        tma_store_2d(map, buf, x, y);
+        bulk_commit();
+    }
+}
+
 // Spin for `ns` nanoseconds (bounded); lets copies already issued by a CTA
 // that gave up land before it leaves.
 __device__ __forceinline__ void settle_ns(uint64_t ns) {
@@ -460,7 +493,8 @@ __device__ __forceinline__ void settle_ns(uint64_t ns) {
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, 1)
     k_fp8_block_gemm(const __grid_constant__ CUtensorMap map_p,
-                     const __grid_constant__ CUtensorMap map_q, const GemmArgs args) {
+                     const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_d,
+                     const GemmArgs args) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -852,6 +886,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         const int quarter = warp & 3;     // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;  // accumulator lane = P-operand row
         const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
+        // the warpgroup's staging buffer, and the thread that issues its TMA stores
+        const uint32_t stage_buf = s_base + static_cast<uint32_t>(C::kOffStage + wg * C::kStageBytes);
+        const bool stage_leader = (ew & 3) == 0 && lane == 0;
+        if constexpr (!C::SWAP) {
+            if (ew == 0 && lane == 0) tma_prefetch_desc(&map_d);
+        }
         int sstage = 0, abuf = 0;
         uint32_t sphase = 0, aphase = 0;
         uint32_t fix_phase = 0;
@@ -1033,23 +1073,44 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 }
             }
             // ---- store the tile
+            // Dense and grouped tiles, TMA-store mode: each epilogue warpgroup sends its 128
+            // rows out through its staging buffer, 32 bf16 columns (or 64 E4M3 codes) per TMA
+            // store, which the tensor map clips at the M and N edges.  A tile whose rows end
+            // at a row_end inside the output (a masked or prefix-sum group's last rows), and
+            // every tile in direct mode, is stored row by row from the registers instead
+            // (16-byte stores; rows from row_end on stay untouched).
+            const bool whole_tile = args.tma_store != 0 && (tc.row_end >= args.M || tc.p0 + C::kP <= tc.row_end);
+            // the 64 bytes of this thread's row from column x; elem_bytes 2 (bf16) or 1 (E4M3)
+            auto out_round = [&](const uint32_t (&w)[16], int x, void* row_ptr, int elem_bytes) {
+                if (whole_tile) {
+                    stage_store_round(stage_buf, row, stage_leader, 1u + static_cast<uint32_t>(wg), w, &map_d, x, tc.p0);
+                } else if (row_ptr != nullptr) {
+                    // 16-byte chunks that lie inside the row (N is a multiple of 16)
+                    const int chunks = min(4, (args.N - x) * elem_bytes / 16);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        if (c < chunks)
+                            reinterpret_cast<uint4*>(row_ptr)[c] =
+                                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                }
+            };
             if constexpr (C::SILU) {
                 // h[m][q0 + wg*64 + i] = silu(gate_i) * up_i: acc[0 .. kCW/4) hold the gate
                 // columns in pairs, acc[kCW/4 ..) the up columns of the same outputs
                 const int m = tc.p0 + row;
                 const int n0 = tc.q0 + wg * (C::kCW / 2);
-                if (m < tc.row_end && n0 < args.N) {
-                    uint16_t* hrow = args.d + static_cast<long long>(m) * args.N + n0;
+                if (n0 < args.N) {
 #pragma unroll
-                    for (int c = 0; c < C::kCW / 16; ++c) {
-                        uint32_t w[4];
+                    for (int rr = 0; rr < C::kCW / 64; ++rr) {
+                        uint32_t w[16];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float2 g = acc[c * 4 + i];
-                            const float2 u = acc[C::kCW / 4 + c * 4 + i];
+                        for (int i = 0; i < 16; ++i) {
+                            const float2 g = acc[rr * 16 + i];
+                            const float2 u = acc[C::kCW / 4 + rr * 16 + i];
                             w[i] = pack_bf16x2(g.x / (1.0f + expf(-g.x)) * u.x, g.y / (1.0f + expf(-g.y)) * u.y);
                         }
-                        *reinterpret_cast<uint4*>(hrow + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                        const int n = n0 + 32 * rr;
+                        out_round(w, n, m < tc.row_end ? args.d + static_cast<long long>(m) * args.N + n : nullptr, 2);
                     }
                 }
             } else if constexpr (!C::SWAP) {
@@ -1071,8 +1132,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     if constexpr (C::kCW == 128) {
                         // this thread's 128 columns are one 1 x 128 group of row m: round
                         // to bf16 as the D store would, then quantize exactly as the
-                        // activation quantize kernel does
-                        if (n0 < args.N && m < tc.row_end) {
+                        // activation quantize kernel does (rows past M hold zeros and are
+                        // clipped by the store)
+                        if (n0 < args.N) {
                             uint32_t h[64];
 #pragma unroll
                             for (int i = 0; i < 64; ++i) h[i] = pack_bf16x2(acc[i].x, acc[i].y);
@@ -1083,39 +1145,52 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                             const float sv = scale_of_amax(amax);
                             float r_lo = 0.f, r_hi = 0.f;
                             if (sv >= 0x1p-125f) bracket_rcp(sv, r_lo, r_hi);
-                            uint8_t* qrow = args.q_out + static_cast<long long>(m) * args.N + n0;
+                            const bool zero_group = sv == 0.0f, exact_group = !(sv >= 0x1p-125f);
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const uint4 r0 = make_uint4(h[8 * j + 0], h[8 * j + 1], h[8 * j + 2], h[8 * j + 3]);
-                                const uint4 r1 = make_uint4(h[8 * j + 4], h[8 * j + 5], h[8 * j + 6], h[8 * j + 7]);
-                                const uint2 p0 = codes8(r0, sv, r_lo, r_hi, sv == 0.0f, !(sv >= 0x1p-125f));
-                                const uint2 p1 = codes8(r1, sv, r_lo, r_hi, sv == 0.0f, !(sv >= 0x1p-125f));
-                                *reinterpret_cast<uint4*>(qrow + 16 * j) = make_uint4(p0.x, p0.y, p1.x, p1.y);
+                            for (int rr = 0; rr < 2; ++rr) {
+                                // codes of columns 64 rr .. 64 rr + 63
+                                uint32_t w[16];
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const int k = 32 * rr + 4 * j;
+                                    const uint2 c = codes8(make_uint4(h[k], h[k + 1], h[k + 2], h[k + 3]), sv, r_lo, r_hi,
+                                                           zero_group, exact_group);
+                                    w[2 * j] = c.x;
+                                    w[2 * j + 1] = c.y;
+                                }
+                                out_round(w, n0 + 64 * rr,
+                                          m < tc.row_end ? args.q_out + static_cast<long long>(m) * args.N + n0 + 64 * rr
+                                                         : nullptr,
+                                          1);
                             }
-                            args.sfa_out[static_cast<long long>(n0 >> 7) * args.M4_out + m] = sv;
-                        } else if (n0 < args.N && m >= args.M && m < args.M4_out) {
-                            // rows past M up to the padded scale count carry a zero scale
-                            args.sfa_out[static_cast<long long>(n0 >> 7) * args.M4_out + m] = 0.f;
+                            if (m < tc.row_end) {
+                                args.sfa_out[static_cast<long long>(n0 >> 7) * args.M4_out + m] = sv;
+                            } else if (m >= args.M && m < args.M4_out) {
+                                // rows past M up to the padded scale count carry a zero scale
+                                args.sfa_out[static_cast<long long>(n0 >> 7) * args.M4_out + m] = 0.f;
+                            }
                         }
                     }
-                } else if (m < tc.row_end) {
-                    uint16_t* drow = args.d + static_cast<long long>(m) * args.N;
+                } else {
 #pragma unroll
-                    for (int c = 0; c < C::kCW / 8; ++c) {
-                        const int n = n0 + c * 8;
+                    for (int rr = 0; rr < C::kCW / 32; ++rr) {
+                        const int n = n0 + 32 * rr;
                         if (n < args.N) {
-                            uint4 w;
-                            w.x = pack_bf16x2(acc[c * 4 + 0].x, acc[c * 4 + 0].y);
-                            w.y = pack_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
-                            w.z = pack_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
-                            w.w = pack_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
-                            *reinterpret_cast<uint4*>(drow + n) = w;
+                            uint32_t w[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(acc[16 * rr + i].x, acc[16 * rr + i].y);
+                            out_round(w, n, m < tc.row_end ? args.d + static_cast<long long>(m) * args.N + n : nullptr, 2);
                         }
                     }
                 }
             } else {
                 store_decode_tile<C>(args, tc, row, wg * C::kCW, acc);
             }
+        }
+        // every TMA store of this warpgroup has completed before the CTA may leave
+        if constexpr (!C::SWAP) {
+            if (stage_leader) bulk_wait_all();
+            __syncwarp();
         }
     }
 

@@ -10,3 +10,13 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
+
+
+@pytest.fixture(params=[False, True], ids=["row_stores", "tma_store"])
+def store_path(request):
+    """Runs a GPU test with each output path of the dense and grouped GEMMs: every
+    thread storing its own row, and shared-memory staging with TMA stores."""
+    import moe_grouped_gemm_quantize_b200 as lnq
+    previous = lnq.lnq_set_tma_store(request.param)
+    yield request.param
+    lnq.lnq_set_tma_store(previous)

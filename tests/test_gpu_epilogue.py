@@ -34,7 +34,7 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 384, 512), (129, 256, 256), (8, 256, 1024), (64, 4096, 512)])
-def test_bias_bf16_output(M, N, K):
+def test_bias_bf16_output(M, N, K, store_path):
     a = synthetic.gaussian_bf16((M, K), 1.0, seed=M + N)
     w = synthetic.gaussian_bf16((N, K), 0.02, seed=N + K)
     bias = synthetic.gaussian_bf16((N,), 1.0, seed=K)
@@ -50,7 +50,7 @@ def test_bias_bf16_output(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,with_bias", [(203, 384, True), (256, 256, False), (1000, 512, True)])
-def test_fp8_output_exact_integer_case(M, N, with_bias):
+def test_fp8_output_exact_integer_case(M, N, with_bias, store_path):
     K = 128
     rng = np.random.default_rng(M + N)
     small = oracle.e4m3_encode(np.array([-1.0, 0.0, 1.0], np.float32))
@@ -73,7 +73,7 @@ def test_fp8_output_exact_integer_case(M, N, with_bias):
     assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
-def test_fp8_output_gaussian_against_the_oracle():
+def test_fp8_output_gaussian_against_the_oracle(store_path):
     M, N, K = 512, 1024, 1024
     a = synthetic.gaussian_bf16((M, K), 1.0, seed=5)
     w = synthetic.gaussian_bf16((N, K), 0.02, seed=6)

@@ -73,7 +73,7 @@ def weight_prefetch(request):
     (65, 256, 128), (100, 128, 256), (128, 16, 128), (130, 272, 384), (200, 640, 512),
     (257, 384, 640), (384, 1024, 1024), (129, 48, 256), (300, 4096, 128), (640, 768, 512),
 ])
-def test_dense_shapes_elementwise(M, N, K, dense_pairs, weight_prefetch):
+def test_dense_shapes_elementwise(M, N, K, dense_pairs, weight_prefetch, store_path):
     a = synthetic.gaussian_bf16((M, K), 1.0, seed=M + 7 * N + K)
     w = synthetic.gaussian_bf16((N, K), 0.02, seed=M + N + 3 * K)
     check_full(a, w, f"{M}x{N}x{K}")
@@ -123,7 +123,7 @@ def check_workload(name, what=None):
 
 
 @pytest.mark.parametrize("idx", range(4))
-def test_prefill_workloads_full(idx, dense_pairs):
+def test_prefill_workloads_full(idx, dense_pairs, store_path):
     check_workload(synthetic.PREFILL[idx].name)
 
 
@@ -132,7 +132,7 @@ def test_decode_workloads_full(idx, weight_prefetch):
     check_workload(synthetic.DECODE[idx].name)
 
 
-def test_square_outlier_workload_full(dense_pairs):
+def test_square_outlier_workload_full(dense_pairs, store_path):
     check_workload(synthetic.SQUARE.name)
 
 
@@ -149,7 +149,7 @@ def many_tiles_case():
     return a, w, oracle.gemm_nt(qa, sa, qb, sb)
 
 
-def test_many_tiles_per_cta_elementwise(dense_pairs, weight_prefetch):
+def test_many_tiles_per_cta_elementwise(dense_pairs, weight_prefetch, store_path):
     a, w, ref = many_tiles_case()
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     assert (a.shape[0] // 256) * (w.shape[0] // 256) > 3 * sms // 2

@@ -59,7 +59,7 @@ def run_oracle(a, w, m_indices, G):
     ([300, 17], 384, 1024),
     ([64, 200, 129, 3], 48, 256),
 ])
-def test_grouped_elementwise(sizes, N, K):
+def test_grouped_elementwise(sizes, N, K, store_path):
     a, w, m_indices, G = make_inputs(sizes, N, K, seed=sum(sizes) + N)
     d = run_gpu(a, w, m_indices, G)
     ref = run_oracle(a, w, m_indices, G)
@@ -67,7 +67,7 @@ def test_grouped_elementwise(sizes, N, K):
     assert_gemm_close(d[real], ref[real], f"grouped {sizes} N={N} K={K}")
 
 
-def test_blocks_led_by_a_pad_row_are_not_written():
+def test_blocks_led_by_a_pad_row_are_not_written(store_path):
     sizes = [130, 60]
     N, K = 256, 256
     a, w, m_indices, G = make_inputs(sizes, N, K, seed=3)
@@ -91,7 +91,7 @@ def test_single_group_equals_dense():
     assert np.array_equal(d, to_f64(dd))
 
 
-def test_moe_workload_full():
+def test_moe_workload_full(store_path):
     # every token row of the 32-expert MoE workload, element by element
     cfg = synthetic.MOE
     a, w, m_indices, _, _ = full_refs.moe_inputs()

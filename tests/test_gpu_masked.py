@@ -51,7 +51,7 @@ def run_gpu(a, w, masked, M_max, expected_m=0):
     ([200, 17], 256, 128, 1024),
     ([3, 128, 90], 128, 48, 256),
 ])
-def test_masked_elementwise(masked, M_max, N, K):
+def test_masked_elementwise(masked, M_max, N, K, store_path):
     G = len(masked)
     a, w = make_inputs(G, M_max, N, K, seed=G * 10 + N)
     d = run_gpu(a, w, masked, M_max)
@@ -67,7 +67,7 @@ def test_masked_elementwise(masked, M_max, N, K):
     assert np.all(np.isnan(got[~valid]))
 
 
-def test_decode_moe_workload_full():
+def test_decode_moe_workload_full(store_path):
     # 32 experts with 128-row buffers, 2048 routed tokens (multinomial, seed 3): every
     # token row is compared, each group's rows with the dense oracle product of its
     # weights (the definition of the masked product)

@@ -63,7 +63,7 @@ CASES = [
 
 @pytest.mark.parametrize("pairs", [0, 1])
 @pytest.mark.parametrize("sizes,alignment,N,K,extra", CASES)
-def test_psum_elementwise(sizes, alignment, N, K, extra, pairs):
+def test_psum_elementwise(sizes, alignment, N, K, extra, pairs, store_path):
     G = len(sizes)
     psum, starts, M_total = synthetic.psum_layout(sizes, alignment)
     M_total += extra
@@ -116,7 +116,7 @@ def test_128_alignment_matches_the_group_id_layout_bit_for_bit():
 
 
 @pytest.mark.parametrize("pairs", [0, 1])
-def test_moe_workload_full(pairs):
+def test_moe_workload_full(pairs, store_path):
     # the 32-expert MoE workload (16384 tokens, multinomial seed 0) moved into the
     # prefix-sum arena with 256-row alignment: every token row is compared with the
     # group-id layout's full reference (the same tokens, the same weights)

@@ -38,7 +38,7 @@ def run_gpu(a, w, pairs):
 @pytest.mark.parametrize("pairs", [0, 1])
 @pytest.mark.parametrize("M,I,K", [(300, 256, 512), (129, 128, 256), (100, 384, 256), (8, 128, 1024),
                                    (1000, 512, 384), (1, 256, 128)])
-def test_silu_mul_elementwise(M, I, K, pairs):
+def test_silu_mul_elementwise(M, I, K, pairs, store_path):
     a = synthetic.gaussian_bf16((M, K), 1.0, seed=M + I)
     w = synthetic.gaussian_bf16((2 * I, K), 0.05, seed=I + K)
     h = run_gpu(a, w, pairs)
@@ -64,7 +64,7 @@ def test_gate_and_up_are_not_swapped():
     assert np.all(np.abs(h) < 1e-30)
 
 
-def test_prefill_gate_up_full():
+def test_prefill_gate_up_full(store_path):
     # the prefill gate_up linear: M = 2048 tokens, I = 12288, K = 4096; h is compared
     # over the whole [M, I] output with silu(gate) * up of the full FP64 product
     cfg = synthetic.PREFILL[2]
