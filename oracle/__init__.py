@@ -94,6 +94,10 @@ def _load():
         lib.oracle_m_grouped_gemm_masked_points.restype = ctypes.c_int
         lib.oracle_m_grouped_gemm_masked_points.argtypes = [
             P, P, I64, P, P, P, ctypes.c_int32, I64, I64, I64, P, P, I64, P]
+        lib.oracle_quantize_mxfp8.restype = ctypes.c_int
+        lib.oracle_quantize_mxfp8.argtypes = [P, I64, I64, I64, P, I64, P]
+        lib.oracle_gemm_nt_mx32.restype = ctypes.c_int
+        lib.oracle_gemm_nt_mx32.argtypes = [P, P, P, P, I64, I64, I64, P]
         _lib = lib
         return lib
 
@@ -350,3 +354,33 @@ def ue8m0_value(sfe) -> np.ndarray:
     """The scale 2^(b - 127) of UE8M0 bytes, as float32 (exact for b in 0..254)."""
     b = np.asarray(sfe, dtype=np.int32)
     return np.ldexp(np.float32(1.0), b - 127).astype(np.float32)
+
+
+MX_BLOCK = 32
+
+
+def quantize_mxfp8(x_bf16_bits: np.ndarray):
+    """MXFP8 gran-32: every row of a bf16 matrix (uint16 bits [R, K]) in 1x32 blocks
+    along K, each with the UE8M0 scale 2^(sfe - 127), the smallest power of two p with
+    448 p >= amax (deepgemm-rust README, benchmark block "SM100 FP8: DeepSeek gran-128
+    recipe and MXFP8 gran-32").  Returns (q uint8 [R, K], sfe uint8 [R, K/32])."""
+    x = _c(x_bf16_bits, np.uint16)
+    R, K = x.shape
+    q = np.empty((R, K), dtype=np.uint8)
+    sfe = np.empty((R, K // MX_BLOCK), dtype=np.uint8)
+    _check(_load().oracle_quantize_mxfp8(_ptr(x), R, K, K, _ptr(q), K, _ptr(sfe)), "quantize_mxfp8")
+    return q, sfe
+
+
+def gemm_nt_mx32(qa, ea, qb, eb) -> np.ndarray:
+    """FP64 D [M, N] of two MXFP8 gran-32 operands: codes qa [M, K], qb [N, K] with
+    exponent bytes ea [M, K/32], eb [N, K/32]."""
+    qa = _c(qa, np.uint8)
+    qb = _c(qb, np.uint8)
+    ea = _c(ea, np.uint8)
+    eb = _c(eb, np.uint8)
+    M, K = qa.shape
+    N = qb.shape[0]
+    D = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_gemm_nt_mx32(_ptr(qa), _ptr(ea), _ptr(qb), _ptr(eb), M, N, K, _ptr(D)), "gemm_nt_mx32")
+    return D

@@ -685,3 +685,80 @@ int oracle_quantize_ue8m0_blocks(const uint16_t* w, int64_t N, int64_t K, uint8_
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* MXFP8 gran-32 (deepgemm-rust README, benchmark block "SM100 FP8: DeepSeek gran-128
+ * recipe and MXFP8 gran-32"; kernel table, kind::mxf8f6f4): every row of an operand,
+ * activations and weights alike, in 1 x 32 blocks along K, each block with its own
+ * UE8M0 scale chosen by the rule of the gran-128 recipe above (the smallest power of two
+ * p with 448 p >= amax; p = 1 for an all-zero block), codes the E4M3 RNE of x / p.
+ *   x    bf16 [R][ld_x];  q  E4M3 [R][ld_q];
+ *   sfe  uint8 [R][K/32], sfe[r*(K/32) + b] = e + 127 of row r's block b. */
+#define ORACLE_MX_BLOCK 32
+
+int oracle_quantize_mxfp8(const uint16_t* x, int64_t R, int64_t K, int64_t ld_x, uint8_t* q, int64_t ld_q,
+                          uint8_t* sfe)
+{
+    int64_t B, r;
+    if (R <= 0 || K <= 0 || K % ORACLE_MX_BLOCK != 0 || ld_x < K || ld_q < K)
+        return -1;
+    B = K / ORACLE_MX_BLOCK;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < R; ++r) {
+        int64_t b, k;
+        for (b = 0; b < B; ++b) {
+            float amax = 0.0f;
+            int e;
+            for (k = 0; k < ORACLE_MX_BLOCK; ++k) {
+                float v = fabsf(bf16_bits_to_float(x[r * ld_x + b * ORACLE_MX_BLOCK + k]));
+                if (v > amax)
+                    amax = v;
+            }
+            e = ue8m0_exponent(amax);
+            sfe[r * B + b] = (uint8_t)(e + 127);
+            for (k = 0; k < ORACLE_MX_BLOCK; ++k) {
+                int64_t col = b * ORACLE_MX_BLOCK + k;
+                q[r * ld_q + col] = quantize_pow2(bf16_bits_to_float(x[r * ld_x + col]), e);
+            }
+        }
+    }
+    return 0;
+}
+
+/* D[m][n] = sum_k (value(qa[m][k]) * 2^(ea[m][k/32] - 127)) * (value(qb[n][k]) * 2^(eb[n][k/32] - 127))
+ * in FP64 (each term exact), for qa [M][K], ea [M][K/32], qb [N][K], eb [N][K/32]; D [M][N]. */
+int oracle_gemm_nt_mx32(const uint8_t* qa, const uint8_t* ea, const uint8_t* qb, const uint8_t* eb, int64_t M,
+                        int64_t N, int64_t K, double* D)
+{
+    double* bd;
+    int64_t n, m, B;
+    if (M <= 0 || N <= 0 || K <= 0 || K % ORACLE_MX_BLOCK != 0)
+        return -1;
+    B = K / ORACLE_MX_BLOCK;
+    bd = (double*)malloc(sizeof(double) * (size_t)N * (size_t)K);
+    if (!bd)
+        return -2;
+#pragma omp parallel for schedule(static)
+    for (n = 0; n < N; ++n) {
+        int64_t k;
+        for (k = 0; k < K; ++k)
+            bd[n * K + k] = oracle_e4m3_value(qb[n * K + k]) * ldexp(1.0, (int)eb[n * B + k / ORACLE_MX_BLOCK] - 127);
+    }
+#pragma omp parallel
+    {
+        double* ad = (double*)malloc(sizeof(double) * (size_t)K);
+#pragma omp for schedule(dynamic, 1)
+        for (m = 0; m < M; ++m) {
+            int64_t j, k;
+            if (!ad)
+                continue;
+            for (k = 0; k < K; ++k)
+                ad[k] = oracle_e4m3_value(qa[m * K + k]) * ldexp(1.0, (int)ea[m * B + k / ORACLE_MX_BLOCK] - 127);
+            for (j = 0; j < N; ++j)
+                D[m * N + j] = dot(ad, bd + j * K, K);
+        }
+        free(ad);
+    }
+    free(bd);
+    return 0;
+}

@@ -9,7 +9,9 @@ the wrong scale of an all-zero group, a block amax over one row, an off-by-one g
 the next group's weights, the plain (non-aligned) row order of the prefix-sum layout, a
 dropped weight scale, a wrong rounding of E4M3 ties, a wrong scale divisor, row-major
 instead of MN-major activation scales, a transposed activation-scale index in the product,
-and a masked count taken as inclusive.
+a masked count taken as inclusive, and for the MXFP8 gran-32 recipe a scale index taken per
+128 columns, a weight scale read from the wrong row and a block's scale stored at the next
+block.
 """
 import os
 import subprocess
@@ -76,6 +78,18 @@ MUTATIONS = {
         "            if (m >= masked_m[gr] || !ad || !bd)",
         "            if (m > masked_m[gr] || !ad || !bd)",
         "tests/test_oracle_masked.py"),
+    "mx32_product_block_per_128": (
+        "            ad[k] = oracle_e4m3_value(qa[m * K + k]) * ldexp(1.0, (int)ea[m * B + k / ORACLE_MX_BLOCK] - 127);",
+        "            ad[k] = oracle_e4m3_value(qa[m * K + k]) * ldexp(1.0, (int)ea[m * B + (k / 128) * 4] - 127);",
+        "tests/test_oracle_mxfp8.py"),
+    "mx32_weight_scale_from_activation_row": (
+        "            bd[n * K + k] = oracle_e4m3_value(qb[n * K + k]) * ldexp(1.0, (int)eb[n * B + k / ORACLE_MX_BLOCK] - 127);",
+        "            bd[n * K + k] = oracle_e4m3_value(qb[n * K + k]) * ldexp(1.0, (int)eb[k / ORACLE_MX_BLOCK] - 127);",
+        "tests/test_oracle_mxfp8.py"),
+    "mx32_quantize_scale_of_next_block": (
+        "            sfe[r * B + b] = (uint8_t)(e + 127);",
+        "            sfe[r * B + (b + 1) % B] = (uint8_t)(e + 127);",
+        "tests/test_oracle_mxfp8.py"),
     "gemm_weight_scale_dropped": (
         "        out[k] = oracle_e4m3_value(qb[row * K + k]) * (double)sfb[sb_row * KB + k / ORACLE_GROUP];",
         "        out[k] = oracle_e4m3_value(qb[row * K + k]);",
