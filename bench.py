@@ -205,9 +205,13 @@ class Linear:
         self.cfg = cfg
         a, w = synthetic.make_linear_inputs(cfg)
         self.x = a.to(dev)
-        # UE8M0 recipe: power-of-two scales applied by the tensor core (no promotion)
-        self.ue8m0 = recipe == "ue8m0"
-        if self.ue8m0:
+        # UE8M0 recipes: power-of-two scales applied by the tensor core (no promotion), in
+        # 1x128 / 128x128 blocks (ue8m0) or 1x32 blocks on both operands (mxfp8)
+        self.recipe = recipe
+        self.ue8m0 = recipe in ("ue8m0", "mxfp8")
+        if recipe == "mxfp8":
+            self.wq, self.ws = lnq.quantize_mxfp8(w.to(dev))
+        elif self.ue8m0:
             self.wq, self.ws = lnq.quantize_weights_ue8m0(w.to(dev))
         else:
             self.wq, self.ws = lnq.quantize_weights(w.to(dev))
@@ -271,6 +275,8 @@ class Linear:
                      P(self.sfa.data_ptr()), s)
             margs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), P(self.wq.data_ptr()), P(self.ws.data_ptr()),
                      P(self.d.data_ptr()), c.M, c.N, c.K, s)
+            if self.recipe == "mxfp8":
+                return (L.lnq_quantize_mxfp8, qargs), (L.lnq_mxfp8_gemm_nt, margs)
             return (L.lnq_quantize_ue8m0_groups, qargs), (L.lnq_mx_block_gemm_nt, margs)
         qargs = (P(self.x.data_ptr()), c.M, c.K, self.x.stride(0), P(self.q.data_ptr()), c.K,
                  P(self.sfa.data_ptr()), self.M4, s)
@@ -301,12 +307,15 @@ class Grouped:
         from moe_grouped_gemm_quantize_b200 import synthetic
         self.cfg = cfg
         self.alignment = alignment
-        # UE8M0 recipe (group-id layout only): power-of-two scales applied by the tensor core
-        self.ue8m0 = recipe == "ue8m0" and alignment is None
+        # UE8M0 recipes (group-id layout only): power-of-two scales applied by the tensor core
+        self.recipe = recipe
+        self.ue8m0 = recipe in ("ue8m0", "mxfp8") and alignment is None
         a, w, m_indices, sizes = synthetic.make_moe_inputs(cfg, alignment=alignment or 128)
         self.M = a.shape[0]
         self.x = a.to(dev)
-        if self.ue8m0:
+        if self.ue8m0 and recipe == "mxfp8":
+            self.wq, self.ws = lnq.quantize_mxfp8(w.to(dev))
+        elif self.ue8m0:
             self.wq, self.ws = lnq.quantize_weights_ue8m0(w.to(dev))
         else:
             self.wq, self.ws = lnq.quantize_weights_grouped(w.to(dev), cfg.groups)
@@ -346,6 +355,8 @@ class Grouped:
             qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K, P(self.sfa.data_ptr()), s)
             gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), P(self.wq.data_ptr()), P(self.ws.data_ptr()),
                      P(self.mi.data_ptr()), c.groups, P(self.d.data_ptr()), self.M, c.N, c.K, s)
+            if self.recipe == "mxfp8":
+                return (L.lnq_quantize_mxfp8, qargs), (L.lnq_m_grouped_mxfp8_gemm_contiguous, gargs)
             return (L.lnq_quantize_ue8m0_groups, qargs), (L.lnq_m_grouped_mx_gemm_contiguous, gargs)
         qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K,
                  P(self.sfa.data_ptr()), self.M, s)
@@ -657,7 +668,7 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
         iso = [u.flops / (statistics.median(t) * 1e-3) / 1e12 for u, t in zip(units, per_gemm)]
     ue8m0 = any(getattr(u, "ue8m0", False) for u in units)
     kernel_name = "k_mx_block_gemm" if ue8m0 else "k_fp8_block_gemm"
-    roof["traffic"] = recorded_traffic(kernel_name, name)
+    roof["traffic"] = recorded_traffic(kernel_name, name if args.recipe == "fp32" else f"{name}_{args.recipe}")
     roof["kernel"] = kernel_name
     roof["peak_source"] = peak_note
     roof["duration"] = ("mean period per GEMM launch over the workload's GEMMs captured back to "
@@ -688,7 +699,9 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
         "clocks": clocks.summary(),
         "e2e": e2e,
         "desc": WORKLOAD_DESC[name],
-        "recipe": ("UE8M0 power-of-two scales in the tensor core" if ue8m0
+        "recipe": ("MXFP8 gran-32: UE8M0 scales per 1x32 block on both operands, in the tensor core"
+                   if args.recipe == "mxfp8" else
+                   "UE8M0 power-of-two scales (gran-128) in the tensor core" if ue8m0
                    else "FP32 scales, per-128-K-block promotion"),
         "epilogue": ("fp8 output (E4M3 + 1x128 scales)" if any(getattr(u, "fp8_out", False) for u in units)
                      else "gate_up with SiLU.mul (bf16 h)" if any(getattr(u, "silu", False) for u in units)
@@ -741,7 +754,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": ("e4m3 x e4m3 with UE8M0 block scales -> f32 accumulate, bf16 out" if args.recipe == "ue8m0"
+        "dtype": ("e4m3 x e4m3 with UE8M0 block scales -> f32 accumulate, bf16 out" if args.recipe != "fp32"
                   else "e4m3 x e4m3 -> f32 accumulate, bf16 out"),
         "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights, bf16)",
         "config": {"workload": (f"{head_name} (headline; every workload under `configs`)"
@@ -946,9 +959,10 @@ def main():
                          "per CTA at N = 12288 on B200)")
     ap.add_argument("--no-weight-prefetch", action="store_true",
                     help="GEMMs wait for the previous kernel before streaming weights")
-    ap.add_argument("--recipe", choices=["fp32", "ue8m0"], default="fp32",
-                    help="dense and moe workloads: FP32 scales with promotion (the default), or UE8M0 "
-                         "power-of-two scales applied by the block-scaled MMA")
+    ap.add_argument("--recipe", choices=["fp32", "ue8m0", "mxfp8"], default="fp32",
+                    help="dense and moe workloads: FP32 scales with promotion (the default), UE8M0 "
+                         "power-of-two scales in 1x128 / 128x128 blocks, or MXFP8 gran-32 (1x32 UE8M0 "
+                         "blocks on both operands), both applied by the block-scaled MMA")
     ap.add_argument("--grouped-cta-pairs", type=int, default=0, choices=[0, 1],
                     help="moe_psum: 256x256 tiles on CTA pairs (1) or 128-row tiles (0)")
     ap.add_argument("--tma-store", type=int, default=1, choices=[0, 1],

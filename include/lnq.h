@@ -379,6 +379,44 @@ lnq_status lnq_m_grouped_mx_gemm_contiguous(const void* a_e4m3, const void* sfa_
                                             const void* sfb_atoms, const int32_t* m_indices, int32_t num_groups,
                                             void* d_bf16, int64_t M_total, int64_t N, int64_t K, void* stream);
 
+/*
+ * MXFP8 gran-32 recipe (deepgemm-rust README, benchmark block "SM100 FP8:
+ * DeepSeek gran-128 recipe and MXFP8 gran-32"; kernel table, kind::mxf8f6f4
+ * with UE8M0 scales).  Every row of an operand, activations and weights alike,
+ * is quantized in 1 x 32 blocks along K, each block with its own UE8M0 scale
+ * chosen by the rule of the gran-128 recipe above (the smallest power of two p
+ * with 448 p >= amax; p = 1 for an all-zero block), codes the E4M3 RNE of x / p.
+ *
+ * Scale atoms as for the gran-128 recipe ([K/128][ceil(rows/128)][128] uint32
+ * words, row r = r0 + 32 r1 of a 128-row block in word 4 r0 + r1), except that
+ * the word of a row holds the exponent bytes of its four 32-blocks of the 128-wide
+ * K block: 32-block j in byte j.  The tensor core reads byte j for the j-th K = 32
+ * step (the scale-ID fields of the block-scaled MMA).
+ *
+ * lnq_quantize_mxfp8: x bf16 [rows][ld_x] -> q E4M3 [rows][ld_q] and sf_atoms
+ *   uint32 [K/128][ceil(rows/128)][128]; rows past `rows` in the last 128-row
+ *   block get p = 1 in all four bytes.  The same call quantizes activations and
+ *   weights.  Requires K % 128 == 0, ld_x % 8 == 0, ld_q % 16 == 0, pointers
+ *   16-byte aligned.
+ * lnq_mxfp8_gemm_nt: D[m][n] = bf16( sum_k a[m][k] 2^ea[m][k/32] b[n][k]
+ *   2^eb[n][k/32] ), the scales applied by the tensor core
+ *   (tcgen05.mma kind::mxf8f6f4.block_scale, one scale byte per row per K = 32)
+ *   and the sum accumulated in FP32 over the whole K range.  a_e4m3 [M][K],
+ *   b_e4m3 [N][K], d_bf16 [M][N] fully overwritten.  Requires N % 16 == 0,
+ *   K % 128 == 0, pointers 16-byte aligned.
+ * lnq_m_grouped_mxfp8_gemm_contiguous: the same for the M-grouped contiguous
+ *   layout, with the arguments and requirements of
+ *   lnq_m_grouped_mx_gemm_contiguous (sfb_atoms from lnq_quantize_mxfp8 over all
+ *   num_groups*N weight rows).
+ */
+lnq_status lnq_quantize_mxfp8(const void* x_bf16, int64_t rows, int64_t K, int64_t ld_x, void* q_e4m3, int64_t ld_q,
+                              void* sf_atoms, void* stream);
+lnq_status lnq_mxfp8_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3, const void* sfb_atoms,
+                             void* d_bf16, int64_t M, int64_t N, int64_t K, void* stream);
+lnq_status lnq_m_grouped_mxfp8_gemm_contiguous(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                               const void* sfb_atoms, const int32_t* m_indices, int32_t num_groups,
+                                               void* d_bf16, int64_t M_total, int64_t N, int64_t K, void* stream);
+
 /* Static text for a status code. */
 const char* lnq_status_string(lnq_status status);
 

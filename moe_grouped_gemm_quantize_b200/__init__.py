@@ -29,7 +29,8 @@ __all__ = [
     "lnq_quantize_fp8_groups", "lnq_quantize_fp8_blocks", "lnq_fp8_block_gemm_nt",
     "lnq_m_grouped_fp8_gemm_contiguous", "lnq_m_grouped_fp8_gemm_contiguous_psum",
     "lnq_fp8_block_gemm_nt_silu_mul", "lnq_mx_block_gemm_nt", "lnq_m_grouped_mx_gemm_contiguous", "quantize_activations_ue8m0",
-    "quantize_weights_ue8m0", "ue8m0_atoms",
+    "quantize_weights_ue8m0", "ue8m0_atoms", "quantize_mxfp8", "lnq_mxfp8_gemm_nt",
+    "lnq_m_grouped_mxfp8_gemm_contiguous",
     "lnq_m_grouped_fp8_gemm_masked", "lnq_get_last_device_error", "lnq_status_string",
     "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs",
     "lnq_set_weight_prefetch", "lnq_set_tma_store",
@@ -87,6 +88,9 @@ def lib() -> ctypes.CDLL:
             "lnq_quantize_ue8m0_blocks": [P, I64, I64, P, P, P],
             "lnq_mx_block_gemm_nt": [P, P, P, P, P, I64, I64, I64, P],
             "lnq_m_grouped_mx_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
+            "lnq_quantize_mxfp8": [P, I64, I64, I64, P, I64, P, P],
+            "lnq_mxfp8_gemm_nt": [P, P, P, P, P, I64, I64, I64, P],
+            "lnq_m_grouped_mxfp8_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
             "lnq_get_last_device_error": [P],
             "lnq_selftest_wait_timeout": [I64, P],
         }
@@ -390,6 +394,61 @@ def lnq_m_grouped_mx_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: torc
     _check(lib().lnq_m_grouped_mx_gemm_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(m_indices), G,
                                                   _ptr(d), M_total, N, K, _stream(stream)),
            "lnq_m_grouped_mx_gemm_contiguous")
+
+
+def quantize_mxfp8(x: torch.Tensor, stream=None):
+    """MXFP8 gran-32: every row in 1x32 blocks along K (activations and weights alike):
+    (q e4m3 [rows, K], scale atoms int32 [K/128, ceil(rows/128)*128], four exponent bytes
+    per word)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise TypeError("x must be a row-major bf16 matrix")
+    R, K = x.shape
+    q = torch.empty((R, K), dtype=torch.float8_e4m3fn, device=x.device)
+    sf = ue8m0_atoms(R, K, x.device)
+    _check(lib().lnq_quantize_mxfp8(_ptr(x), R, K, x.stride(0), _ptr(q), K, _ptr(sf), _stream(stream)),
+           "lnq_quantize_mxfp8")
+    return q, sf
+
+
+def lnq_mxfp8_gemm_nt(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                      d: torch.Tensor, stream=None) -> None:
+    """MXFP8 gran-32 GEMM: a e4m3 [M, K], b e4m3 [N, K], their scale atoms, d bf16 [M, N]."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.int32 or sfb.dtype != torch.int32 or \
+            d.dtype != torch.bfloat16:
+        raise TypeError("a, b e4m3; sfa, sfb int32 scale atoms; d bf16")
+    for t in (a, sfa, b, sfb, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K or tuple(d.shape) != (M, N) or tuple(sfa.shape) != (K // 128, -(-M // 128) * 128) or \
+            tuple(sfb.shape) != (K // 128, -(-N // 128) * 128):
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_mxfp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream(stream)),
+           "lnq_mxfp8_gemm_nt")
+
+
+def lnq_m_grouped_mxfp8_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                                        m_indices: torch.Tensor, num_groups: int, d: torch.Tensor,
+                                        stream=None) -> None:
+    """MXFP8 gran-32, M-grouped contiguous: as lnq_m_grouped_mx_gemm_contiguous with the scale
+    atoms of lnq_quantize_mxfp8 on both operands."""
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.int32 or sfb.dtype != torch.int32 or \
+            d.dtype != torch.bfloat16 or m_indices.dtype != torch.int32:
+        raise TypeError("a, b e4m3; sfa, sfb int32 scale atoms; m_indices int32; d bf16")
+    for t in (a, sfa, b, sfb, m_indices, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    M_total, K = a.shape
+    G = int(num_groups)
+    N = d.shape[1]
+    if b.shape[0] != G * N or b.shape[1] != K or d.shape[0] != M_total or m_indices.shape[0] != M_total or \
+            tuple(sfa.shape) != (K // 128, -(-M_total // 128) * 128) or \
+            tuple(sfb.shape) != (K // 128, -(-G * N // 128) * 128):
+        raise ValueError("inconsistent shapes")
+    _check(lib().lnq_m_grouped_mxfp8_gemm_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(m_indices), G,
+                                                     _ptr(d), M_total, N, K, _stream(stream)),
+           "lnq_m_grouped_mxfp8_gemm_contiguous")
 
 
 def lnq_m_grouped_fp8_gemm_contiguous_psum(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,

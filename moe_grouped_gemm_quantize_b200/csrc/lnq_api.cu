@@ -445,26 +445,69 @@ lnq_status lnq_quantize_ue8m0_blocks(const void* w_bf16, int64_t N, int64_t K, v
     return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
 }
 
-lnq_status lnq_mx_block_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
-                                const void* sfb_atoms, void* d_bf16, int64_t M, int64_t N, int64_t K,
-                                void* stream) {
-    using C = MxCfg<4>;
-    if (M <= 0 || N <= 0 || K <= 0) return LNQ_ERR_INVALID_ARG;
-    if (K % 128 != 0 || N % 16 != 0 || M > kMaxRows || N > kMaxRows || K > (int64_t{1} << 31))
-        return LNQ_ERR_UNSUPPORTED_SHAPE;
-    if (!a_e4m3 || !sfa_atoms || !b_e4m3 || !sfb_atoms || !d_bf16) return LNQ_ERR_INVALID_ARG;
-    if (!aligned16(a_e4m3) || !aligned16(sfa_atoms) || !aligned16(b_e4m3) || !aligned16(sfb_atoms) ||
-        !aligned16(d_bf16))
+lnq_status lnq_quantize_mxfp8(const void* x_bf16, int64_t rows, int64_t K, int64_t ld_x, void* q_e4m3, int64_t ld_q,
+                              void* sf_atoms, void* stream) {
+    if (rows <= 0 || K <= 0 || ld_x < K || ld_q < K) return LNQ_ERR_INVALID_ARG;
+    if (K % 128 != 0 || rows > kMaxRows || K > (int64_t{1} << 31)) return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!x_bf16 || !q_e4m3 || !sf_atoms) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(q_e4m3) || !aligned16(sf_atoms) || ld_x % 8 != 0 || ld_q % 16 != 0)
         return LNQ_ERR_MISALIGNED;
     DeviceInfo* dev = nullptr;
     lnq_status st = device_info(&dev);
     if (st != LNQ_OK) return st;
+    const int64_t Rpad = (rows + 127) / 128 * 128;
+    const int64_t units = Rpad * (K / 128);
+    const int64_t want = (units + 15) / 16;  // 8 warps of two four-group halves per CTA
+    const int grid = static_cast<int>(want < 4 * dev->sm_count ? want : 4 * dev->sm_count);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_quantize_mxfp8, static_cast<const uint16_t*>(x_bf16), static_cast<int>(rows),
+                           static_cast<int>(K), static_cast<long long>(ld_x), static_cast<uint8_t*>(q_e4m3),
+                           static_cast<long long>(ld_q), static_cast<uint32_t*>(sf_atoms),
+                           static_cast<int>(Rpad)) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace {
+
+// The block-scaled product of the UE8M0 recipes: gran-128 scales (GRAN32 false) or the
+// MXFP8 gran-32 scales, dense or M-grouped contiguous (m_indices != nullptr).
+template <bool GRAN32>
+lnq_status mx_gemm(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3, const void* sfb_atoms,
+                   const int32_t* m_indices, int32_t num_groups, void* d_bf16, int64_t M, int64_t N, int64_t K,
+                   void* stream) {
+    using C = MxCfg<4>;
+    const bool grouped = m_indices != nullptr;
+    if (M <= 0 || N <= 0 || K <= 0 || (grouped && num_groups <= 0)) return LNQ_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N % 16 != 0 || M > kMaxRows || N > kMaxRows || K > (int64_t{1} << 31))
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (grouped && (M % 128 != 0 || N % 128 != 0 || static_cast<int64_t>(num_groups) * N > kMaxRows))
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (!a_e4m3 || !sfa_atoms || !b_e4m3 || !sfb_atoms || !d_bf16) return LNQ_ERR_INVALID_ARG;
+    if (!aligned16(a_e4m3) || !aligned16(sfa_atoms) || !aligned16(b_e4m3) || !aligned16(sfb_atoms) ||
+        !aligned16(d_bf16) || (grouped && !aligned4(m_indices)))
+        return LNQ_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    lnq_status st = device_info(&dev);
+    if (st != LNQ_OK) return st;
+    const int64_t wrows = grouped ? static_cast<int64_t>(num_groups) * N : N;
     CUtensorMap map_a, map_b;
     st = encode_e4m3_map(&map_a, a_e4m3, M, K, 128);
-    if (st == LNQ_OK) st = encode_e4m3_map(&map_b, b_e4m3, N, K, 256);
+    if (st == LNQ_OK) st = encode_e4m3_map(&map_b, b_e4m3, wrows, K, 256);
     if (st != LNQ_OK) return st;
-    static std::atomic<bool> attr_set[kMaxDevices];
-    st = smem_attr_once(attr_set, dev->ordinal, k_mx_block_gemm<4>, C::kSmemBytes);
+    static std::atomic<bool> attr_dense[kMaxDevices], attr_grouped[kMaxDevices];
+    st = grouped ? smem_attr_once(attr_grouped, dev->ordinal, k_mx_block_gemm<4, true, GRAN32>, C::kSmemBytes)
+                 : smem_attr_once(attr_dense, dev->ordinal, k_mx_block_gemm<4, false, GRAN32>, C::kSmemBytes);
     if (st != LNQ_OK) return st;
     MxArgs args{};
     args.sfa = static_cast<const uint32_t*>(sfa_atoms);
@@ -476,10 +519,12 @@ lnq_status lnq_mx_block_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const
     args.N = static_cast<int>(N);
     args.num_kb = static_cast<int>(K / 128);
     args.mblocks = static_cast<int>((M + 127) / 128);
-    args.nblocks = static_cast<int>((N + 127) / 128);
+    args.nblocks = static_cast<int>((wrows + 127) / 128);
     args.tiles_p = args.mblocks;
     args.tiles_q = static_cast<int>((N + 255) / 256);
     args.num_tiles = args.tiles_p * args.tiles_q;
+    args.m_indices = m_indices;
+    args.num_groups = grouped ? num_groups : 1;
     const int grid = args.num_tiles < dev->sm_count ? args.num_tiles : dev->sm_count;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -491,8 +536,33 @@ lnq_status lnq_mx_block_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const
     cfg.stream = static_cast<cudaStream_t>(stream);
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4>, map_a, map_b, args) != cudaSuccess) return LNQ_ERR_CUDA;
+    const cudaError_t e = grouped ? cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4, true, GRAN32>, map_a, map_b, args)
+                                  : cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4, false, GRAN32>, map_a, map_b, args);
+    if (e != cudaSuccess) return LNQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+lnq_status lnq_mxfp8_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3, const void* sfb_atoms,
+                             void* d_bf16, int64_t M, int64_t N, int64_t K, void* stream) {
+    return mx_gemm<true>(a_e4m3, sfa_atoms, b_e4m3, sfb_atoms, nullptr, 0, d_bf16, M, N, K, stream);
+}
+
+lnq_status lnq_m_grouped_mxfp8_gemm_contiguous(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                               const void* sfb_atoms, const int32_t* m_indices, int32_t num_groups,
+                                               void* d_bf16, int64_t M_total, int64_t N, int64_t K, void* stream) {
+    if (!m_indices) return LNQ_ERR_INVALID_ARG;
+    return mx_gemm<true>(a_e4m3, sfa_atoms, b_e4m3, sfb_atoms, m_indices, num_groups, d_bf16, M_total, N, K,
+                         stream);
+}
+
+lnq_status lnq_mx_block_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                const void* sfb_atoms, void* d_bf16, int64_t M, int64_t N, int64_t K,
+                                void* stream) {
+    return mx_gemm<false>(a_e4m3, sfa_atoms, b_e4m3, sfb_atoms, nullptr, 0, d_bf16, M, N, K, stream);
 }
 
 namespace {
@@ -782,55 +852,9 @@ lnq_status lnq_fp8_block_gemm_nt_silu_mul(const void* a_e4m3, const float* sfa, 
 lnq_status lnq_m_grouped_mx_gemm_contiguous(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
                                             const void* sfb_atoms, const int32_t* m_indices, int32_t num_groups,
                                             void* d_bf16, int64_t M_total, int64_t N, int64_t K, void* stream) {
-    using C = MxCfg<4>;
-    if (M_total <= 0 || N <= 0 || K <= 0 || num_groups <= 0) return LNQ_ERR_INVALID_ARG;
-    if (M_total % 128 != 0 || N % 128 != 0 || K % 128 != 0 || M_total > kMaxRows || K > (int64_t{1} << 31) ||
-        static_cast<int64_t>(num_groups) * N > kMaxRows)
-        return LNQ_ERR_UNSUPPORTED_SHAPE;
-    if (!a_e4m3 || !sfa_atoms || !b_e4m3 || !sfb_atoms || !m_indices || !d_bf16) return LNQ_ERR_INVALID_ARG;
-    if (!aligned16(a_e4m3) || !aligned16(sfa_atoms) || !aligned16(b_e4m3) || !aligned16(sfb_atoms) ||
-        !aligned16(d_bf16) || !aligned4(m_indices))
-        return LNQ_ERR_MISALIGNED;
-    DeviceInfo* dev = nullptr;
-    lnq_status st = device_info(&dev);
-    if (st != LNQ_OK) return st;
-    const int64_t wrows = static_cast<int64_t>(num_groups) * N;
-    CUtensorMap map_a, map_b;
-    st = encode_e4m3_map(&map_a, a_e4m3, M_total, K, 128);
-    if (st == LNQ_OK) st = encode_e4m3_map(&map_b, b_e4m3, wrows, K, 256);
-    if (st != LNQ_OK) return st;
-    static std::atomic<bool> attr_set[kMaxDevices];
-    st = smem_attr_once(attr_set, dev->ordinal, k_mx_block_gemm<4, true>, C::kSmemBytes);
-    if (st != LNQ_OK) return st;
-    MxArgs args{};
-    args.sfa = static_cast<const uint32_t*>(sfa_atoms);
-    args.sfb = static_cast<const uint32_t*>(sfb_atoms);
-    args.d = static_cast<uint16_t*>(d_bf16);
-    args.status = dev->status;
-    args.timeout_ns = kDefaultTimeoutNs;
-    args.M = static_cast<int>(M_total);
-    args.N = static_cast<int>(N);
-    args.num_kb = static_cast<int>(K / 128);
-    args.mblocks = static_cast<int>(M_total / 128);
-    args.nblocks = static_cast<int>(wrows / 128);
-    args.tiles_p = args.mblocks;
-    args.tiles_q = static_cast<int>((N + 255) / 256);
-    args.num_tiles = args.tiles_p * args.tiles_q;
-    args.m_indices = m_indices;
-    args.num_groups = num_groups;
-    const int grid = args.num_tiles < dev->sm_count ? args.num_tiles : dev->sm_count;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(C::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = static_cast<cudaStream_t>(stream);
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4, true>, map_a, map_b, args) != cudaSuccess) return LNQ_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+    if (!m_indices) return LNQ_ERR_INVALID_ARG;
+    return mx_gemm<false>(a_e4m3, sfa_atoms, b_e4m3, sfb_atoms, m_indices, num_groups, d_bf16, M_total, N, K,
+                          stream);
 }
 
 lnq_status lnq_m_grouped_fp8_gemm_contiguous_psum(const void* a_e4m3, const float* sfa,

@@ -22,6 +22,13 @@
 // MMA reads row r's scale at lane r, column base + r / 32, byte 0.
 //   activations: [K/128][ceil(M/128)][128] words;
 //   weights:     [K/128][ceil(N/128)][128] words, every row of a block the block's.
+//
+// The MXFP8 gran-32 recipe (deepgemm-rust README, benchmark block "SM100 FP8: DeepSeek
+// gran-128 recipe and MXFP8 gran-32") uses the same scale rule per 1 x 32 block along K,
+// on activations and weights alike, and the same atoms: the word of row r then holds
+// the exponent bytes of the row's four 32-blocks of the K block, block j in byte j, and
+// the j-th K = 32 MMA of the K block reads byte j (the scale-ID fields of the
+// instruction descriptor).
 #pragma once
 
 #include <cstdint>
@@ -84,6 +91,12 @@ __device__ __forceinline__ void scale_copy(uint32_t taddr, uint64_t sdesc) {
 // M >> 4 in bits 24-28, A scale byte id 0 (bits 29-30), K = 32 (bit 31 = 0).
 __host__ __device__ constexpr uint32_t mxf8_idesc(int M, int N) {
     return (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// The same descriptor with scale byte j for both operands (A's scale ID in bits 29-30,
+// B's in bits 4-5): the j-th K = 32 step of a K block under 1 x 32 scales.
+__host__ __device__ constexpr uint32_t mxf8_idesc_byte(uint32_t idesc, int j) {
+    return idesc | (static_cast<uint32_t>(j) << 29) | (static_cast<uint32_t>(j) << 4);
 }
 
 // D[tmem] (+)= (A * 2^sa) (B * 2^sb)^T over K = 32, the scales read from tensor memory.
@@ -204,6 +217,66 @@ __global__ void __launch_bounds__(256) k_quantize_ue8m0_blocks(const uint16_t* _
     if (tid < 128) sf[(static_cast<long long>(kb) * nblocks + nb) * 128 + atom_word(tid)] = static_cast<uint32_t>(e + 127);
 }
 
+// MXFP8 gran-32: every row in 1 x 32 blocks.  As the gran-128 activation quantizer, a
+// half warp takes four consecutive 128-groups of a row per step, 8 inputs per lane and
+// group; the four lanes of a 32-block reduce its amax by two shuffles, and the block's
+// first lane writes its exponent byte into byte (block within the group) of the row's
+// atom word.  Rows R .. Rpad-1 get the word of p = 1 in all four bytes.
+__global__ void __launch_bounds__(256) k_quantize_mxfp8(const uint16_t* __restrict__ x, int R, int K, long long ld_x,
+                                                        uint8_t* __restrict__ q, long long ld_q,
+                                                        uint32_t* __restrict__ sf, int Rpad) {
+    constexpr int kPerHalf = 4;
+    wait_prior_grids();
+    launch_dependents();
+    const int G = K / 128;
+    const long long units = static_cast<long long>(Rpad) * G;
+    const int lane = threadIdx.x & 31;
+    const int half = lane >> 4, l16 = lane & 15;
+    const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+    const long long warp = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int rblocks = Rpad / 128;
+    uint8_t* sf_bytes = reinterpret_cast<uint8_t*>(sf);
+    for (long long base = warp * 2 * kPerHalf; base < units; base += warps * 2 * kPerHalf) {
+        uint4 raw[kPerHalf];
+        int m[kPerHalf], g[kPerHalf];
+        bool valid[kPerHalf], real[kPerHalf];
+#pragma unroll
+        for (int j = 0; j < kPerHalf; ++j) {
+            const long long u = base + half * kPerHalf + j;
+            valid[j] = u < units;
+            m[j] = valid[j] ? static_cast<int>(u / G) : 0;
+            g[j] = valid[j] ? static_cast<int>(u % G) : 0;
+            real[j] = valid[j] && m[j] < R;
+            raw[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (real[j]) raw[j] = ld_nc_v4(x + m[j] * ld_x + g[j] * 128 + l16 * 8);
+        }
+#pragma unroll
+        for (int j = 0; j < kPerHalf; ++j) {
+            float amax = absmax8_packed(raw[j]);
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            const int e = ue8m0_exponent(amax);
+            const long long word = (static_cast<long long>(g[j]) * rblocks + m[j] / 128) * 128 + atom_word(m[j] & 127);
+            if (real[j]) {
+                const float r = pow2_neg(e);
+                float t[8];
+                t[0] = bf16_lo(raw[j].x) * r;
+                t[1] = bf16_hi(raw[j].x) * r;
+                t[2] = bf16_lo(raw[j].y) * r;
+                t[3] = bf16_hi(raw[j].y) * r;
+                t[4] = bf16_lo(raw[j].z) * r;
+                t[5] = bf16_hi(raw[j].z) * r;
+                t[6] = bf16_lo(raw[j].w) * r;
+                t[7] = bf16_hi(raw[j].w) * r;
+                *reinterpret_cast<uint2*>(q + m[j] * ld_q + g[j] * 128 + l16 * 8) = pack8(t);
+                if ((l16 & 3) == 0) sf_bytes[word * 4 + (l16 >> 2)] = static_cast<uint8_t>(e + 127);
+            } else if (valid[j] && l16 == 0) {
+                sf[word] = 0x7F7F7F7Fu;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ GEMM
 
 struct MxArgs {
@@ -256,7 +329,7 @@ struct MxCfg {
     static_assert(kSfCol0 + 16 * STAGES <= kTmemCols, "scale columns");
 };
 
-template <int STAGES, bool GROUPED = false>
+template <int STAGES, bool GROUPED = false, bool GRAN32 = false>
 __global__ void __launch_bounds__(384, 1)
     k_mx_block_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const MxArgs args) {
@@ -412,7 +485,8 @@ __global__ void __launch_bounds__(384, 1)
                         const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
 #pragma unroll
                         for (int k = 0; k < C::kBK / 32; ++k)
-                            mma_mxf8(tmem_base, adesc + 2u * k, bdesc + 2u * k, kIdesc, sfa_t, sfb_t,
+                            mma_mxf8(tmem_base, adesc + 2u * k, bdesc + 2u * k,
+                                     GRAN32 ? mxf8_idesc_byte(kIdesc, k) : kIdesc, sfa_t, sfb_t,
                                      (kb > 0 || k > 0) ? 1u : 0u);
                         mma_commit(empty_bar(stage));
                         if (kb + 1 == args.num_kb) mma_commit(tfull_bar);

@@ -267,3 +267,22 @@ def test_no_cpu_fallback_in_the_product():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in text and "from oracle" not in text, fn
                 assert "lnq_oracle" not in text, fn
+
+
+def test_mxfp8_argument_errors(L):
+    q = L.lnq_quantize_mxfp8
+    assert q(A16, 0, 128, 128, A16b, 128, A16c, None) == INVALID
+    assert q(A16, 4, 256, 128, A16b, 256, A16c, None) == INVALID       # ld_x < K
+    assert q(A16, 4, 96, 96, A16b, 96, A16c, None) == SHAPE            # K % 128
+    assert q(None, 4, 128, 128, A16b, 128, A16c, None) == INVALID
+    assert q(A16, 4, 128, 128, A16b + 4, 128, A16c, None) == MISALIGNED
+    g = L.lnq_mxfp8_gemm_nt
+    assert g(A16, A16b, A16c, A16d, A16e, 0, 256, 128, None) == INVALID
+    assert g(A16, A16b, A16c, A16d, A16e, 4, 250, 128, None) == SHAPE   # N % 16
+    assert g(A16, A16b, A16c, A16d, None, 4, 256, 128, None) == INVALID
+    assert g(A16, A16b, A16c, A16d, A16e + 8, 4, 256, 128, None) == MISALIGNED
+    h = L.lnq_m_grouped_mxfp8_gemm_contiguous
+    assert h(A16, A16b, A16c, A16d, None, 2, A16e, 256, 256, 128, None) == INVALID
+    assert h(A16, A16b, A16c, A16d, A16e + 0x100, 0, A16e, 256, 256, 128, None) == INVALID
+    assert h(A16, A16b, A16c, A16d, A16e + 0x100, 2, A16e, 200, 256, 128, None) == SHAPE   # M_total % 128
+    assert h(A16, A16b, A16c, A16d, A16e + 0x102, 2, A16e, 256, 256, 128, None) == MISALIGNED
