@@ -169,6 +169,19 @@ lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
     args.timeout_ns = kDefaultTimeoutNs;
     args.prefetch_weights = g_weight_prefetch.load(std::memory_order_relaxed);
     args.tma_store = g_tma_store.load(std::memory_order_relaxed);
+    if (!C::SWAP) {
+        // raster bands: grouped tiles 8 row blocks; dense tiles as many row tiles as keep
+        // the band's activation rows within 32 MB of L2 (every weight column tile is
+        // read once per band)
+        int64_t band = 8;
+        if (!C::GROUPED) {
+            band = (int64_t{32} << 20) / (static_cast<int64_t>(C::kTileM) * K);
+            if (band < 1) band = 1;
+        }
+        args.band = static_cast<int>(band < args.tiles_p ? band : (args.tiles_p > 0 ? args.tiles_p : 1));
+    } else {
+        args.band = 1;
+    }
     if constexpr (C::PAIR) {
         // clusters of two CTAs sharing one MMA; as many pairs as can be resident
         constexpr int kCluster = 2;

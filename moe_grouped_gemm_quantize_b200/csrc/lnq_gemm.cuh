@@ -68,6 +68,7 @@ struct GemmArgs {
     int tiles_p;      // tiles along the MMA M slot (of 256 rows for PAIR)
     int tiles_q;      // tiles along the MMA N slot
     int num_tiles;
+    int band;         // dense and grouped raster: row tiles per band (>= 1)
     int prefetch_weights;  // issue the first weight stages before waiting on the prior kernel
     // Split configuration only: the grid's CTAs share the num_tiles * num_kb (tile, K
     // block) units in contiguous runs; a CTA that covers part of a tile leaves an FP32
@@ -146,9 +147,12 @@ struct GemmCfg {
     static constexpr int kScaleSlotFloats = kScaleBatch * kScaleKbFloats;
     static_assert(kScaleKbFloats % 4 == 0, "16-byte aligned scale runs");
     static constexpr int kCW = BNQ / EPI_WG;      // accumulator columns per epilogue thread
-    // TMEM columns per load in the promotion (each load issued one chunk ahead); a decode
-    // thread loads all of its columns of a K block at once
-    static constexpr int kLdCols = SWAP ? kCW : 32;
+    // TMEM columns per load in the promotion: a decode thread loads all of its columns of
+    // a K block at once; dense and grouped threads in chunks of 64 columns, each waited for
+    // before its FMAs (a tcgen05.ld wait covers every load in flight, so a second chunk
+    // loaded ahead would hide nothing; with 64 columns the load latency is paid twice per
+    // K block for 128 columns instead of four times)
+    static constexpr int kLdCols = SWAP ? kCW : (kCW >= 64 ? 64 : 32);
     static_assert(kCW % kLdCols == 0, "promotion chunks tile the thread's columns");
     // TMEM column of the thread's promotion chunk c, from its first column: SiLU.mul
     // threads take kCW/2 gate columns and the kCW/2 up columns 128 further on
@@ -322,11 +326,13 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t, uint32
         c.row_end = a.M;
     } else {
         // Bands of row tiles, column-major inside a band: a wave of tiles shares a
-        // band of activation rows and a few weight column tiles.  Grouped: the
-        // 128-row blocks of one group sit next to each other, so a band's blocks of a
-        // group walk that group's weight columns together (a narrow band keeps the
-        // weights of the groups in flight within L2).
-        constexpr int kBand = (C::PAIR || C::GROUPED) ? 8 : 16;
+        // band of activation rows and a few weight column tiles, and every weight
+        // column tile is read once per band.  The host sizes the band so that its
+        // activation rows stay within a share of L2.  Grouped: the 128-row blocks of
+        // one group sit next to each other, so a band's blocks of a group walk that
+        // group's weight columns together (a narrow band keeps the weights of the
+        // groups in flight within L2).
+        const int kBand = a.band;
         const int band_tiles = kBand * a.tiles_q;
         const int band = t / band_tiles;
         const int first = band * kBand;
@@ -419,23 +425,36 @@ __device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint3
         s2 = make_float2(sb, sb);
         s2_up = s2;
     }
-    uint32_t ra[X], rb[X];
-    tmem_ld_async(taddr + C::chunk_col(0), ra);
-    tmem_wait_ld(ra);
-    if (NC == 1) release();
+    if constexpr (X == 64) {
+        // one 64-column chunk at a time: load, wait, (after the last load) release, FMAs
+        uint32_t r[X];
 #pragma unroll
-    for (int c = 0; c < NC; ++c) {
-        if (c + 1 < NC) {
-            if (c & 1) tmem_ld_async(taddr + C::chunk_col(c + 1), ra);
-            else tmem_ld_async(taddr + C::chunk_col(c + 1), rb);
+        for (int c = 0; c < NC; ++c) {
+            tmem_ld_async(taddr + C::chunk_col(c), r);
+            tmem_wait_ld(r);
+            if (c + 1 == NC) release();
+            const float2 sc = (C::SILU && c >= NC / 2) ? s2_up : s2;
+            promote_chunk<C, X>(acc, r, c * X, slot, sc);
         }
-        const float2 sc = (C::SILU && c >= NC / 2) ? s2_up : s2;
-        if (c & 1) promote_chunk<C, X>(acc, rb, c * X, slot, sc);
-        else promote_chunk<C, X>(acc, ra, c * X, slot, sc);
-        if (c + 1 < NC) {
-            if (c & 1) tmem_wait_ld(ra);
-            else tmem_wait_ld(rb);
-            if (c + 2 == NC) release();
+    } else {
+        uint32_t ra[X], rb[X];
+        tmem_ld_async(taddr + C::chunk_col(0), ra);
+        tmem_wait_ld(ra);
+        if (NC == 1) release();
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            if (c + 1 < NC) {
+                if (c & 1) tmem_ld_async(taddr + C::chunk_col(c + 1), ra);
+                else tmem_ld_async(taddr + C::chunk_col(c + 1), rb);
+            }
+            const float2 sc = (C::SILU && c >= NC / 2) ? s2_up : s2;
+            if (c & 1) promote_chunk<C, X>(acc, rb, c * X, slot, sc);
+            else promote_chunk<C, X>(acc, ra, c * X, slot, sc);
+            if (c + 1 < NC) {
+                if (c & 1) tmem_wait_ld(ra);
+                else tmem_wait_ld(rb);
+                if (c + 2 == NC) release();
+            }
         }
     }
 }
