@@ -549,6 +549,7 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
     R = max(K, args.kernel_reps)
     g_step = capture(launch_step)
     g_chain = capture(lambda: [run(g, "gemm") for _ in range(R) for _, g in calls])
+    g_qchain = capture(lambda: [run(q, "quantize") for _ in range(R) for q, _ in calls])
     g_quant = [capture(lambda q=q: run(q, "quantize")) for q, _ in calls]
     g_gemm = [capture(lambda g=g: run(g, "gemm")) for _, g in calls]
     torch.cuda.synchronize()
@@ -560,6 +561,7 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
 
     replay(g_step, 3)
     replay(g_chain)
+    replay(g_qchain)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -604,9 +606,16 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
         c1.record(stream)
         torch.cuda.synchronize()
         chained_ms = c0.elapsed_time(c1)
+        # ---- the activation quantizes alone, R rounds back to back
+        torch.cuda.synchronize()
+        c0.record(stream)
+        replay(g_qchain)
+        c1.record(stream)
+        torch.cuda.synchronize()
+        qchained_ms = c0.elapsed_time(c1)
         if lnq.lnq_get_last_device_error() != 0:
             raise RuntimeError(f"{name}: device reported an error in the kernel loops")
-    del g_step, g_chain, g_quant, g_gemm
+    del g_step, g_chain, g_qchain, g_quant, g_gemm
     ms = max_over_ranks(ms_local, dist, dev)
     chained_ms = max_over_ranks(chained_ms, dist, dev)
 
@@ -680,7 +689,8 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
                                "note": "each GEMM alone (a one-launch graph between its own two events)"}
     q_total = sum(statistics.median(t) for t in per_quant)
     g_total = sum(statistics.median(t) for t in per_gemm)
-    quant_gbs = sum(u.quant_bytes for u in units) / (q_total * 1e-3) / 1e9
+    quant_gbs_isolated = sum(u.quant_bytes for u in units) / (q_total * 1e-3) / 1e9
+    quant_gbs = sum(u.quant_bytes for u in units) * R / (qchained_ms * 1e-3) / 1e9
     out = {
         "value": round(value, 3),
         "unit": unit,
@@ -691,8 +701,14 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
             "gemm_ms_per_launch": [describe_times(t) for t in per_gemm],
             "quantize_ms_per_launch": [describe_times(t) for t in per_quant],
             "gemm_chained_ms_per_launch": round(gemm_period_ms, 5),
+            "quantize_chained_ms_per_launch": round(qchained_ms / (R * n_units), 5),
             "quantize_gbs": round(quant_gbs, 1),
             "quantize_frac_of_hbm": round(quant_gbs / peaks["hbm_gbs"], 4),
+            "quantize_gbs_isolated": round(quant_gbs_isolated, 1),
+            "quantize_note": ("quantize_gbs: algorithmic bytes (bf16 in, E4M3 and scales out) over the mean "
+                              "period of the quantizes launched back to back in one graph; _isolated: each "
+                              "launch alone between two events, which adds several microseconds of launch "
+                              "latency to these microsecond kernels"),
             "gemm_share_of_step": round(g_total / (g_total + q_total), 4),
         },
         "gpu_launches": K * 2 * n_units,
