@@ -350,7 +350,8 @@ lnq_status lnq_m_grouped_fp8_gemm_masked(const void* a_e4m3, const float* sfa, c
  *   (tcgen05.mma kind::mxf8f6f4.block_scale) and the sum accumulated in FP32
  *   over the whole K range.  a_e4m3 [M][K], b_e4m3 [N][K] (K-major), d_bf16
  *   [M][N] fully overwritten.  Requires N % 16 == 0, K % 128 == 0, pointers
- *   16-byte aligned.
+ *   16-byte aligned.  M > 128 runs 256 x 256 tiles on CTA pairs (unless
+ *   lnq_set_dense_cta_pairs(0)).
  */
 lnq_status lnq_quantize_ue8m0_groups(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, void* q_e4m3,
                                      int64_t ld_q, void* sfa_atoms, void* stream);
@@ -450,6 +451,9 @@ lnq_status lnq_selftest_wait_timeout(int64_t timeout_ns, void* stream);
  *   2  pairs of CTAs on 256 x 128 tiles with four accumulators per CTA
  *      (N >= 128).
  * Other values select 0.  Results are the same up to FP32 summation order.
+ * The same knob serves the dense UE8M0 and MXFP8 GEMMs (lnq_mx_block_gemm_nt,
+ * lnq_mxfp8_gemm_nt) with M > 128: 0 one CTA per 128 x 256 tile, any other mode pairs
+ * of CTAs on 256 x 256 tiles (tcgen05.mma.cta_group::2 with block scaling).
  * Returns the previous setting.
  */
 int32_t lnq_set_dense_cta_pairs(int32_t enable);

@@ -509,7 +509,8 @@ def lnq_get_last_device_error(stream=None) -> int:
 
 def lnq_set_dense_cta_pairs(mode: int) -> int:
     """Dense GEMM configuration for M > 128: 0 one CTA per 128x256 tile, 1 CTA pairs on
-    256x256 tiles, 2 CTA pairs on 256x128 tiles.  Returns the previous setting."""
+    256x256 tiles, 2 CTA pairs on 256x128 tiles (the block-scaled UE8M0 / MXFP8 GEMMs:
+    0 single CTAs, otherwise CTA pairs on 256x256 tiles).  Returns the previous setting."""
     return int(lib().lnq_set_dense_cta_pairs(int(mode)))
 
 

@@ -137,6 +137,19 @@ lnq_status encode_out_map(CUtensorMap* map, const void* base, int64_t rows, int6
     return r == CUDA_SUCCESS ? LNQ_OK : LNQ_ERR_CUDA;
 }
 
+// UE8M0 scale atoms viewed as rows of 128 32-bit words (one 512-byte atom per row), box
+// of `box_rows` atoms, no swizzle: the CTA-pair block-scaled GEMM loads them by TMA.
+lnq_status encode_atom_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
+    cuuint64_t dims[2] = {128u, static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {512u};
+    cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
 template <class C>
 lnq_status launch_gemm(const DeviceInfo& dev, const void* act, int64_t act_rows,
                        const void* wgt, int64_t wgt_rows, int64_t K, GemmArgs args,
@@ -500,6 +513,7 @@ lnq_status mx_gemm(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3
                    const int32_t* m_indices, int32_t num_groups, void* d_bf16, int64_t M, int64_t N, int64_t K,
                    void* stream) {
     using C = MxCfg<4>;
+    using CP = MxCfg<6, true>;
     const bool grouped = m_indices != nullptr;
     if (M <= 0 || N <= 0 || K <= 0 || (grouped && num_groups <= 0)) return LNQ_ERR_INVALID_ARG;
     if (K % 128 != 0 || N % 16 != 0 || M > kMaxRows || N > kMaxRows || K > (int64_t{1} << 31))
@@ -513,15 +527,10 @@ lnq_status mx_gemm(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3
     DeviceInfo* dev = nullptr;
     lnq_status st = device_info(&dev);
     if (st != LNQ_OK) return st;
+    // dense products of more than 128 rows run 256 x 256 tiles on CTA pairs unless the
+    // dense configuration knob selects single CTAs
+    const bool pair = !grouped && M > 128 && g_dense_pairs.load(std::memory_order_relaxed) != 0;
     const int64_t wrows = grouped ? static_cast<int64_t>(num_groups) * N : N;
-    CUtensorMap map_a, map_b;
-    st = encode_e4m3_map(&map_a, a_e4m3, M, K, 128);
-    if (st == LNQ_OK) st = encode_e4m3_map(&map_b, b_e4m3, wrows, K, 256);
-    if (st != LNQ_OK) return st;
-    static std::atomic<bool> attr_dense[kMaxDevices], attr_grouped[kMaxDevices];
-    st = grouped ? smem_attr_once(attr_grouped, dev->ordinal, k_mx_block_gemm<4, true, GRAN32>, C::kSmemBytes)
-                 : smem_attr_once(attr_dense, dev->ordinal, k_mx_block_gemm<4, false, GRAN32>, C::kSmemBytes);
-    if (st != LNQ_OK) return st;
     MxArgs args{};
     args.sfa = static_cast<const uint32_t*>(sfa_atoms);
     args.sfb = static_cast<const uint32_t*>(sfb_atoms);
@@ -533,24 +542,63 @@ lnq_status mx_gemm(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3
     args.num_kb = static_cast<int>(K / 128);
     args.mblocks = static_cast<int>((M + 127) / 128);
     args.nblocks = static_cast<int>((wrows + 127) / 128);
-    args.tiles_p = args.mblocks;
+    args.tiles_p = pair ? static_cast<int>((M + 255) / 256) : args.mblocks;
     args.tiles_q = static_cast<int>((N + 255) / 256);
     args.num_tiles = args.tiles_p * args.tiles_q;
     args.m_indices = m_indices;
     args.num_groups = grouped ? num_groups : 1;
-    const int grid = args.num_tiles < dev->sm_count ? args.num_tiles : dev->sm_count;
+    CUtensorMap map_a, map_b, map_sfa, map_sfb;
+    std::memset(&map_sfa, 0, sizeof map_sfa);
+    std::memset(&map_sfb, 0, sizeof map_sfb);
+    st = encode_e4m3_map(&map_a, a_e4m3, M, K, 128);
+    if (st == LNQ_OK) st = encode_e4m3_map(&map_b, b_e4m3, wrows, K, pair ? 128 : 256);
+    if (st == LNQ_OK && pair) {
+        st = encode_atom_map(&map_sfa, sfa_atoms, (K / 128) * args.mblocks, 1);
+        if (st == LNQ_OK) st = encode_atom_map(&map_sfb, sfb_atoms, (K / 128) * args.nblocks, 2);
+    }
+    if (st != LNQ_OK) return st;
+    static std::atomic<bool> attr_dense[kMaxDevices], attr_grouped[kMaxDevices], attr_pair[kMaxDevices];
+    st = pair      ? smem_attr_once(attr_pair, dev->ordinal, k_mx_block_gemm<6, false, GRAN32, true>, CP::kSmemBytes)
+         : grouped ? smem_attr_once(attr_grouped, dev->ordinal, k_mx_block_gemm<4, true, GRAN32>, C::kSmemBytes)
+                   : smem_attr_once(attr_dense, dev->ordinal, k_mx_block_gemm<4, false, GRAN32>, C::kSmemBytes);
+    if (st != LNQ_OK) return st;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(C::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = grouped ? cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4, true, GRAN32>, map_a, map_b, args)
-                                  : cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4, false, GRAN32>, map_a, map_b, args);
+    cudaError_t e;
+    if (pair) {
+        // clusters of two CTAs sharing one MMA; as many pairs as can be resident
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = 2;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+        cfg.dynamicSmemBytes = CP::kSmemBytes;
+        static std::atomic<int> max_clusters[kMaxDevices];
+        int resident = max_clusters[dev->ordinal].load(std::memory_order_relaxed);
+        if (resident == 0) {
+            cfg.gridDim = dim3(2 * (dev->sm_count / 2), 1, 1);
+            if (cudaOccupancyMaxActiveClusters(&resident, k_mx_block_gemm<6, false, GRAN32, true>, &cfg) !=
+                    cudaSuccess ||
+                resident <= 0)
+                return LNQ_ERR_CUDA;
+            max_clusters[dev->ordinal].store(resident, std::memory_order_relaxed);
+        }
+        const int clusters = args.num_tiles < resident ? args.num_tiles : resident;
+        cfg.gridDim = dim3(2 * clusters, 1, 1);
+        e = cudaLaunchKernelEx(&cfg, k_mx_block_gemm<6, false, GRAN32, true>, map_a, map_b, map_sfa, map_sfb, args);
+    } else {
+        const int grid = args.num_tiles < dev->sm_count ? args.num_tiles : dev->sm_count;
+        cfg.gridDim = dim3(grid, 1, 1);
+        cfg.numAttrs = 1;
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        e = grouped ? cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4, true, GRAN32>, map_a, map_b, map_sfa, map_sfb, args)
+                    : cudaLaunchKernelEx(&cfg, k_mx_block_gemm<4, false, GRAN32>, map_a, map_b, map_sfa, map_sfb, args);
+    }
     if (e != cudaSuccess) return LNQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
 }

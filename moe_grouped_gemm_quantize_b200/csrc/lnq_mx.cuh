@@ -85,6 +85,12 @@ __device__ __forceinline__ void scale_copy(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// CTA pairs: the pair's leader copies a scale atom from each CTA's shared memory (the
+// same offset in both) into the same tensor-memory columns of each CTA.
+__device__ __forceinline__ void scale_copy_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Instruction descriptor of tcgen05.mma kind::mxf8f6f4.block_scale for E4M3 x E4M3,
 // both K-major, UE8M0 scales: B scale byte id 0 (bits 4-5), A and B formats 0 (E4M3,
 // bits 7-9 and 10-12), N >> 3 in bits 17-22, scale format 1 (E8M0) in bit 23,
@@ -106,6 +112,18 @@ __device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// The same over a CTA pair (M = 256): each CTA holds its 128 rows of A, its half of B
+// and, in its own tensor memory, the scales of its A rows and of all N columns of B.
+__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
 }
@@ -295,7 +313,8 @@ struct MxArgs {
     int num_groups;
 };
 
-// One persistent CTA per SM, tiles of 128 rows x 256 columns, 384 threads:
+// One persistent CTA per SM, tiles of 128 rows x 256 columns (256 x 256 on CTA pairs), 384
+// threads:
 //   warp 0      TMA producer: per K block the A and B boxes and the three scale atoms
 //               (A's, and B's two 128-row halves) of the tile on one barrier;
 //   warp 1      tensor memory (512 columns) and the MMA issuer: per K block three
@@ -309,11 +328,17 @@ struct MxArgs {
 // 256 + 16 s .. + 3 and its B scales in 256 + 16 s + 4 .. + 11.  The scales are
 // applied by the tensor core, so no promotion FMAs run and the accumulator is read
 // once per tile; its single buffer costs the MMA one readout per tile.
-template <int STAGES>
+// PAIR (dense): a cluster of two CTAs runs one tcgen05.mma.cta_group::2 of 256 x 256; each
+// CTA loads its 128 rows of A, 128 of the 256 rows of B, its A rows' scale atom and both of
+// B's atoms, all by TMA onto the first CTA's barrier, whose MMA warp copies the atoms
+// into both CTAs' tensor memory and issues the pair's MMAs.  Each SM then loads 32 KB of
+// operands per K block instead of 48 KB.
+template <int STAGES, bool PAIR = false>
 struct MxCfg {
     static constexpr int kBK = 128;
     static constexpr int kABytes = 128 * kBK;
-    static constexpr int kBBytes = 256 * kBK;
+    static constexpr int kBRows = PAIR ? 128 : 256;
+    static constexpr int kBBytes = kBRows * kBK;
     static constexpr int kSfBytes = 3 * 512;
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kOffA + STAGES * kABytes;
@@ -329,11 +354,15 @@ struct MxCfg {
     static_assert(kSfCol0 + 16 * STAGES <= kTmemCols, "scale columns");
 };
 
-template <int STAGES, bool GROUPED = false, bool GRAN32 = false>
+// map_sfa and map_sfb (CTA pairs only) view the scale atoms as rows of 128 words: rows
+// kb * mblocks + mb of A's, kb * nblocks + nb of B's.
+template <int STAGES, bool GROUPED = false, bool GRAN32 = false, bool PAIR = false>
 __global__ void __launch_bounds__(384, 1)
     k_mx_block_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                    const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                     const MxArgs args) {
-    using C = MxCfg<STAGES>;
+    static_assert(!(PAIR && GROUPED), "CTA pairs serve the dense product");
+    using C = MxCfg<STAGES, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -351,6 +380,10 @@ __global__ void __launch_bounds__(384, 1)
     volatile uint32_t* abort_flag = misc + 1;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // CTA pairs: rank in the pair; tiles are numbered per pair
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -358,17 +391,23 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(tfull_bar, 1);
-        mbar_init(tempty_bar, 8);
+        mbar_init(tempty_bar, PAIR ? 16 : 8);
         mbar_init(drain_bar, 1);
         *abort_flag = 0u;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(misc), C::kTmemCols);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_u32(misc), C::kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(misc), C::kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (PAIR) cluster_sync();  // the peer's barriers exist before any remote signal
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
     launch_dependents();
@@ -389,7 +428,7 @@ __global__ void __launch_bounds__(384, 1)
         const int first = band * kBand;
         const int rows = min(args.tiles_p - first, kBand);
         const int r = t - band * band_tiles;
-        p0 = (first + r % rows) * 128;
+        p0 = (first + r % rows) * (PAIR ? 256 : 128) + static_cast<int>(rank) * 128;
         q0 = (r / rows) * 256;
         int g = 0;
         if constexpr (GROUPED) {
@@ -410,12 +449,16 @@ __global__ void __launch_bounds__(384, 1)
             if (elect_one()) {
                 tma_prefetch_desc(&map_a);
                 tma_prefetch_desc(&map_b);
+                if constexpr (PAIR) {
+                    tma_prefetch_desc(&map_sfa);
+                    tma_prefetch_desc(&map_sfb);
+                }
             }
             __syncwarp();
             int stage = 0;
             uint32_t phase = 0, filled = 0, fill_parity = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
+            for (int t = unit; ok && t < args.num_tiles; t += units) {
                 int p0, q0, b_row;
                 if (tile_rc(t, p0, q0, b_row) < 0) continue;
                 const int mb = p0 / 128;
@@ -427,15 +470,29 @@ __global__ void __launch_bounds__(384, 1)
                         break;
                     }
                     if (elect_one()) {
-                        const uint32_t fb = full_bar(stage);
                         const uint32_t sf = sSf + stage * C::kSfBytes;
-                        mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes + C::kSfBytes);
-                        tma_load_2d(sA + stage * C::kABytes, &map_a, fb, kb * C::kBK, p0);
-                        tma_load_2d(sB + stage * C::kBBytes, &map_b, fb, kb * C::kBK, b_row);
-                        const long long kbase = static_cast<long long>(kb);
-                        bulk_load(sf, args.sfa + (kbase * args.mblocks + mb) * 128, 512u, fb);
-                        bulk_load(sf + 512u, args.sfb + (kbase * args.nblocks + nb0) * 128, 512u, fb);
-                        bulk_load(sf + 1024u, args.sfb + (kbase * args.nblocks + nb1) * 128, 512u, fb);
+                        if constexpr (PAIR) {
+                            // both CTAs' bytes complete on the first CTA's full barrier; B's two
+                            // atoms are adjacent rows of its atom view (a second row past the
+                            // last block only scales columns past N, which are never stored)
+                            const uint32_t fb = mapa_shared(full_bar(stage), 0);
+                            if (rank == 0)
+                                mbar_arrive_expect_tx(full_bar(stage), 2 * (C::kABytes + C::kBBytes + C::kSfBytes));
+                            tma_load_2d_pair(sA + stage * C::kABytes, &map_a, fb, kb * C::kBK, p0);
+                            tma_load_2d_pair(sB + stage * C::kBBytes, &map_b, fb, kb * C::kBK,
+                                             b_row + static_cast<int>(rank) * 128);
+                            tma_load_2d_pair(sf, &map_sfa, fb, 0, kb * args.mblocks + mb);
+                            tma_load_2d_pair(sf + 512u, &map_sfb, fb, 0, kb * args.nblocks + nb0);
+                        } else {
+                            const uint32_t fb = full_bar(stage);
+                            mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes + C::kSfBytes);
+                            tma_load_2d(sA + stage * C::kABytes, &map_a, fb, kb * C::kBK, p0);
+                            tma_load_2d(sB + stage * C::kBBytes, &map_b, fb, kb * C::kBK, b_row);
+                            const long long kbase = static_cast<long long>(kb);
+                            bulk_load(sf, args.sfa + (kbase * args.mblocks + mb) * 128, 512u, fb);
+                            bulk_load(sf + 512u, args.sfb + (kbase * args.nblocks + nb0) * 128, 512u, fb);
+                            bulk_load(sf + 1024u, args.sfb + (kbase * args.nblocks + nb1) * 128, 512u, fb);
+                        }
                     }
                     __syncwarp();
                     filled |= 1u << stage;
@@ -447,22 +504,33 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             if (!ok) {
-                // the copies already issued land before the CTA can leave
-                WaitCtx drain = wctx;
-                uint32_t never = 0u;
-                drain.abort = &never;
-                for (int s = 0; s < STAGES; ++s)
-                    if (filled & (1u << s)) (void)mbar_wait_warp(full_bar(s), (fill_parity >> s) & 1u, drain);
+                // the copies already issued land before the CTA can leave (a pair's second
+                // CTA cannot see the first's barriers: it waits out a fixed delay)
+                const uint64_t t0 = global_timer_ns();
+                if (PAIR && rank != 0) {
+                    while (global_timer_ns() - t0 < 200000ull) {
+                    }
+                } else {
+                    WaitCtx drain = wctx;
+                    uint32_t never = 0u;
+                    drain.abort = &never;
+                    for (int s = 0; s < STAGES; ++s)
+                        if (filled & (1u << s)) (void)mbar_wait_warp(full_bar(s), (fill_parity >> s) & 1u, drain);
+                    if (PAIR) {
+                        while (global_timer_ns() - t0 < 200000ull) {
+                        }
+                    }
+                }
             }
-        } else if (warp == 1) {
+        } else if (warp == 1 && rank == 0) {
             // ---------------------------------------------------------------- MMA
-            constexpr uint32_t kIdesc = mxf8_idesc(128, 256);
+            constexpr uint32_t kIdesc = mxf8_idesc(PAIR ? 256 : 128, 256);
             const uint64_t adesc0 = sw128_kmajor_desc(sA);
             const uint64_t bdesc0 = sw128_kmajor_desc(sB);
             int stage = 0;
             uint32_t phase = 0, aphase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
+            for (int t = unit; ok && t < args.num_tiles; t += units) {
                 int p0, q0, b_row;
                 if (tile_rc(t, p0, q0, b_row) < 0) continue;
                 // the epilogue has read the previous tile's accumulator
@@ -478,18 +546,35 @@ __global__ void __launch_bounds__(384, 1)
                     const uint32_t sfb_t = sfa_t + 4u;
                     if (elect_one()) {
                         const uint32_t sf = sSf + stage * C::kSfBytes;
-                        scale_copy(sfa_t, atom_desc(sf));
-                        scale_copy(sfb_t, atom_desc(sf + 512u));
-                        scale_copy(sfb_t + 4u, atom_desc(sf + 1024u));
                         const uint64_t adesc = adesc0 + static_cast<uint64_t>((stage * C::kABytes) >> 4);
                         const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((stage * C::kBBytes) >> 4);
+                        if constexpr (PAIR) {
+                            scale_copy_pair(sfa_t, atom_desc(sf));
+                            scale_copy_pair(sfb_t, atom_desc(sf + 512u));
+                            scale_copy_pair(sfb_t + 4u, atom_desc(sf + 1024u));
 #pragma unroll
-                        for (int k = 0; k < C::kBK / 32; ++k)
-                            mma_mxf8(tmem_base, adesc + 2u * k, bdesc + 2u * k,
-                                     GRAN32 ? mxf8_idesc_byte(kIdesc, k) : kIdesc, sfa_t, sfb_t,
-                                     (kb > 0 || k > 0) ? 1u : 0u);
-                        mma_commit(empty_bar(stage));
-                        if (kb + 1 == args.num_kb) mma_commit(tfull_bar);
+                            for (int k = 0; k < C::kBK / 32; ++k)
+                                mma_mxf8_pair(tmem_base, adesc + 2u * k, bdesc + 2u * k,
+                                              GRAN32 ? mxf8_idesc_byte(kIdesc, k) : kIdesc, sfa_t, sfb_t,
+                                              (kb > 0 || k > 0) ? 1u : 0u);
+                            mma_commit_pair(mapa_shared(empty_bar(stage), 0));
+                            mma_commit_pair(mapa_shared(empty_bar(stage), 1));
+                            if (kb + 1 == args.num_kb) {
+                                mma_commit_pair(mapa_shared(tfull_bar, 0));
+                                mma_commit_pair(mapa_shared(tfull_bar, 1));
+                            }
+                        } else {
+                            scale_copy(sfa_t, atom_desc(sf));
+                            scale_copy(sfb_t, atom_desc(sf + 512u));
+                            scale_copy(sfb_t + 4u, atom_desc(sf + 1024u));
+#pragma unroll
+                            for (int k = 0; k < C::kBK / 32; ++k)
+                                mma_mxf8(tmem_base, adesc + 2u * k, bdesc + 2u * k,
+                                         GRAN32 ? mxf8_idesc_byte(kIdesc, k) : kIdesc, sfa_t, sfb_t,
+                                         (kb > 0 || k > 0) ? 1u : 0u);
+                            mma_commit(empty_bar(stage));
+                            if (kb + 1 == args.num_kb) mma_commit(tfull_bar);
+                        }
                     }
                     __syncwarp();
                     if (++stage == STAGES) {
@@ -500,7 +585,10 @@ __global__ void __launch_bounds__(384, 1)
                 aphase ^= 1u;
             }
             // every MMA and copy completes before tensor memory is released
-            if (elect_one()) mma_commit(drain_bar);
+            if (elect_one()) {
+                if constexpr (PAIR) mma_commit_pair(mapa_shared(drain_bar, 0));
+                else mma_commit(drain_bar);
+            }
             __syncwarp();
             WaitCtx drain = wctx;
             uint32_t never = 0u;
@@ -515,7 +603,7 @@ __global__ void __launch_bounds__(384, 1)
         const int row = quarter * 32 + lane;
         const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
         uint32_t aphase = 0;
-        for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
+        for (int t = unit; t < args.num_tiles; t += units) {
             int p0, q0, b_row;
             if (tile_rc(t, p0, q0, b_row) < 0) continue;
             if (!mbar_wait_warp(tfull_bar, aphase, wctx)) break;
@@ -529,7 +617,10 @@ __global__ void __launch_bounds__(384, 1)
             // the accumulator may take the next tile
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar);
+            if (lane == 0) {
+                if constexpr (PAIR) mbar_arrive_cluster_relaxed(mapa_shared(tempty_bar, 0));
+                else mbar_arrive(tempty_bar);
+            }
             aphase ^= 1u;
             const int m = p0 + row;
             const int n0 = q0 + wg * 128;
@@ -553,10 +644,20 @@ __global__ void __launch_bounds__(384, 1)
         }
     }
 
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+    if constexpr (PAIR) {
+        // no CTA leaves while its peer may still signal its barriers or read its TMEM
+        tc_fence_before();
+        cluster_sync();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc_pair(tmem_base, C::kTmemCols);
+        }
+    } else {
+        __syncthreads();
+        if (warp == 1) {
+            tc_fence_after();
+            tmem_dealloc(tmem_base, C::kTmemCols);
+        }
     }
 }
 

@@ -20,3 +20,13 @@ def store_path(request):
     previous = lnq.lnq_set_tma_store(request.param)
     yield request.param
     lnq.lnq_set_tma_store(previous)
+
+
+@pytest.fixture(params=[0, 1], ids=["one_cta", "cta_pairs"])
+def mx_pairs(request):
+    """Runs a block-scaled (UE8M0 / MXFP8) GEMM test with single CTAs on 128 x 256 tiles
+    and with CTA pairs on 256 x 256 tiles (dense products of more than 128 rows)."""
+    import moe_grouped_gemm_quantize_b200 as lnq
+    previous = lnq.lnq_set_dense_cta_pairs(request.param)
+    yield request.param
+    lnq.lnq_set_dense_cta_pairs(previous)

@@ -87,7 +87,7 @@ def oracle_gemm(a, w):
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (300, 384, 512), (1, 256, 128), (129, 16, 256),
                                    (64, 4096, 1024), (1000, 768, 384)])
-def test_gemm_elementwise(M, N, K):
+def test_gemm_elementwise(M, N, K, mx_pairs):
     a = synthetic.gaussian_bf16((M, K), 1.0, seed=M + N)
     w = synthetic.gaussian_bf16((N, K), 0.02, seed=N + K)
     d = run_gemm(a, w)
@@ -95,7 +95,7 @@ def test_gemm_elementwise(M, N, K):
     assert_gemm_close(to_f64(d), oracle_gemm(a, w), f"ue8m0 {M}x{N}x{K}")
 
 
-def test_gemm_prefill_full():
+def test_gemm_prefill_full(mx_pairs):
     cfg = synthetic.PREFILL[0]
     a, w = full_refs.linear_inputs(cfg.name)
     d = run_gemm(a, w)
@@ -103,12 +103,23 @@ def test_gemm_prefill_full():
     assert_gemm_close(to_f64(d), oracle_gemm(a, w), "ue8m0 prefill QKV")
 
 
-def test_repeated_runs_are_identical():
+def test_repeated_runs_are_identical(mx_pairs):
     a = synthetic.gaussian_bf16((256, 512), 1.0, seed=5)
     w = synthetic.gaussian_bf16((512, 512), 0.02, seed=6)
     d1, d2 = run_gemm(a, w), run_gemm(a, w)
     torch.cuda.synchronize()
     assert torch.equal(d1.view(torch.int16), d2.view(torch.int16))
+
+
+def test_many_tiles_per_cta_elementwise(mx_pairs):
+    # 4096 x 8192 at K = 256: 1024 tiles of 128 x 256 (512 pair tiles of 256 x 256), several
+    # per persistent CTA, so the accumulator hand-over between tiles is checked element by
+    # element
+    a = synthetic.gaussian_bf16((4096, 256), 1.0, seed=411)
+    w = synthetic.gaussian_bf16((8192, 256), 0.02, seed=412)
+    d = run_gemm(a, w)
+    assert lnq.lnq_get_last_device_error() == 0
+    assert_gemm_close(to_f64(d), oracle_gemm(a, w), "ue8m0 many tiles")
 
 
 def run_grouped(a, w, m_indices, G):

@@ -79,7 +79,7 @@ def oracle_gemm(a, w):
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (300, 384, 512), (1, 256, 128), (129, 16, 256),
                                    (64, 4096, 1024), (1000, 768, 384)])
-def test_gemm_elementwise(M, N, K):
+def test_gemm_elementwise(M, N, K, mx_pairs):
     a = synthetic.gaussian_bf16_with_outliers((M, K), 1.0, M + N, 3, frac=0.1)
     w = synthetic.gaussian_bf16((N, K), 0.02, seed=N + K)
     d = run_gemm(a, w)
@@ -87,11 +87,12 @@ def test_gemm_elementwise(M, N, K):
     assert_gemm_close(to_f64(d), oracle_gemm(a, w), f"mxfp8 {M}x{N}x{K}")
 
 
-def test_every_32_block_takes_its_own_scale():
+@pytest.mark.parametrize("M", [128, 384])
+def test_every_32_block_takes_its_own_scale(M, mx_pairs):
     # codes 1.0 throughout, 32-block b of A row m at 2^(m % 4 + b % 5) and of B row n at
     # 2^-(n % 3): every output is an exact small sum that a scale taken per 128 columns, or
-    # from a neighbouring block, would change
-    M, N, K = 128, 256, 512
+    # from a neighbouring block (or from the other CTA of a pair), would change
+    N, K = 256, 512
     B = K // 32
     a = torch.ones((M, K), dtype=torch.float32)
     w = torch.ones((N, K), dtype=torch.float32)
@@ -106,7 +107,7 @@ def test_every_32_block_takes_its_own_scale():
     assert np.array_equal(oracle_gemm(a, w), want)
 
 
-def test_gemm_prefill_full():
+def test_gemm_prefill_full(mx_pairs):
     cfg = synthetic.PREFILL[0]
     a, w = full_refs.linear_inputs(cfg.name)
     d = run_gemm(a, w)
