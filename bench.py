@@ -256,11 +256,16 @@ class Linear:
 
     def copy_out(self):
         """The step's result to pinned host memory (asynchronous)."""
+        for dev_t, host_t in self.out_pairs():
+            host_t.copy_(dev_t, non_blocking=True)
+
+    def out_pairs(self):
+        """(device tensor, pinned host tensor) of each output the step reads back."""
         if self.fp8_out:
-            self.host_qo.copy_(self.qo.view(torch.uint8), non_blocking=True)
-            self.host_so.copy_(self.so, non_blocking=True)
-        else:
-            self.host_d.copy_(self.d, non_blocking=True)
+            return [(self.qo.view(torch.uint8), self.host_qo), (self.so, self.host_so)]
+        return [(self.d, self.host_d)]
+
+    OUTPUTS = ("d", "qo", "so")
 
     def calls(self, stream_ptr):
         """Pre-marshalled C-ABI calls (quantize, gemm)."""
@@ -344,6 +349,11 @@ class Grouped:
     def copy_out(self):
         self.host_d.copy_(self.d, non_blocking=True)
 
+    def out_pairs(self):
+        return [(self.d, self.host_d)]
+
+    OUTPUTS = ("d",)
+
     def calls(self, stream_ptr):
         import ctypes
         import moe_grouped_gemm_quantize_b200 as lnq
@@ -403,6 +413,11 @@ class Masked:
 
     def copy_out(self):
         self.host_d.copy_(self.d, non_blocking=True)
+
+    def out_pairs(self):
+        return [(self.d, self.host_d)]
+
+    OUTPUTS = ("d",)
 
     def calls(self, stream_ptr):
         import ctypes
@@ -491,6 +506,27 @@ def describe_times(ms):
             "mean": round(statistics.mean(ms), 5), "reps": len(ms)}
 
 
+class IoSlot:
+    """One set of a unit's input and output device buffers for the end-to-end loop, with
+    the unit's calls marshalled against them (the quantized activations and the weights
+    are shared: the compute stream runs the steps in order)."""
+
+    def __init__(self, u, stream_ptr, fresh: bool):
+        names = ["x"] + [n for n in u.OUTPUTS if getattr(u, n, None) is not None]
+        saved = {n: getattr(u, n) for n in names}
+        self.bufs = {n: (torch.empty_like(t) if fresh else t) for n, t in saved.items()}
+        for n, t in self.bufs.items():
+            setattr(u, n, t)
+        try:
+            self.calls = u.calls(stream_ptr)
+            self.outs = u.out_pairs()
+        finally:
+            for n, t in saved.items():
+                setattr(u, n, t)
+        self.x = self.bufs["x"]
+        self.host_x = u.host_x
+
+
 def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seconds: float):
     """Everything the bench reports for one workload, as a dict (the same keys as the
     top-level JSON line, without `metric`).
@@ -507,8 +543,10 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
       device timeline, which would otherwise starve the GPU on the microsecond decode
       kernels.
     * e2e: the step through the public calls, issued from the host every step (no graph),
-      with the bf16 activations copied in from pinned host memory and the outputs
-      copied back.
+      with every step's bf16 activations copied in from pinned host memory and its outputs
+      copied back.  The copies in, the kernels and the copies out run on three streams
+      over two sets of input and output buffers, so that step i+1's inputs and step i-1's
+      outputs cross PCIe while step i computes (events order every buffer's reuse).
     """
     import moe_grouped_gemm_quantize_b200 as lnq
 
@@ -623,27 +661,65 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
     e2e = None
     if not args.no_e2e:
         Ke = max(1, min(K, args.e2e_steps))
-        with torch.cuda.stream(stream):
-            for u in units:                   # warm the copy paths
-                u.x.copy_(u.host_x, non_blocking=True)
-                u.copy_out()
+        # a step whose PCIe transfers are small (decode) gains nothing from overlapping them and
+        # would pay the cross-stream waits: it runs copies and kernels in order on one stream
+        pipelined = sum(u.h2d_bytes + u.d2h_bytes for u in units) >= (32 << 20)
+        s_in = torch.cuda.Stream(dev) if pipelined else stream
+        s_out = torch.cuda.Stream(dev) if pipelined else stream
+        slots = [[IoSlot(u, stream.cuda_stream, fresh=(k == 1)) for u in units]
+                 for k in range(2 if pipelined else 1)]
+        ev = lambda: torch.cuda.Event()
+        in_done = [[ev() for _ in units] for _ in range(2)]      # slot's inputs landed
+        comp_done = [[ev() for _ in units] for _ in range(2)]    # slot's kernels done
+        out_done = [[ev() for _ in units] for _ in range(2)]     # slot's outputs read back
+
+        def e2e_step(i):
+            k = i % 2 if pipelined else 0
+            for j, (u, sl) in enumerate(zip(units, slots[k])):
+                q, g = sl.calls
+                with torch.cuda.stream(s_in):
+                    if i >= 2 and pipelined:
+                        s_in.wait_event(comp_done[k][j])      # step i-2 has read this input buffer
+                    sl.x.copy_(sl.host_x, non_blocking=True)
+                    in_done[k][j].record(s_in)
+                with torch.cuda.stream(stream):
+                    if pipelined:
+                        stream.wait_event(in_done[k][j])
+                        if i >= 2:
+                            stream.wait_event(out_done[k][j])  # step i-2's outputs are read back
+                    run(q, "e2e quantize")
+                    run(g, "e2e gemm")
+                    comp_done[k][j].record(stream)
+                with torch.cuda.stream(s_out):
+                    if pipelined:
+                        s_out.wait_event(comp_done[k][j])
+                    for dev_t, host_t in sl.outs:
+                        host_t.copy_(dev_t, non_blocking=True)
+                    out_done[k][j].record(s_out)
+
+        for i in range(2):                    # warm the copy paths and both buffer sets
+            e2e_step(i)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         barrier(dist)
         torch.cuda.synchronize()
-        e0.record(stream)
-        with torch.cuda.stream(stream):
-            for _ in range(Ke):
-                for u, (q, g) in zip(units, calls):
-                    u.x.copy_(u.host_x, non_blocking=True)
-                    run(q, "e2e quantize")
-                    run(g, "e2e gemm")
-                    u.copy_out()
-        e1.record(stream)
+        e0.record(s_in)
+        if pipelined:
+            stream.wait_event(e0)
+            s_out.wait_event(e0)
+        for i in range(Ke):
+            e2e_step(i)
+        if pipelined:
+            s_out.wait_stream(stream)
+            s_out.wait_stream(s_in)
+        e1.record(s_out)
         torch.cuda.synchronize()
         barrier(dist)
+        if lnq.lnq_get_last_device_error() != 0:
+            raise RuntimeError(f"{name}: device reported an error in the end-to-end loop")
         e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+        del slots
         if hbm:
             ev_val, ev_unit = job_throughput(bytes_step, Ke, world, e_ms, 1e9), "GB/s"
         else:
@@ -651,8 +727,11 @@ def measure_workload(name: str, args, dev, dist, world: int, rank: int, cpu_seco
         e2e = {"value": round(ev_val, 3), "unit": ev_unit, "steps": Ke,
                "h2d_bytes_per_step": int(sum(u.h2d_bytes for u in units)),
                "d2h_bytes_per_step": int(sum(u.d2h_bytes for u in units)),
-               "note": "pinned host bf16 activations copied in and the outputs copied back "
-                       "every step; weights resident (model parameters)"}
+               "schedule": ("copies in, kernels and copies out on three streams over two buffer sets"
+                            if pipelined else "copies and kernels in order on one stream"),
+               "note": "every step: pinned host bf16 activations copied in and the outputs copied back "
+                       "(weights resident, model parameters); with 32 MB or more of PCIe transfers per "
+                       "step, those of neighbouring steps overlap the kernels"}
 
     # ---- numbers
     peaks, peak_src = load_peaks()
