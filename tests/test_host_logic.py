@@ -71,3 +71,42 @@ def test_psum_layout_matches_the_group_id_layout():
 def test_job_throughput_counts_all_ranks_over_the_slowest():
     # 2 ranks, each 1e12 units per step, 10 steps in 5 ms (max over ranks): 4e15 units/s
     assert abs(bench.job_throughput(1e12, 10, 2, 5.0, 1.0) - 4e15) < 1e3
+
+
+class _FakeUnit:
+    """A unit with the attributes the end-to-end loop's buffer sets swap."""
+
+    OUTPUTS = ("d", "qo")
+
+    def __init__(self):
+        import torch
+        self.x = torch.arange(12, dtype=torch.float32).reshape(3, 4)
+        self.d = torch.zeros((3, 5), dtype=torch.float32)
+        self.qo = None                       # an output this configuration does not produce
+        self.host_x = self.x.clone()
+        self.host_d = torch.zeros_like(self.d)
+
+    def calls(self, stream_ptr):
+        return ("quantize", self.x.data_ptr(), stream_ptr), ("gemm", self.d.data_ptr(), stream_ptr)
+
+    def out_pairs(self):
+        return [(self.d, self.host_d)]
+
+
+def test_io_slot_marshals_calls_against_its_own_buffers():
+    u = _FakeUnit()
+    x0, d0 = u.x, u.d
+    first = bench.IoSlot(u, 7, fresh=False)
+    second = bench.IoSlot(u, 7, fresh=True)
+    # the unit keeps its own buffers
+    assert u.x is x0 and u.d is d0 and u.qo is None
+    # the first set is the unit's; the second has buffers of its own, of the same shapes
+    assert first.x is x0 and first.calls[1][1] == d0.data_ptr()
+    assert second.x is not x0 and second.x.shape == x0.shape and second.x.dtype == x0.dtype
+    assert second.calls[0][1] == second.x.data_ptr() != x0.data_ptr()
+    assert second.calls[1][1] == second.bufs["d"].data_ptr() != d0.data_ptr()
+    # both read back into the same pinned host buffer, from their own device buffer
+    (dev0, host0), = first.outs
+    (dev1, host1), = second.outs
+    assert dev0 is d0 and dev1 is second.bufs["d"] and host0 is host1 is u.host_d
+    assert "qo" not in second.bufs
