@@ -549,25 +549,26 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     const int unit = C::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int units = C::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
-        }
-        for (int b = 0; b < kSlots; ++b) {
-            mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), C::kEpiWarpsPerSlice);
-        }
-        for (int s = 0; s < C::kScaleStages; ++s) {
-            mbar_init(sfull_bar(s), 32);
-            mbar_init(sempty_bar(s), C::kEpiThreads / 32);
-        }
-        mbar_init(drain_bar, 2);
-        if constexpr (C::SPLITK) {
-            mbar_init(fix_bar, C::kEpiThreads / 32);
-            mbar_init(dec_bar, 1);
-        }
-        *abort_flag = 0u;
+    if (warp == 0) {
+        // The barriers lie in one array in this order: stage full and empty, accumulator
+        // full and empty, scale full and empty, drain (and the split's two); the lanes of
+        // warp 0 initialize them together (a decode CTA has about sixty).
+        auto arrivals = [](int i) -> uint32_t {
+            if (i < 2 * C::STAGES) return 1u;
+            i -= 2 * C::STAGES;
+            if (i < kSlots) return 1u;
+            i -= kSlots;
+            if (i < kSlots) return static_cast<uint32_t>(C::kEpiWarpsPerSlice);
+            i -= kSlots;
+            if (i < C::kScaleStages) return 32u;
+            i -= C::kScaleStages;
+            if (i < C::kScaleStages) return static_cast<uint32_t>(C::kEpiThreads / 32);
+            i -= C::kScaleStages;
+            if (i == 0) return 2u;                                             // drain
+            return i == 1 ? static_cast<uint32_t>(C::kEpiThreads / 32) : 1u;  // split: fix, count
+        };
+        for (int i = lane; i < C::kNumBars; i += 32) mbar_init(bars + 8u * static_cast<uint32_t>(i), arrivals(i));
+        if (lane == 0) *abort_flag = 0u;
         fence_barrier_init();
     }
     if (warp == 1) {
