@@ -254,11 +254,6 @@ class Linear:
             self.d2h_bytes = M * N
             self.host_d = torch.empty((M, N // 2), dtype=torch.bfloat16).pin_memory()
 
-    def copy_out(self):
-        """The step's result to pinned host memory (asynchronous)."""
-        for dev_t, host_t in self.out_pairs():
-            host_t.copy_(dev_t, non_blocking=True)
-
     def out_pairs(self):
         """(device tensor, pinned host tensor) of each output the step reads back."""
         if self.fp8_out:
@@ -346,9 +341,6 @@ class Grouped:
         self.host_x = self.x.cpu().pin_memory()
         self.host_d = torch.empty((self.M, N), dtype=torch.bfloat16).pin_memory()
 
-    def copy_out(self):
-        self.host_d.copy_(self.d, non_blocking=True)
-
     def out_pairs(self):
         return [(self.d, self.host_d)]
 
@@ -410,9 +402,6 @@ class Masked:
         self.d2h_bytes = 2 * self.M * N
         self.host_x = self.x.cpu().pin_memory()
         self.host_d = torch.empty((self.M, N), dtype=torch.bfloat16).pin_memory()
-
-    def copy_out(self):
-        self.host_d.copy_(self.d, non_blocking=True)
 
     def out_pairs(self):
         return [(self.d, self.host_d)]
