@@ -374,17 +374,26 @@ class Grouped:
 
 
 class Masked:
-    """The M-grouped masked MoE GEMM: 32 expert buffers of 128 rows, 2048 routed tokens."""
+    """The M-grouped masked MoE GEMM: 32 expert buffers of 128 rows, 2048 routed tokens;
+    in the FP32-scale recipe or (recipe ue8m0 / mxfp8) with power-of-two scales applied
+    by the tensor core."""
 
-    def __init__(self, cfg, dev):
+    def __init__(self, cfg, dev, recipe: str = "fp32"):
         import moe_grouped_gemm_quantize_b200 as lnq
         from moe_grouped_gemm_quantize_b200 import synthetic
         self.cfg = cfg
+        self.recipe = recipe
+        self.ue8m0 = recipe in ("ue8m0", "mxfp8")
         a, w, counts = synthetic.make_moe_masked_inputs(cfg)
         G, Mm, N, K = cfg.groups, cfg.m_max, cfg.N, cfg.K
         self.M = G * Mm
         self.x = a.to(dev)
-        self.wq, self.ws = lnq.quantize_weights_grouped(w.to(dev), G)
+        if recipe == "mxfp8":
+            self.wq, self.ws = lnq.quantize_mxfp8(w.to(dev))
+        elif self.ue8m0:
+            self.wq, self.ws = lnq.quantize_weights_ue8m0(w.to(dev))
+        else:
+            self.wq, self.ws = lnq.quantize_weights_grouped(w.to(dev), G)
         del w
         self.mm = torch.from_numpy(counts).to(dev)
         real = int(counts.sum())
@@ -398,6 +407,10 @@ class Masked:
         self.gemm_bytes = (real * K + 4 * (K // 128) * real + busy * N * K
                            + 4 * busy * (-(-N // 128)) * (K // 128) + 2 * real * N + 4 * G)
         self.quant_bytes = 3 * self.M * K + 4 * (K // 128) * self.M
+        if self.ue8m0:
+            # scale atoms: 4 bytes per row per K block on both operands
+            self.sfa = lnq.ue8m0_atoms(self.M, K, dev)
+            self.gemm_bytes += 4 * (K // 128) * busy * N - 4 * busy * (-(-N // 128)) * (K // 128)
         self.h2d_bytes = 2 * self.M * K
         self.d2h_bytes = 2 * self.M * N
         self.host_x = self.x.cpu().pin_memory()
@@ -415,11 +428,16 @@ class Masked:
         P = ctypes.c_void_p
         c = self.cfg
         s = P(stream_ptr)
-        qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K,
-                 P(self.sfa.data_ptr()), self.M, s)
         gargs = (P(self.q.data_ptr()), P(self.sfa.data_ptr()), P(self.wq.data_ptr()),
                  P(self.ws.data_ptr()), P(self.mm.data_ptr()), c.groups, c.m_max,
                  c.tokens // c.groups, P(self.d.data_ptr()), c.N, c.K, s)
+        if self.ue8m0:
+            qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K, P(self.sfa.data_ptr()), s)
+            if self.recipe == "mxfp8":
+                return (L.lnq_quantize_mxfp8, qargs), (L.lnq_m_grouped_mxfp8_gemm_masked, gargs)
+            return (L.lnq_quantize_ue8m0_groups, qargs), (L.lnq_m_grouped_mx_gemm_masked, gargs)
+        qargs = (P(self.x.data_ptr()), self.M, c.K, c.K, P(self.q.data_ptr()), c.K,
+                 P(self.sfa.data_ptr()), self.M, s)
         return (L.lnq_quantize_fp8_groups, qargs), (L.lnq_m_grouped_fp8_gemm_masked, gargs)
 
 
@@ -484,7 +502,7 @@ def make_units(name: str, args, dev):
     cfgs, kind = workload_units(name)
     return [Grouped(c, dev, recipe=args.recipe) if kind == "grouped"
             else Grouped(c, dev, alignment=256) if kind == "psum"
-            else Masked(c, dev) if kind == "masked"
+            else Masked(c, dev, recipe=args.recipe) if kind == "masked"
             else Linear(c, dev, split=args.split, fp8_out=args.epilogue == "fp8",
                         silu=args.epilogue == "silu", recipe=args.recipe) for c in cfgs]
 

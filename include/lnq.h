@@ -418,6 +418,36 @@ lnq_status lnq_m_grouped_mxfp8_gemm_contiguous(const void* a_e4m3, const void* s
                                                const void* sfb_atoms, const int32_t* m_indices, int32_t num_groups,
                                                void* d_bf16, int64_t M_total, int64_t N, int64_t K, void* stream);
 
+/*
+ * The UE8M0 (gran-128) and MXFP8 (gran-32) recipes in the M-grouped masked layout
+ * (deepgemm-rust README, "What's implemented": the masked_m scheduler of the
+ * DeepEP-style dispatch output, zero CPU sync; "Full recipes": gran-32 and
+ * gran-128 on either side): as lnq_m_grouped_fp8_gemm_masked, with the scales in
+ * atoms.
+ *   a_e4m3      [num_groups*M_max][K] E4M3, group g's buffer in rows g*M_max ..
+ *               g*M_max + M_max - 1; sfa_atoms over all num_groups*M_max rows, from
+ *               lnq_quantize_ue8m0_groups (lnq_m_grouped_mx_gemm_masked) or
+ *               lnq_quantize_mxfp8 (lnq_m_grouped_mxfp8_gemm_masked).
+ *   b_e4m3      [num_groups*N][K] E4M3 and sfb_atoms over all num_groups*N rows, from
+ *               lnq_quantize_ue8m0_blocks or lnq_quantize_mxfp8.
+ *   masked_m    [num_groups] int32 on the device: real rows of each group, 0 .. M_max;
+ *               a count outside that range is clamped and reported by
+ *               lnq_get_last_device_error as LNQ_ERR_INVALID_ARG.
+ *   expected_m  a scheduling hint (>= 0); results do not depend on it.
+ *   d_bf16      [num_groups*M_max][N] bf16: rows g*M_max + m for m < masked_m[g] are
+ *               written, the other rows left untouched.
+ *   Requires M_max % 128 == 0, N % 128 == 0, K % 128 == 0, masked_m 4-byte aligned,
+ *   the other pointers 16-byte aligned.
+ */
+lnq_status lnq_m_grouped_mx_gemm_masked(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                        const void* sfb_atoms, const int32_t* masked_m, int32_t num_groups,
+                                        int64_t M_max, int64_t expected_m, void* d_bf16, int64_t N, int64_t K,
+                                        void* stream);
+lnq_status lnq_m_grouped_mxfp8_gemm_masked(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                           const void* sfb_atoms, const int32_t* masked_m, int32_t num_groups,
+                                           int64_t M_max, int64_t expected_m, void* d_bf16, int64_t N, int64_t K,
+                                           void* stream);
+
 /* Static text for a status code. */
 const char* lnq_status_string(lnq_status status);
 

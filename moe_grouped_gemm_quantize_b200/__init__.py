@@ -30,7 +30,7 @@ __all__ = [
     "lnq_m_grouped_fp8_gemm_contiguous", "lnq_m_grouped_fp8_gemm_contiguous_psum",
     "lnq_fp8_block_gemm_nt_silu_mul", "lnq_mx_block_gemm_nt", "lnq_m_grouped_mx_gemm_contiguous", "quantize_activations_ue8m0",
     "quantize_weights_ue8m0", "ue8m0_atoms", "quantize_mxfp8", "lnq_mxfp8_gemm_nt",
-    "lnq_m_grouped_mxfp8_gemm_contiguous",
+    "lnq_m_grouped_mxfp8_gemm_contiguous", "lnq_m_grouped_mx_gemm_masked", "lnq_m_grouped_mxfp8_gemm_masked",
     "lnq_m_grouped_fp8_gemm_masked", "lnq_get_last_device_error", "lnq_status_string",
     "lnq_selftest_wait_timeout", "lnq_set_dense_cta_pairs", "lnq_set_grouped_cta_pairs",
     "lnq_set_weight_prefetch", "lnq_set_tma_store",
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
             "lnq_quantize_mxfp8": [P, I64, I64, I64, P, I64, P, P],
             "lnq_mxfp8_gemm_nt": [P, P, P, P, P, I64, I64, I64, P],
             "lnq_m_grouped_mxfp8_gemm_contiguous": [P, P, P, P, P, I32, P, I64, I64, I64, P],
+            "lnq_m_grouped_mx_gemm_masked": [P, P, P, P, P, I32, I64, I64, P, I64, I64, P],
+            "lnq_m_grouped_mxfp8_gemm_masked": [P, P, P, P, P, I32, I64, I64, P, I64, I64, P],
             "lnq_get_last_device_error": [P],
             "lnq_selftest_wait_timeout": [I64, P],
         }
@@ -449,6 +451,46 @@ def lnq_m_grouped_mxfp8_gemm_contiguous(a: torch.Tensor, sfa: torch.Tensor, b: t
     _check(lib().lnq_m_grouped_mxfp8_gemm_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(m_indices), G,
                                                      _ptr(d), M_total, N, K, _stream(stream)),
            "lnq_m_grouped_mxfp8_gemm_contiguous")
+
+
+def _mx_masked(fn_name: str, a, sfa, b, sfb, masked_m, d, expected_m, stream) -> None:
+    if not (_is_fp8(a) and _is_fp8(b)) or sfa.dtype != torch.int32 or sfb.dtype != torch.int32 or \
+            d.dtype != torch.bfloat16 or masked_m.dtype != torch.int32:
+        raise TypeError("a, b e4m3; sfa, sfb int32 scale atoms; masked_m int32; d bf16")
+    G = masked_m.numel()
+    if a.dim() == 3:
+        if a.shape[0] != G:
+            raise ValueError("a's first dimension must be the number of groups")
+        M_max, K = a.shape[1], a.shape[2]
+    else:
+        M_max, K = a.shape[0] // G, a.shape[1]
+    N = (b.shape[1] if b.dim() == 3 else b.shape[0] // G)
+    for t in (a, sfa, b, sfb, masked_m, d):
+        if not t.is_contiguous():
+            raise ValueError("all operands must be contiguous")
+    if a.numel() != G * M_max * K or b.numel() != G * N * K or d.numel() != G * M_max * N or \
+            tuple(sfa.shape) != (K // 128, -(-G * M_max // 128) * 128) or \
+            tuple(sfb.shape) != (K // 128, -(-G * N // 128) * 128):
+        raise ValueError("inconsistent shapes")
+    _check(getattr(lib(), fn_name)(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(masked_m), G, M_max,
+                                   int(expected_m), _ptr(d), N, K, _stream(stream)), fn_name)
+
+
+def lnq_m_grouped_mx_gemm_masked(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                                 masked_m: torch.Tensor, d: torch.Tensor, expected_m: int = 0,
+                                 stream=None) -> None:
+    """UE8M0 recipe, M-grouped masked: a e4m3 [G, M_max, K] (or [G*M_max, K]) and its scale atoms
+    over G*M_max rows, b e4m3 [G*N, K] and its atoms, masked_m int32 [G] on the device, d bf16
+    [G*M_max, N]: group g's first masked_m[g] rows of d are written."""
+    _mx_masked("lnq_m_grouped_mx_gemm_masked", a, sfa, b, sfb, masked_m, d, expected_m, stream)
+
+
+def lnq_m_grouped_mxfp8_gemm_masked(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor, sfb: torch.Tensor,
+                                    masked_m: torch.Tensor, d: torch.Tensor, expected_m: int = 0,
+                                    stream=None) -> None:
+    """MXFP8 gran-32, M-grouped masked: as lnq_m_grouped_mx_gemm_masked with the scale atoms of
+    lnq_quantize_mxfp8 on both operands."""
+    _mx_masked("lnq_m_grouped_mxfp8_gemm_masked", a, sfa, b, sfb, masked_m, d, expected_m, stream)
 
 
 def lnq_m_grouped_fp8_gemm_contiguous_psum(a: torch.Tensor, sfa: torch.Tensor, b: torch.Tensor,

@@ -508,21 +508,26 @@ namespace {
 
 // The block-scaled product of the UE8M0 recipes: gran-128 scales (GRAN32 false) or the
 // MXFP8 gran-32 scales, dense or M-grouped contiguous (m_indices != nullptr).
+// The UE8M0 / MXFP8 block-scaled GEMM: dense (m_indices and masked_m null), M-grouped
+// contiguous (m_indices) or M-grouped masked (masked_m, groups of m_max rows, M the total).
 template <bool GRAN32>
 lnq_status mx_gemm(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3, const void* sfb_atoms,
                    const int32_t* m_indices, int32_t num_groups, void* d_bf16, int64_t M, int64_t N, int64_t K,
-                   void* stream) {
+                   void* stream, const int32_t* masked_m = nullptr, int64_t m_max = 0) {
     using C = MxCfg<4>;
     using CP = MxCfg<6, true>;
-    const bool grouped = m_indices != nullptr;
+    const bool grouped = m_indices != nullptr || masked_m != nullptr;
     if (M <= 0 || N <= 0 || K <= 0 || (grouped && num_groups <= 0)) return LNQ_ERR_INVALID_ARG;
     if (K % 128 != 0 || N % 16 != 0 || M > kMaxRows || N > kMaxRows || K > (int64_t{1} << 31))
         return LNQ_ERR_UNSUPPORTED_SHAPE;
     if (grouped && (M % 128 != 0 || N % 128 != 0 || static_cast<int64_t>(num_groups) * N > kMaxRows))
         return LNQ_ERR_UNSUPPORTED_SHAPE;
+    if (masked_m != nullptr && (m_max <= 0 || m_max % 128 != 0 || M != static_cast<int64_t>(num_groups) * m_max))
+        return LNQ_ERR_UNSUPPORTED_SHAPE;
     if (!a_e4m3 || !sfa_atoms || !b_e4m3 || !sfb_atoms || !d_bf16) return LNQ_ERR_INVALID_ARG;
     if (!aligned16(a_e4m3) || !aligned16(sfa_atoms) || !aligned16(b_e4m3) || !aligned16(sfb_atoms) ||
-        !aligned16(d_bf16) || (grouped && !aligned4(m_indices)))
+        !aligned16(d_bf16) || (m_indices != nullptr && !aligned4(m_indices)) ||
+        (masked_m != nullptr && !aligned4(masked_m)))
         return LNQ_ERR_MISALIGNED;
     DeviceInfo* dev = nullptr;
     lnq_status st = device_info(&dev);
@@ -547,6 +552,8 @@ lnq_status mx_gemm(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3
     args.num_tiles = args.tiles_p * args.tiles_q;
     args.m_indices = m_indices;
     args.num_groups = grouped ? num_groups : 1;
+    args.masked_m = masked_m;
+    args.m_max = static_cast<int>(m_max);
     CUtensorMap map_a, map_b, map_sfa, map_sfb;
     std::memset(&map_sfa, 0, sizeof map_sfa);
     std::memset(&map_sfb, 0, sizeof map_sfb);
@@ -618,6 +625,24 @@ lnq_status lnq_m_grouped_mxfp8_gemm_contiguous(const void* a_e4m3, const void* s
     if (!m_indices) return LNQ_ERR_INVALID_ARG;
     return mx_gemm<true>(a_e4m3, sfa_atoms, b_e4m3, sfb_atoms, m_indices, num_groups, d_bf16, M_total, N, K,
                          stream);
+}
+
+lnq_status lnq_m_grouped_mx_gemm_masked(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                        const void* sfb_atoms, const int32_t* masked_m, int32_t num_groups,
+                                        int64_t M_max, int64_t expected_m, void* d_bf16, int64_t N, int64_t K,
+                                        void* stream) {
+    if (!masked_m || expected_m < 0 || num_groups <= 0 || M_max <= 0) return LNQ_ERR_INVALID_ARG;
+    return mx_gemm<false>(a_e4m3, sfa_atoms, b_e4m3, sfb_atoms, nullptr, num_groups, d_bf16,
+                          static_cast<int64_t>(num_groups) * M_max, N, K, stream, masked_m, M_max);
+}
+
+lnq_status lnq_m_grouped_mxfp8_gemm_masked(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,
+                                           const void* sfb_atoms, const int32_t* masked_m, int32_t num_groups,
+                                           int64_t M_max, int64_t expected_m, void* d_bf16, int64_t N, int64_t K,
+                                           void* stream) {
+    if (!masked_m || expected_m < 0 || num_groups <= 0 || M_max <= 0) return LNQ_ERR_INVALID_ARG;
+    return mx_gemm<true>(a_e4m3, sfa_atoms, b_e4m3, sfb_atoms, nullptr, num_groups, d_bf16,
+                         static_cast<int64_t>(num_groups) * M_max, N, K, stream, masked_m, M_max);
 }
 
 lnq_status lnq_mx_block_gemm_nt(const void* a_e4m3, const void* sfa_atoms, const void* b_e4m3,

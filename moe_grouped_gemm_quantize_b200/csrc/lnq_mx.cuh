@@ -311,6 +311,11 @@ struct MxArgs {
     // == 0); a block led by a negative id is skipped.
     const int32_t* m_indices;
     int num_groups;
+    // M-grouped masked layout (GROUPED, m_indices == nullptr): group g owns rows
+    // g*m_max .. g*m_max + m_max - 1 of A and D, of which the first masked_m[g] are real;
+    // blocks past the count are skipped and stores stop at it.
+    const int32_t* masked_m;  // [num_groups], on the device
+    int m_max;                // rows per group, a multiple of 128
 };
 
 // One persistent CTA per SM, tiles of 128 rows x 256 columns (256 x 256 on CTA pairs), 384
@@ -420,8 +425,9 @@ __global__ void __launch_bounds__(384, 1)
 
     // banded raster, column-major inside bands of row tiles (16 dense, 8 grouped: the
     // blocks of a group walk its weight columns together).  Returns the tile's group
-    // (0 dense; -1 for a grouped block to skip) and its first row of B.
-    auto tile_rc = [&](int t, int& p0, int& q0, int& b_row) {
+    // (0 dense; -1 for a grouped block to skip), its first row of B and the end of its
+    // rows that are stored (rows from row_end on stay untouched).
+    auto tile_rc = [&](int t, int& p0, int& q0, int& b_row, int& row_end) {
         constexpr int kBand = GROUPED ? 8 : 16;
         const int band_tiles = kBand * args.tiles_q;
         const int band = t / band_tiles;
@@ -430,12 +436,26 @@ __global__ void __launch_bounds__(384, 1)
         const int r = t - band * band_tiles;
         p0 = (first + r % rows) * (PAIR ? 256 : 128) + static_cast<int>(rank) * 128;
         q0 = (r / rows) * 256;
+        row_end = args.M;
         int g = 0;
         if constexpr (GROUPED) {
-            g = __ldg(args.m_indices + p0);
-            if (g >= args.num_groups) {
-                atomicOr(args.status, kStatusBadGroup);
-                g = -1;
+            if (args.m_indices != nullptr) {
+                g = __ldg(args.m_indices + p0);
+                if (g >= args.num_groups) {
+                    atomicOr(args.status, kStatusBadGroup);
+                    g = -1;
+                }
+            } else {
+                // masked: group g's first masked_m[g] rows are real
+                g = p0 / args.m_max;
+                int count = __ldg(args.masked_m + g);
+                if (count < 0 || count > args.m_max) {
+                    atomicOr(args.status, kStatusBadGroup);
+                    count = count < 0 ? 0 : args.m_max;
+                }
+                const int valid = g * args.m_max + count - p0;
+                row_end = p0 + (valid < 128 ? valid : 128);
+                if (valid <= 0) g = -1;
             }
         }
         b_row = (g < 0 ? 0 : g) * args.N + q0;
@@ -459,8 +479,8 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t phase = 0, filled = 0, fill_parity = 0;
             bool ok = true;
             for (int t = unit; ok && t < args.num_tiles; t += units) {
-                int p0, q0, b_row;
-                if (tile_rc(t, p0, q0, b_row) < 0) continue;
+                int p0, q0, b_row, row_end;
+                if (tile_rc(t, p0, q0, b_row, row_end) < 0) continue;
                 const int mb = p0 / 128;
                 const int nb0 = b_row / 128;
                 const int nb1 = min(nb0 + 1, args.nblocks - 1);
@@ -531,8 +551,8 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t phase = 0, aphase = 0;
             bool ok = true;
             for (int t = unit; ok && t < args.num_tiles; t += units) {
-                int p0, q0, b_row;
-                if (tile_rc(t, p0, q0, b_row) < 0) continue;
+                int p0, q0, b_row, row_end;
+                if (tile_rc(t, p0, q0, b_row, row_end) < 0) continue;
                 // the epilogue has read the previous tile's accumulator
                 if (!mbar_wait_warp(tempty_bar, aphase ^ 1u, wctx)) break;
                 tc_fence_after();
@@ -604,8 +624,8 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
         uint32_t aphase = 0;
         for (int t = unit; t < args.num_tiles; t += units) {
-            int p0, q0, b_row;
-            if (tile_rc(t, p0, q0, b_row) < 0) continue;
+            int p0, q0, b_row, row_end;
+            if (tile_rc(t, p0, q0, b_row, row_end) < 0) continue;
             if (!mbar_wait_warp(tfull_bar, aphase, wctx)) break;
             tc_fence_after();
             uint32_t ra[64], rb[64];
@@ -624,7 +644,7 @@ __global__ void __launch_bounds__(384, 1)
             aphase ^= 1u;
             const int m = p0 + row;
             const int n0 = q0 + wg * 128;
-            if (m < args.M) {
+            if (m < row_end) {
                 uint16_t* drow = args.d + static_cast<long long>(m) * args.N;
                 auto store8 = [&](int n, const uint32_t (&r)[64], int i) {
                     if (n < args.N) {

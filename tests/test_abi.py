@@ -286,3 +286,20 @@ def test_mxfp8_argument_errors(L):
     assert h(A16, A16b, A16c, A16d, A16e + 0x100, 0, A16e, 256, 256, 128, None) == INVALID
     assert h(A16, A16b, A16c, A16d, A16e + 0x100, 2, A16e, 200, 256, 128, None) == SHAPE   # M_total % 128
     assert h(A16, A16b, A16c, A16d, A16e + 0x102, 2, A16e, 256, 256, 128, None) == MISALIGNED
+
+
+@pytest.mark.parametrize("entry", ["lnq_m_grouped_mx_gemm_masked", "lnq_m_grouped_mxfp8_gemm_masked"])
+def test_block_scaled_masked_argument_errors(L, entry):
+    f = getattr(L, entry)
+
+    def call(M_max=256, N=256, K=512, G=4, mm=A16e + 0x1000, a=A16, expected=64):
+        return f(a, A16b, A16c, A16d, mm, G, M_max, expected, A16e, N, K, None)
+
+    assert call(G=0) == INVALID
+    assert call(expected=-1) == INVALID
+    assert call(M_max=200) == SHAPE            # M_max % 128
+    assert call(K=100) == SHAPE
+    assert call(N=144) == SHAPE                # grouped weights: N % 128
+    assert call(mm=None) == INVALID
+    assert call(mm=A16e + 0x1002) == MISALIGNED
+    assert call(a=A16 + 1) == MISALIGNED
