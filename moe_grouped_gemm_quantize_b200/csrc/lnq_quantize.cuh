@@ -153,6 +153,23 @@ constexpr int kQuantConsumerWarps = 8;
 constexpr int kQuantThreads = 32 * (kQuantConsumerWarps + 1);
 constexpr int kQuantSmemBytes = kQuantStages * kQuantTileBytes + 2 * kQuantStages * 8 + 16 + 128;
 
+// Row and column tile of t = blockIdx.x + i * gridDim.x, advanced by the grid size
+// (t = r * cols + c) without a division per tile.
+struct TileWalk {
+    int r, c, dr, dc;
+    __device__ __forceinline__ explicit TileWalk(int cols)
+        : r(static_cast<int>(blockIdx.x) / cols), c(static_cast<int>(blockIdx.x) % cols),
+          dr(static_cast<int>(gridDim.x) / cols), dc(static_cast<int>(gridDim.x) % cols) {}
+    __device__ __forceinline__ void next(int cols) {
+        r += dr;
+        c += dc;
+        if (c >= cols) {
+            c -= cols;
+            ++r;
+        }
+    }
+};
+
 struct QuantArgs {
     uint8_t* q;
     float* sfa;
@@ -165,11 +182,14 @@ struct QuantArgs {
 
 // Persistent 1x128 activation quantize.  A producer warp streams 32 x 256 bf16
 // tiles into a 4-stage shared-memory ring with TMA (rows past M arrive as
-// zeros); eight consumer warps each own four consecutive rows of a tile: lane
-// l holds columns 8l .. 8l+7, so lanes 0-15 form the first 128-group and
-// 16-31 the second.  The amax is a half-warp shuffle reduction; lanes 0 and 16
-// store their four rows' scales as one 16-byte run (M4 is a multiple of 4).
-// Consumer warps never wait for one another.
+// zeros); eight consumer warps each own four consecutive rows of a tile.  The
+// lanes of half h of a warp take the warp's rows 2h and 2h+1, lane j of the half
+// holding columns 16j .. 16j+15 of both, so that eight lanes form a 128-group and
+// every lane codes 32 values with two rows' worth of scale work.  The two rows'
+// amaxes travel as one packed bf16 pair through a three-step shuffle; the first
+// lane of every eight stores the pair of scales (rows 2h, 2h+1; M4 is a multiple
+// of 4).  Consumer warps never wait for one another.  Tile indices advance by the
+// grid size without a division per tile.
 __global__ void __launch_bounds__(kQuantThreads)
     k_quantize_groups(const __grid_constant__ CUtensorMap xmap, const QuantArgs args) {
     extern __shared__ uint8_t qsmem_raw[];
@@ -207,16 +227,15 @@ __global__ void __launch_bounds__(kQuantThreads)
             int stage = 0;
             uint32_t phase = 0, filled = 0, fill_parity = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
+            TileWalk tw(args.col_tiles);
+            for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x, tw.next(args.col_tiles)) {
                 if (!mbar_wait(empty_bar(stage), phase ^ 1u, wctx)) {
                     ok = false;
                     break;
                 }
-                const int row0 = (t / args.col_tiles) * kQuantRows;
-                const int col0 = (t % args.col_tiles) * kQuantCols;
                 mbar_arrive_expect_tx(full_bar(stage), kQuantTileBytes);
-                tma_load_2d(smem_u32(smem + stage * kQuantTileBytes), &xmap, full_bar(stage), col0,
-                            row0);
+                tma_load_2d(smem_u32(smem + stage * kQuantTileBytes), &xmap, full_bar(stage),
+                            tw.c * kQuantCols, tw.r * kQuantRows);
                 filled |= 1u << stage;
                 fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == kQuantStages) {
@@ -236,47 +255,60 @@ __global__ void __launch_bounds__(kQuantThreads)
     }
 
     // -------------------------------------------------------------- consumers
-    // warp w owns rows 4w .. 4w+3 of each tile and writes their scales itself
     constexpr int kRowsPerWarp = kQuantRows / kQuantConsumerWarps;
-    static_assert(kRowsPerWarp == 4, "one float4 of scales per warp and group");
+    static_assert(kRowsPerWarp == 4, "two rows per half-warp");
+    constexpr int kRowBytes = kQuantCols * 2;
     const int half = lane >> 4;
+    const int j = lane & 15;       // columns 16j .. 16j+15 of the tile
+    const int gsel = j >> 3;       // the tile's first or second 128-group
+    const long long k_groups = args.K >> 7;
     int stage = 0;
     uint32_t phase = 0;
-    for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
-        const long long row0 = static_cast<long long>(t / args.col_tiles) * kQuantRows + warp * kRowsPerWarp;
-        const long long col0 = static_cast<long long>(t % args.col_tiles) * kQuantCols;
-        const long long group = (col0 >> 7) + half;
-        const bool group_ok = group < (args.K >> 7);
+    TileWalk tw(args.col_tiles);
+    for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x, tw.next(args.col_tiles)) {
+        // first of this lane's two rows, and its first column
+        const long long row0 = static_cast<long long>(tw.r) * kQuantRows + warp * kRowsPerWarp + 2 * half;
+        const long long col = static_cast<long long>(tw.c) * kQuantCols + 16 * j;
+        const long long group = (col >> 7);
+        const bool group_ok = group < k_groups;
         if (!mbar_wait(full_bar(stage), phase, wctx)) break;
-        const uint8_t* tile = smem + stage * kQuantTileBytes + warp * kRowsPerWarp * (kQuantCols * 2);
-        uint4 raw[kRowsPerWarp];
+        const uint8_t* src = smem + stage * kQuantTileBytes + (warp * kRowsPerWarp + 2 * half) * kRowBytes + 32 * j;
+        uint4 raw[2][2];
 #pragma unroll
-        for (int i = 0; i < kRowsPerWarp; ++i)
-            raw[i] = *reinterpret_cast<const uint4*>(tile + i * (kQuantCols * 2) + lane * 16);
+        for (int p = 0; p < 2; ++p) {
+            raw[p][0] = *reinterpret_cast<const uint4*>(src + p * kRowBytes);
+            raw[p][1] = *reinterpret_cast<const uint4*>(src + p * kRowBytes + 16);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar(stage));
-        float sv[kRowsPerWarp];
+        // each row's largest magnitude over this lane's 16 values (both bf16 halves of
+        // m[p] are candidates), then row 0 in the low and row 1 in the high half of one
+        // word, reduced over the group's eight lanes; exact throughout
+        uint32_t m[2];
 #pragma unroll
-        for (int i = 0; i < kRowsPerWarp; ++i) {
-            float amax = absmax8_packed(raw[i]);
+        for (int p = 0; p < 2; ++p)
+            m[p] = maxabs_bf16x2(maxabs_bf16x2(maxabs_bf16x2(raw[p][0].x, raw[p][0].y),
+                                               maxabs_bf16x2(raw[p][0].z, raw[p][0].w)),
+                                 maxabs_bf16x2(maxabs_bf16x2(raw[p][1].x, raw[p][1].y),
+                                               maxabs_bf16x2(raw[p][1].z, raw[p][1].w)));
+        uint32_t z = maxabs_bf16x2(__byte_perm(m[0], m[1], 0x5410), __byte_perm(m[0], m[1], 0x7632));
 #pragma unroll
-            for (int off = 8; off >= 1; off >>= 1)
-                amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
-            sv[i] = scale_of_amax(amax);
-        }
+        for (int off = 1; off <= 4; off <<= 1) z = maxabs_bf16x2(z, __shfl_xor_sync(0xFFFFFFFFu, z, off));
+        const float sv[2] = {scale_of_amax(fabsf(bf16_lo(z))), scale_of_amax(fabsf(bf16_hi(z)))};
 #pragma unroll
-        for (int i = 0; i < kRowsPerWarp; ++i) {
-            const long long r = row0 + i;
+        for (int p = 0; p < 2; ++p) {
+            const long long r = row0 + p;
             if (r < args.M && group_ok) {
                 float r_lo, r_hi;
-                bracket_rcp(sv[i], r_lo, r_hi);
-                *reinterpret_cast<uint2*>(args.q + r * args.ld_q + col0 + lane * 8) =
-                    codes8(raw[i], sv[i], r_lo, r_hi, sv[i] == 0.0f, !(sv[i] >= 0x1p-125f));
+                bracket_rcp(sv[p], r_lo, r_hi);
+                const bool zero_group = sv[p] == 0.0f, exact_group = !(sv[p] >= 0x1p-125f);
+                const uint2 a = codes8(raw[p][0], sv[p], r_lo, r_hi, zero_group, exact_group);
+                const uint2 b = codes8(raw[p][1], sv[p], r_lo, r_hi, zero_group, exact_group);
+                *reinterpret_cast<uint4*>(args.q + r * args.ld_q + col) = make_uint4(a.x, a.y, b.x, b.y);
             }
         }
-        if ((lane & 15) == 0 && group_ok && row0 < args.M4)
-            *reinterpret_cast<float4*>(args.sfa + group * args.M4 + row0) =
-                make_float4(sv[0], sv[1], sv[2], sv[3]);
+        if ((j & 7) == 0 && group_ok && row0 < args.M4)
+            *reinterpret_cast<float2*>(args.sfa + group * args.M4 + row0) = make_float2(sv[0], sv[1]);
         if (++stage == kQuantStages) {
             stage = 0;
             phase ^= 1u;
