@@ -432,15 +432,16 @@ __device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint3
         for (int c = 0; c < NC; ++c) {
             tmem_ld_async(taddr + C::chunk_col(c), r);
             tmem_wait_ld(r);
-            if (c + 1 == NC) release();
+            if (NC > 1 && c + 1 == NC) release();
             const float2 sc = (C::SILU && c >= NC / 2) ? s2_up : s2;
             promote_chunk<C, X>(acc, r, c * X, slot, sc);
+            // one chunk: release once the FMAs have consumed the scale slot's values
+            if (NC == 1) release();
         }
     } else {
         uint32_t ra[X], rb[X];
         tmem_ld_async(taddr + C::chunk_col(0), ra);
         tmem_wait_ld(ra);
-        if (NC == 1) release();
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
             if (c + 1 < NC) {
@@ -450,6 +451,7 @@ __device__ __forceinline__ void promote_k_block(float2 (&acc)[C::kCW / 2], uint3
             const float2 sc = (C::SILU && c >= NC / 2) ? s2_up : s2;
             if (c & 1) promote_chunk<C, X>(acc, rb, c * X, slot, sc);
             else promote_chunk<C, X>(acc, ra, c * X, slot, sc);
+            if (NC == 1) release();  // after the FMAs that consumed the scale slot's values
             if (c + 1 < NC) {
                 if (c & 1) tmem_wait_ld(ra);
                 else tmem_wait_ld(rb);
@@ -998,10 +1000,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 const float* slot = scale_slots + sstage * C::kScaleSlotFloats + j * C::kScaleKbFloats;
                 const uint32_t taddr = tmem_base + t_lane + static_cast<uint32_t>(abuf * C::BNQ + C::wg_col(wg));
                 // the accumulator slice and the scale slot are only read, and each arrival
-                // follows the completion of those reads: no release fence is needed (one
-                // would also wait for this warp's outstanding output stores).  The slice is
-                // released as soon as its last chunk is in registers, the scale slot after
-                // the last K block of its batch.
+                // follows the completion of those reads: the TMEM loads are waited for, and
+                // the scale values have fed FMAs issued before the arrival.  No release fence
+                // is needed (one would also wait for this warp's outstanding output stores).
+                // The slice is released as soon as its last chunk is in registers (with a
+                // single chunk, after its FMAs), the scale slot after the last K block of its
+                // batch.
                 const uint32_t sempty = sempty_bar(sstage);
                 promote_k_block<C>(acc, taddr, slot, row, wg, [&]() {
                     tc_fence_before();
@@ -1009,7 +1013,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     if (lane == 0) {
                         if constexpr (C::PAIR) mbar_arrive_cluster_relaxed(mapa_shared(tempty_bar(slot_id), 0));
                         else mbar_arrive_relaxed(tempty_bar(slot_id));
-                        // the scales were read before the first TMEM load
+                        // the scale values were consumed by FMAs issued before this arrival
                         if (batch_last) mbar_arrive_relaxed(sempty);
                     }
                 });

@@ -279,8 +279,6 @@ __global__ void __launch_bounds__(kQuantThreads)
             raw[p][0] = *reinterpret_cast<const uint4*>(src + p * kRowBytes);
             raw[p][1] = *reinterpret_cast<const uint4*>(src + p * kRowBytes + 16);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty_bar(stage));
         // each row's largest magnitude over this lane's 16 values (both bf16 halves of
         // m[p] are candidates), then row 0 in the low and row 1 in the high half of one
         // word, reduced over the group's eight lanes; exact throughout
@@ -309,6 +307,13 @@ __global__ void __launch_bounds__(kQuantThreads)
         }
         if ((j & 7) == 0 && group_ok && row0 < args.M4)
             *reinterpret_cast<float2*>(args.sfa + group * args.M4 + row0) = make_float2(sv[0], sv[1]);
+        // The stage goes back to the producer only now: every value this warp read from it
+        // fed the stores above (codes, or through the shuffles the scales), so the reads
+        // have completed, and the release orders them before the next TMA write.  An
+        // arrival straight after the reads let a shared-memory read still queued behind
+        // bank-conflicted ones see the next tile.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(stage));
         if (++stage == kQuantStages) {
             stage = 0;
             phase ^= 1u;
