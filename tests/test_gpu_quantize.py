@@ -221,3 +221,30 @@ def test_zero_rows_write_zero_pad_scales():
 def test_activation_more_ragged_shapes(M, K):
     # K not a multiple of 256 (a half-empty column tile) and row counts off the 32-row tile
     assert_same_a(synthetic.gaussian_bf16((M, K), 1.0, seed=M + K))
+
+
+@pytest.mark.parametrize("M,K", [(8192, 8192), (2048, 12288)])
+def test_activation_quantize_is_repeatable(M, K):
+    # Every launch must write the same bytes, whatever the output buffers held before and
+    # however the launches overlap: a consumer warp that handed a ring stage back before its
+    # shared-memory reads completed would let some groups see the next tile (wrong scales at
+    # places that change from run to run).  Inputs larger than L2 keep the producer ahead of
+    # the consumers; twelve launches per shape, chained as a step chains them.
+    g = torch.Generator(device=DEV)
+    g.manual_seed(M + K)
+    x = (torch.randn((M, K), generator=g, device=DEV)
+         * torch.exp(torch.randn((M, 1), generator=g, device=DEV))).to(torch.bfloat16)
+    M4 = lnq.ceil4(M)
+    ref_q = torch.empty((M, K), dtype=torch.uint8, device=DEV)
+    ref_s = torch.empty((K // 128, M4), dtype=torch.float32, device=DEV)
+    lnq.lnq_quantize_fp8_groups(x, ref_q, ref_s)
+    for fill in (0x00, 0xAB, 0x55, 0xFF):
+        q = torch.full((M, K), fill, dtype=torch.uint8, device=DEV)
+        s = torch.full((K // 128, M4), float(fill), dtype=torch.float32, device=DEV)
+        for _ in range(3):
+            lnq.lnq_quantize_fp8_groups(x, q, s)
+        torch.cuda.synchronize()
+        assert lnq.lnq_get_last_device_error() == 0
+        bad = (q != ref_q).nonzero()
+        assert bad.shape[0] == 0, f"fill {fill:#x}: {bad.shape[0]} codes differ, first {bad[:4].tolist()}"
+        assert torch.equal(s.view(torch.int32), ref_s.view(torch.int32)), f"fill {fill:#x}: scales differ"
